@@ -1,0 +1,346 @@
+"""Pins for the CPU oracle, run without a GPU.
+
+Each test ties an oracle function to something other than itself: numbers
+printed on the pages (fixtures under tests/golden/, each with its source),
+closed forms, invariants, or brute force on tiny inputs written as plain
+Python loops.  A dropped term, a wrong sign, a transposed operand or a wrong
+group index in the oracle fails at least one of them.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+import workloads
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+# ---------------------------------------------------------------------------
+# P1: the 130x70x129 worked example (quantized GEMM case study, section 3)
+# ---------------------------------------------------------------------------
+def test_p1_tiling_counts_match_page():
+    g = _golden("qg_tiling_130x70x129.json")
+    w = workloads.cfg0_gemm_small()
+    assert (w["M"], w["N"], w["K"]) == (g["M"], g["N"], g["K"])
+    A, B = w["A"][:, :w["K"]], w["B"][:, :w["N"]]
+    acc_t, st = oracle.tiled_int8_gemm(A, B, w["za"], w["zb"], w["bias"],
+                                       g["Tm"], g["Tn"], g["Tk"])
+    assert st["tiles_mnk"] == (g["tiles_m"], g["tiles_n"], g["tiles_k"])
+    assert st["tiles"] == g["tiles"]
+    assert st["useful_macs"] == g["useful_macs"]
+    assert st["slots"] == g["slots"]
+    assert round(100 * st["shape_efficiency"], 2) == g["shape_efficiency_percent_approx"]
+    # level 3 of the verification ladder: the tiled model equals the full GEMM
+    acc = oracle.int8_gemm_acc(A, B, w["za"], w["zb"], w["bias"])
+    np.testing.assert_array_equal(acc_t, acc)
+
+
+def test_p1_buffer_budget_matches_page():
+    g = _golden("qg_tiling_130x70x129.json")
+    b = oracle.tile_budget_bytes(g["Tm"], g["Tn"], g["Tk"], g["reserve_bytes"])
+    assert b["S_input"] == g["S_input_bytes"]
+    assert b["S_acc"] == g["S_acc_bytes"]
+    assert b["S_total"] == g["S_total_bytes"]
+
+
+# ---------------------------------------------------------------------------
+# P2: INT32 overflow bound (section 4)
+# ---------------------------------------------------------------------------
+def test_p2_overflow_constants():
+    g = _golden("qg_overflow_bound.json")
+    assert oracle.worst_zp_corrected_magnitude() == g["worst_magnitude"]
+    assert oracle.overflow_bound(1, 0) == g["product_bound"]
+    assert oracle.fits_int32(g["K_safe_example"], 5000)
+    assert oracle.overflow_bound(129, 0) == 129 * 65025 == 8388225
+
+
+def test_p2_extreme_case_reaches_bound_exactly():
+    K = 129
+    A = np.full((2, K), 127, np.int8)
+    B = np.full((K, 3), -128, np.int8)
+    acc = oracle.int8_gemm_acc(A, B, za=-128, zb=127)
+    assert (acc == -K * 65025).all()
+    A2 = np.full((1, K), -128, np.int8)
+    acc2 = oracle.int8_gemm_acc(A2, B, za=127, zb=127)
+    assert (acc2 == K * 65025).all()
+
+
+def test_p2_bound_edge_and_rejection():
+    # 33025*65025 = 2147450625 <= 2^31-1 < 33026*65025 = 2147515650
+    assert oracle.fits_int32(33025, 0)
+    assert not oracle.fits_int32(33026, 0)
+    assert not oracle.fits_int32(33025, 2 ** 31 - 1 - 2147450625 + 1)
+    A = np.zeros((1, 33026), np.int8)
+    B = np.zeros((33026, 1), np.int8)
+    with pytest.raises(OverflowError):
+        oracle.qgemm_s8s8_requant(A, B, 0, 0, None, 2 ** 30, 0, 0, -128, 127)
+
+
+# ---------------------------------------------------------------------------
+# P3: padding stands for real zero (section 2)
+# ---------------------------------------------------------------------------
+def test_p3_zero_point_padding_invariance():
+    w = workloads.cfg0_gemm_small()
+    A, B = w["A"][:, :129], w["B"][:, :70]
+    za, zb = 11, -7        # non-zero on both sides so raw-zero padding is visible
+    acc = oracle.int8_gemm_acc(A, B, za, zb, w["bias"])
+    Ap = np.full((130, 256), za, np.int8); Ap[:, :129] = A
+    Bp = np.full((256, 70), zb, np.int8); Bp[:129] = B
+    np.testing.assert_array_equal(oracle.int8_gemm_acc(Ap, Bp, za, zb, w["bias"]), acc)
+    A0 = np.zeros((130, 256), np.int8); A0[:, :129] = A
+    B0 = np.zeros((256, 70), np.int8); B0[:129] = B
+    assert (oracle.int8_gemm_acc(A0, B0, za, zb, w["bias"]) != acc).any()
+
+
+def _im2col_zp(x, KH, KW, stride, pad, za):
+    Nb, H, W, C = x.shape
+    OH = oracle.conv_out_size(H, KH, stride[0], pad[0])
+    OW = oracle.conv_out_size(W, KW, stride[1], pad[1])
+    xp = np.full((Nb, H + 2 * pad[0], W + 2 * pad[1], C), za, np.int8)
+    xp[:, pad[0]:pad[0] + H, pad[1]:pad[1] + W] = x
+    cols = np.empty((Nb, OH, OW, KH, KW, C), np.int8)
+    for kh in range(KH):
+        for kw in range(KW):
+            cols[:, :, :, kh, kw] = xp[:, kh:kh + stride[0] * OH:stride[0],
+                                       kw:kw + stride[1] * OW:stride[1]]
+    return cols.reshape(Nb * OH * OW, KH * KW * C)
+
+
+def test_p3_conv_equals_zp_padded_im2col_gemm():
+    w = workloads.int8_conv(1, 9, 7, 8, 5, 3, 3, (1, 1), (1, 1), seed=7)
+    acc = oracle.qconv2d_s8_acc(w["x"], w["w"], w["stride"], w["pad"], w["za"], w["bias"])
+    cols = _im2col_zp(w["x"], 3, 3, w["stride"], w["pad"], w["za"])
+    Bm = w["w"].reshape(w["Cout"], -1).T
+    acc2 = oracle.int8_gemm_acc(cols, Bm, w["za"], 0, w["bias"])
+    np.testing.assert_array_equal(acc.reshape(-1, w["Cout"]), acc2)
+    # raw-zero padding would be wrong
+    cols0 = _im2col_zp(w["x"], 3, 3, w["stride"], w["pad"], 0)
+    assert (oracle.int8_gemm_acc(cols0, Bm, w["za"], 0, w["bias"]) != acc2).any()
+
+
+def test_conv_brute_force_loops():
+    rng = np.random.default_rng(3)
+    Nb, H, W, Cin, Cout, KH, KW = 2, 4, 5, 3, 2, 3, 2
+    sh, sw_, ph, pw = 2, 1, 1, 0
+    x = rng.integers(-128, 128, (Nb, H, W, Cin)).astype(np.int8)
+    wt = rng.integers(-127, 128, (Cout, KH, KW, Cin)).astype(np.int8)
+    za = -5
+    bias = rng.integers(-50, 50, Cout).astype(np.int32)
+    OH, OW = (H + 2 * ph - KH) // sh + 1, (W + 2 * pw - KW) // sw_ + 1
+    ref = np.zeros((Nb, OH, OW, Cout), np.int64)
+    for n in range(Nb):
+        for oh in range(OH):
+            for ow in range(OW):
+                for co in range(Cout):
+                    s = int(bias[co])
+                    for kh in range(KH):
+                        for kw in range(KW):
+                            for ci in range(Cin):
+                                ih, iw = oh * sh + kh - ph, ow * sw_ + kw - pw
+                                v = int(x[n, ih, iw, ci]) if (0 <= ih < H and 0 <= iw < W) else za
+                                s += (v - za) * int(wt[co, kh, kw, ci])
+                    ref[n, oh, ow, co] = s
+    got = oracle.qconv2d_s8_acc(x, wt, (sh, sw_), (ph, pw), za, bias)
+    np.testing.assert_array_equal(got, ref)
+
+
+# ---------------------------------------------------------------------------
+# P4: accumulate across K, requantize once (section 4)
+# ---------------------------------------------------------------------------
+def test_p4_k_block_accumulation():
+    w = workloads.cfg0_gemm_small()
+    A, B = w["A"][:, :129], w["B"][:, :70]
+    acc = oracle.int8_gemm_acc(A, B, w["za"], w["zb"])
+    parts = [oracle.int8_gemm_acc(A[:, k:k + 32], B[k:k + 32], w["za"], w["zb"])
+             for k in range(0, 129, 32)]
+    np.testing.assert_array_equal(sum(parts), acc)
+    m0, sh = oracle.requant_params(float(w["ratio"][0]))
+    once = oracle.rq_round(acc, m0, sh)
+    # requantizing every block partial changes the result somewhere
+    m0b, shb = oracle.requant_params(0.37)
+    y1 = oracle.requantize(acc, m0b, shb, 0, -128, 127).astype(np.int64)
+    y2 = sum(oracle.requantize(p, m0b, shb, 0, -128, 127).astype(np.int64) for p in parts)
+    assert (np.clip(y2, -128, 127) != y1).any()
+    assert once.shape == acc.shape
+
+
+# ---------------------------------------------------------------------------
+# P5: brute force (pure Python loops) and float dequant reference
+# ---------------------------------------------------------------------------
+def test_p5_gemm_brute_force_loops():
+    rng = np.random.default_rng(11)
+    M, N, K = 3, 4, 5
+    A = rng.integers(-128, 128, (M, K)).astype(np.int8)
+    B = rng.integers(-128, 128, (K, N)).astype(np.int8)
+    za, zb = -17, 9
+    bias = rng.integers(-5000, 5001, N).astype(np.int32)
+    ref = [[int(bias[n]) + sum((int(A[m, k]) - za) * (int(B[k, n]) - zb) for k in range(K))
+            for n in range(N)] for m in range(M)]
+    np.testing.assert_array_equal(oracle.int8_gemm_acc(A, B, za, zb, bias), np.array(ref))
+
+
+def test_p5_float_dequant_reference():
+    w = workloads.int8_gemm(37, 23, 129, seed=5)
+    A, B = w["A"], w["B"]
+    rng = np.random.default_rng(1)
+    sA = 0.02
+    sB = rng.uniform(1e-3, 1e-1, w["N"])
+    acc = oracle.int8_gemm_acc(A, B, w["za"], w["zb"])
+    real = (sA * (A.astype(np.float64) - w["za"])) @ (sB[None, :] * (B.astype(np.float64) - w["zb"]))
+    np.testing.assert_allclose(sA * sB[None, :] * acc, real, rtol=1e-12, atol=1e-9)
+
+
+def test_p5_requant_within_one_lsb_of_real_ratio():
+    rng = np.random.default_rng(2)
+    acc = rng.integers(-2 ** 24, 2 ** 24, 20000)
+    worst, mism = 0, 0
+    for ratio in np.exp(rng.uniform(np.log(1e-6), np.log(0.99), 50)):
+        m0, sh = oracle.requant_params(ratio)
+        y = oracle.rq_round(acc, m0, sh)
+        ref = np.rint(acc * ratio).astype(np.int64)
+        d = np.abs(y - ref)
+        worst = max(worst, int(d.max()))
+        mism += int((d != 0).sum())
+    assert worst <= 1
+    assert mism < 0.01 * 50 * 20000
+
+
+def test_requant_params_closed_forms():
+    assert oracle.requant_params(0.5) == (2 ** 30, 0)
+    assert oracle.requant_params(0.25) == (2 ** 30, 1)
+    assert oracle.requant_params(2.0 ** -10) == (2 ** 30, 9)
+    assert oracle.requant_params(0.75) == (3 * 2 ** 29, 0)
+    rng = np.random.default_rng(4)
+    for r in np.exp(rng.uniform(np.log(1e-9), np.log(0.999), 200)):
+        m0, sh = oracle.requant_params(r)
+        assert 2 ** 30 <= m0 < 2 ** 31
+        assert abs(m0 * 2.0 ** -(31 + sh) - r) <= 2.0 ** -(32 + sh)
+    for bad in (0.0, 1.0, 1.5, -0.1, 1e-12):
+        with pytest.raises(ValueError):
+            oracle.requant_params(bad)
+
+
+def test_requant_round_half_even_cases():
+    m0, sh = oracle.requant_params(0.5)            # divides by exactly 2
+    acc = np.array([3, 5, 7, -3, -5, -7, 1, -1, 4])
+    y = oracle.requantize(acc, m0, sh, 0, -128, 127)
+    np.testing.assert_array_equal(y, [2, 2, 4, -2, -2, -4, 0, 0, 2])
+    y = oracle.requantize(np.array([1000, -1000]), m0, sh, 3, -128, 127)
+    np.testing.assert_array_equal(y, [127, -128])   # saturating clamp
+    y = oracle.requantize(np.array([-40, 40]), m0, sh, -10, -10, 127)
+    np.testing.assert_array_equal(y, [-10, 10])     # ReLU floor at the out zero-point
+
+
+# ---------------------------------------------------------------------------
+# P6: dynamic activation quantization specials
+# ---------------------------------------------------------------------------
+def test_p6_quantization_specials():
+    for case in _golden("qg_dynamic_quant_specials.json")["cases"]:
+        q, s, z = oracle.quantize_rows_a8(np.array([case["x"]], np.float32))
+        assert s[0] == np.float32(case["scale"])
+        assert z[0] == case["zp"]
+        np.testing.assert_array_equal(q[0], case["q"])
+
+
+def test_p6_constant_row_and_error_bound():
+    q, s, z = oracle.quantize_rows_a8(np.full((1, 10), 1.0, np.float32))
+    assert z[0] == -128 and (q == 127).all()
+    x = np.random.default_rng(9).standard_normal((16, 333)).astype(np.float32) * 3
+    q, s, z = oracle.quantize_rows_a8(x)
+    assert (s > 0).all()
+    # real 0.0 is exactly representable: it maps to the zero-point
+    xz = np.concatenate([x[:, :5], np.zeros((16, 1), np.float32)], 1)
+    q0, _, z0 = oracle.quantize_rows_a8(xz)
+    np.testing.assert_array_equal(q0[:, -1], z0)
+    err = np.abs(oracle.dequantize_rows(q, s, z) - x.astype(np.float64))
+    assert (err <= 0.5 * s[:, None] * (1 + 1e-5)).all()
+    # each row reaches an end of the code range at its extreme value
+    assert ((q.min(1) == -128) | (q.max(1) == 127)).all()
+
+
+def test_p6_grid_exact_round_trip():
+    rng = np.random.default_rng(12)
+    zp = -40
+    s = np.float32(0.125)                 # power of two: exact arithmetic
+    codes = rng.integers(-128, 128, (1, 300))
+    codes[0, 0], codes[0, 1] = -128, 127  # pin the range so min/max give s, zp
+    x = ((codes - zp) * s).astype(np.float32)
+    q, sc, z = oracle.quantize_rows_a8(x)
+    assert sc[0] == s and z[0] == zp
+    np.testing.assert_array_equal(q[0], codes[0])
+
+
+# ---------------------------------------------------------------------------
+# P7: A8W4 special case and brute force
+# ---------------------------------------------------------------------------
+def test_p7_a8w4_integer_special_case():
+    rng = np.random.default_rng(21)
+    N, K = 40, 128
+    x = rng.integers(-100, 156, (1, K)).astype(np.float32)
+    x[0, 0], x[0, 1] = -100, 155          # scale (155+100)/255 = 1 exactly
+    qw = rng.integers(-8, 8, (N, K)).astype(np.int8)
+    sw = np.ones((N, K // 32), np.float32)
+    bias = rng.integers(-9, 10, N).astype(np.float32)
+    y, q, s, z = oracle.qgemm_a8w4_f32(x, qw, sw, bias, -np.inf, np.inf)
+    assert s[0] == 1.0 and z[0] == -28
+    exact = qw.astype(np.int64) @ x[0].astype(np.int64) + bias.astype(np.int64)
+    np.testing.assert_array_equal(y[0], exact.astype(np.float32))
+
+
+def test_p7_a8w4_brute_force_loops():
+    rng = np.random.default_rng(22)
+    M, N, K = 2, 3, 64
+    x = rng.standard_normal((M, K)).astype(np.float32)
+    qw = rng.integers(-8, 8, (N, K)).astype(np.int8)
+    sw = rng.uniform(0.01, 0.1, (N, K // 32)).astype(np.float32)
+    bias = rng.normal(0, 0.1, N).astype(np.float32)
+    y, q, s, z = oracle.qgemm_a8w4_f32(x, qw, sw, bias, -0.5, 0.5)
+    for m in range(M):
+        for n in range(N):
+            t = float(bias[n])
+            for k in range(K):
+                t += float(s[m]) * (int(q[m, k]) - int(z[m])) * float(sw[n, k // 32]) * int(qw[n, k])
+            assert abs(float(y[m, n]) - min(max(t, -0.5), 0.5)) <= 1e-6 * max(1.0, abs(t))
+
+
+def test_p7_a8w4_float_reference():
+    w = workloads.a8w4(3, 50, 256, seed=8, clamp=(-np.inf, np.inf))
+    y, q, s, z = oracle.qgemm_a8w4_f32(w["x"], w["qw"], w["sw"], w["bias"], -np.inf, np.inf)
+    xa = oracle.dequantize_rows(q, s, z)
+    wd = np.repeat(w["sw"].astype(np.float64), 32, axis=1) * w["qw"]
+    ref = xa @ wd.T + w["bias"].astype(np.float64)
+    np.testing.assert_allclose(y, ref, rtol=1e-6, atol=1e-6)
+    # and the quantized activations approximate x to within half a step
+    assert (np.abs(xa - w["x"]) <= 0.5 * s[:, None] * (1 + 1e-5)).all()
+
+
+# ---------------------------------------------------------------------------
+# P8: W4 packed layout (this library's own format, reading R6)
+# ---------------------------------------------------------------------------
+def test_p8_w4_pack_round_trip_and_bytes():
+    w = workloads.a8w4(1, 7, 96, seed=9)
+    packed = oracle.pack_w4_g32(w["qw"], w["sw"])
+    assert packed.size == oracle.pack_w4_g32_bytes(7, 96)
+    qw2, sw2 = oracle.unpack_w4_g32(packed, 7, 96)
+    np.testing.assert_array_equal(qw2, w["qw"])
+    np.testing.assert_array_equal(sw2, w["sw"])
+    # hand-derived pattern: q[k] = (k % 16) - 8 -> nibble value k % 16
+    qw = ((np.arange(32) % 16) - 8).astype(np.int8)[None, :]
+    p = oracle.pack_w4_g32(qw, np.ones((1, 1), np.float32))
+    # word j covers k = 8j..8j+7: low nibble of byte b = k0+b, high = k0+4+b
+    expect = []
+    for j in range(4):
+        for b in range(4):
+            lo, hi = (8 * j + b) % 16, (8 * j + 4 + b) % 16
+            expect.append(lo | (hi << 4))
+    np.testing.assert_array_equal(p[:16], expect)
+    assert p[16:20].view(np.float32)[0] == 1.0
