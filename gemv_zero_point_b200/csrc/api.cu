@@ -1,0 +1,378 @@
+// C ABI entry points: argument checks, workspace layout, dispatch to the
+// kernels, status codes and the per-device status word.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "qg_internal.cuh"
+
+namespace qg {
+
+// ---- kernels implemented in the other translation units ----
+int launch_quantize_rows(int M, int K, const float* x, int64_t ldx, int8_t* q, int64_t ldq,
+                         float* scale, int32_t* zp, cudaStream_t st);
+int launch_pack_w4(int N, int K, const int8_t* w, int64_t ldw, const float* sw, void* packed,
+                   cudaStream_t st);
+int launch_a8w4_gemv(int N, int K, const float* x, const void* packed, const float* bias,
+                     float lo, float hi, float* y, int8_t* q_out, float* scale_out,
+                     int32_t* zp_out, cudaStream_t st);
+int launch_a8w4_gemm_simt(int M, int N, int K, const int8_t* q, const float* sA,
+                          const int32_t* zA, const void* packed, const float* bias, float lo,
+                          float hi, float* y, int64_t ldy, cudaStream_t st);
+int setup_a8w4_gemv();
+int setup_a8w4_gemm_simt();
+int i8gemm_setup();
+
+int i8gemm_pack_b(int K, int N, const int8_t* B, int64_t ldb, void* packed, cudaStream_t st);
+size_t i8gemm_pack_b_bytes(int K, int N);
+size_t i8gemm_packed_workspace_bytes(int M, int K);
+int i8gemm_run_packed(int M, int N, int K, const int8_t* A, int64_t lda, const void* packed_b,
+                      int8_t* C, int64_t ldc, const qg_requant_t& rq, int32_t* acc_out,
+                      int64_t ld_acc, void* ws, size_t ws_bytes, cudaStream_t st);
+size_t conv_workspace_bytes(int Nb, int H, int W, int Cin, int Cout, int KH, int KW, int sh,
+                            int sw, int ph, int pw);
+int conv_run(int Nb, int H, int W, int Cin, int Cout, int KH, int KW, int sh, int sw, int ph,
+             int pw, const int8_t* x, const int8_t* w, int8_t* y, const qg_requant_t& rq,
+             int32_t* acc_out, void* ws, size_t ws_bytes, cudaStream_t st);
+
+// ---- per-device state ----
+static __device__ int g_status_word;
+
+namespace {
+constexpr int kMaxDevices = 64;
+struct DeviceState {
+  bool ready = false;
+  int sms = 0;
+  int* status = nullptr;
+  int setup_rc = QG_OK;
+};
+DeviceState g_dev[kMaxDevices];
+std::mutex g_mu;
+
+DeviceState* current_state() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  DeviceState& s = g_dev[dev];
+  if (s.ready) return &s;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!s.ready) {
+    int major = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&s.sms, cudaDevAttrMultiProcessorCount, dev);
+    void* p = nullptr;
+    if (major != 10 || cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) {
+      cudaGetLastError();
+      s.setup_rc = QG_ERR_NO_DEVICE;
+    } else {
+      s.status = static_cast<int*>(p);
+      int rc = setup_a8w4_gemv();
+      if (rc == QG_OK) rc = setup_a8w4_gemm_simt();
+      if (rc == QG_OK) rc = i8gemm_setup();
+      s.setup_rc = rc;
+    }
+    s.ready = true;
+  }
+  return &s;
+}
+}  // namespace
+
+int* status_word() {
+  DeviceState* s = current_state();
+  return s ? s->status : nullptr;
+}
+
+int num_sms() {
+  DeviceState* s = current_state();
+  return (s && s->sms > 0) ? s->sms : 148;
+}
+
+static int device_ready() {
+  DeviceState* s = current_state();
+  if (!s) return QG_ERR_NO_DEVICE;
+  return s->setup_rc;
+}
+
+}  // namespace qg
+
+using namespace qg;
+
+// ---------------------------------------------------------------------------
+// Status helpers
+// ---------------------------------------------------------------------------
+extern "C" const char* qg_status_string(int status) {
+  switch (status) {
+    case QG_OK: return "QG_OK";
+    case QG_ERR_INVALID_ARG: return "QG_ERR_INVALID_ARG: invalid argument";
+    case QG_ERR_MISALIGNED: return "QG_ERR_MISALIGNED: pointer alignment not met";
+    case QG_ERR_OVERFLOW_BOUND: return "QG_ERR_OVERFLOW_BOUND: K*65025 + |bias| exceeds INT32_MAX";
+    case QG_ERR_UNSUPPORTED: return "QG_ERR_UNSUPPORTED: parameters not supported";
+    case QG_ERR_CUDA: return "QG_ERR_CUDA: CUDA runtime or launch error";
+    case QG_ERR_TIMEOUT: return "QG_ERR_TIMEOUT: a bounded device-side wait ran out";
+    case QG_ERR_WORKSPACE: return "QG_ERR_WORKSPACE: workspace missing or too small";
+    case QG_ERR_NO_DEVICE: return "QG_ERR_NO_DEVICE: no sm_100 device is current";
+    default: return "QG_ERR_UNKNOWN";
+  }
+}
+
+extern "C" int qg_version(void) { return QG_API_VERSION; }
+
+extern "C" int qg_device_status(int reset) {
+  int rc = device_ready();
+  if (rc != QG_OK) return rc;
+  if (cudaDeviceSynchronize() != cudaSuccess) return QG_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, status_word(), sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return QG_ERR_CUDA;
+  if (reset && v != 0) {
+    if (cudaMemset(status_word(), 0, sizeof(int)) != cudaSuccess) return QG_ERR_CUDA;
+  }
+  return v;
+}
+
+extern "C" int qg_requant_params(double ratio, int32_t* m0, int32_t* shift) {
+  if (!m0 || !shift) return QG_ERR_INVALID_ARG;
+  if (!(ratio > 0.0 && ratio < 1.0) || !isfinite(ratio)) return QG_ERR_UNSUPPORTED;
+  int e = 0;
+  double f = frexp(ratio, &e);           // ratio = f * 2^e, f in [0.5, 1)
+  int64_t q = (int64_t)floor(f * 2147483648.0 + 0.5);  // f*2^31 is exact
+  if (q == (int64_t)1 << 31) {
+    q >>= 1;
+    e += 1;
+  }
+  const int s = -e;
+  if (s < 0 || s > 31) return QG_ERR_UNSUPPORTED;
+  *m0 = (int32_t)q;
+  *shift = s;
+  return QG_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Argument checks shared by the INT8 entry points
+// ---------------------------------------------------------------------------
+static bool aligned(const void* p, uintptr_t a) { return ((uintptr_t)p & (a - 1)) == 0; }
+
+static int check_requant(const qg_requant_t* rq, int K) {
+  if (!rq) return QG_ERR_INVALID_ARG;
+  if (rq->a_zero_point < -128 || rq->a_zero_point > 127) return QG_ERR_INVALID_ARG;
+  if (rq->b_zero_point < -128 || rq->b_zero_point > 127) return QG_ERR_INVALID_ARG;
+  if (rq->out_zero_point < -128 || rq->out_zero_point > 127) return QG_ERR_INVALID_ARG;
+  if (rq->clamp_min < -128 || rq->clamp_max > 127 || rq->clamp_min > rq->clamp_max)
+    return QG_ERR_INVALID_ARG;
+  if (rq->per_channel) {
+    if (!rq->multiplier || !rq->shift) return QG_ERR_INVALID_ARG;
+  } else {
+    if (rq->multiplier0 < 0 || rq->shift0 < 0 || rq->shift0 > 31) return QG_ERR_INVALID_ARG;
+  }
+  if (rq->bias && rq->bias_abs_max < 0) return QG_ERR_INVALID_ARG;
+  // [QG] section 4: K*65025 + |bias| must fit INT32
+  const int64_t bound = (int64_t)K * 65025 + (rq->bias ? (int64_t)rq->bias_abs_max : 0);
+  if (bound > (int64_t)INT32_MAX) return QG_ERR_OVERFLOW_BOUND;
+  return QG_OK;
+}
+
+// ---------------------------------------------------------------------------
+// INT8 GEMM
+// ---------------------------------------------------------------------------
+extern "C" size_t qgemm_pack_b_s8_bytes(int K, int N) {
+  if (K <= 0 || N <= 0) return 0;
+  return i8gemm_pack_b_bytes(K, N);
+}
+
+extern "C" int qgemm_pack_b_s8(int K, int N, const int8_t* B, int64_t ldb, void* packed_b,
+                               size_t packed_bytes, void* stream) {
+  if (K <= 0 || N <= 0 || !B || !packed_b || ldb < N) return QG_ERR_INVALID_ARG;
+  if (!aligned(packed_b, 128)) return QG_ERR_MISALIGNED;
+  if (packed_bytes < i8gemm_pack_b_bytes(K, N)) return QG_ERR_WORKSPACE;
+  int rc = device_ready();
+  if (rc != QG_OK) return rc;
+  return i8gemm_pack_b(K, N, B, ldb, packed_b, (cudaStream_t)stream);
+}
+
+extern "C" size_t qgemm_s8s8_packed_workspace_bytes(int M, int K) {
+  if (M <= 0 || K <= 0) return 0;
+  return i8gemm_packed_workspace_bytes(M, K);
+}
+
+extern "C" size_t qgemm_s8s8_workspace_bytes(int M, int N, int K) {
+  if (M <= 0 || N <= 0 || K <= 0) return 0;
+  return round_up(i8gemm_pack_b_bytes(K, N), 256) + i8gemm_packed_workspace_bytes(M, K);
+}
+
+static int check_gemm_args(int M, int N, int K, const int8_t* A, int64_t lda, int8_t* C,
+                           int64_t ldc, const qg_requant_t* rq, int32_t* acc_out,
+                           int64_t ld_acc) {
+  if (M < 0 || N <= 0 || K <= 0) return QG_ERR_INVALID_ARG;
+  if (M > 0 && (!A || !C)) return QG_ERR_INVALID_ARG;
+  if (lda < K || ldc < N) return QG_ERR_INVALID_ARG;
+  if (acc_out && ld_acc < N) return QG_ERR_INVALID_ARG;
+  if (acc_out && !aligned(acc_out, 4)) return QG_ERR_MISALIGNED;
+  return check_requant(rq, K);
+}
+
+extern "C" int qgemm_s8s8_requant_packed(int M, int N, int K, const int8_t* A, int64_t lda,
+                                         const void* packed_b, int8_t* C, int64_t ldc,
+                                         const qg_requant_t* rq, int32_t* acc_out,
+                                         int64_t ld_acc, void* workspace,
+                                         size_t workspace_bytes, void* stream) {
+  int rc = check_gemm_args(M, N, K, A, lda, C, ldc, rq, acc_out, ld_acc);
+  if (rc != QG_OK) return rc;
+  if (!packed_b) return QG_ERR_INVALID_ARG;
+  if (!aligned(packed_b, 128)) return QG_ERR_MISALIGNED;
+  if (workspace && !aligned(workspace, 256)) return QG_ERR_MISALIGNED;
+  if (M == 0) return QG_OK;
+  rc = device_ready();
+  if (rc != QG_OK) return rc;
+  return i8gemm_run_packed(M, N, K, A, lda, packed_b, C, ldc, *rq, acc_out, ld_acc, workspace,
+                           workspace_bytes, (cudaStream_t)stream);
+}
+
+extern "C" int qgemm_s8s8_requant(int M, int N, int K, const int8_t* A, int64_t lda,
+                                  const int8_t* B, int64_t ldb, int8_t* C, int64_t ldc,
+                                  const qg_requant_t* rq, int32_t* acc_out, int64_t ld_acc,
+                                  void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = check_gemm_args(M, N, K, A, lda, C, ldc, rq, acc_out, ld_acc);
+  if (rc != QG_OK) return rc;
+  if (!B || ldb < N) return QG_ERR_INVALID_ARG;
+  if (M == 0) return QG_OK;
+  if (!workspace) return QG_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return QG_ERR_MISALIGNED;
+  const size_t pb = round_up(i8gemm_pack_b_bytes(K, N), 256);
+  if (workspace_bytes < pb + i8gemm_packed_workspace_bytes(M, K)) return QG_ERR_WORKSPACE;
+  rc = device_ready();
+  if (rc != QG_OK) return rc;
+  cudaStream_t st = (cudaStream_t)stream;
+  rc = i8gemm_pack_b(K, N, B, ldb, workspace, st);
+  if (rc != QG_OK) return rc;
+  return i8gemm_run_packed(M, N, K, A, lda, workspace, C, ldc, *rq, acc_out, ld_acc,
+                           (char*)workspace + pb, workspace_bytes - pb, st);
+}
+
+// ---------------------------------------------------------------------------
+// INT8 convolution
+// ---------------------------------------------------------------------------
+extern "C" size_t qconv2d_s8_workspace_bytes(int Nb, int H, int W, int Cin, int Cout, int KH,
+                                             int KW, int stride_h, int stride_w, int pad_h,
+                                             int pad_w) {
+  if (Nb <= 0 || H <= 0 || W <= 0 || Cin <= 0 || Cout <= 0 || KH <= 0 || KW <= 0 ||
+      stride_h <= 0 || stride_w <= 0 || pad_h < 0 || pad_w < 0)
+    return 0;
+  return conv_workspace_bytes(Nb, H, W, Cin, Cout, KH, KW, stride_h, stride_w, pad_h, pad_w);
+}
+
+extern "C" int qconv2d_s8_im2col(int Nb, int H, int W, int Cin, int Cout, int KH, int KW,
+                                 int stride_h, int stride_w, int pad_h, int pad_w,
+                                 const int8_t* x, const int8_t* w, int8_t* y,
+                                 const qg_requant_t* rq, int32_t* acc_out, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+  if (Nb <= 0 || H <= 0 || W <= 0 || Cin <= 0 || Cout <= 0 || KH <= 0 || KW <= 0 ||
+      stride_h <= 0 || stride_w <= 0 || pad_h < 0 || pad_w < 0)
+    return QG_ERR_INVALID_ARG;
+  if (!x || !w || !y) return QG_ERR_INVALID_ARG;
+  if (H + 2 * pad_h < KH || W + 2 * pad_w < KW) return QG_ERR_INVALID_ARG;
+  if (pad_h >= KH || pad_w >= KW) return QG_ERR_UNSUPPORTED;
+  const int64_t K = (int64_t)KH * KW * Cin;
+  if (K > INT32_MAX) return QG_ERR_INVALID_ARG;
+  int rc = check_requant(rq, (int)K);
+  if (rc != QG_OK) return rc;
+  if (rq->b_zero_point != 0) return QG_ERR_UNSUPPORTED;
+  if (acc_out && !aligned(acc_out, 4)) return QG_ERR_MISALIGNED;
+  if (workspace && !aligned(workspace, 256)) return QG_ERR_MISALIGNED;
+  const size_t need =
+      conv_workspace_bytes(Nb, H, W, Cin, Cout, KH, KW, stride_h, stride_w, pad_h, pad_w);
+  if (need && (!workspace || workspace_bytes < need)) return QG_ERR_WORKSPACE;
+  rc = device_ready();
+  if (rc != QG_OK) return rc;
+  return conv_run(Nb, H, W, Cin, Cout, KH, KW, stride_h, stride_w, pad_h, pad_w, x, w, y, *rq,
+                  acc_out, workspace, workspace_bytes, (cudaStream_t)stream);
+}
+
+// ---------------------------------------------------------------------------
+// Dynamic activation quantization, W4 pack, A8W4 linear
+// ---------------------------------------------------------------------------
+extern "C" int quantize_rows_a8(int M, int K, const float* x, int64_t ldx, int8_t* q,
+                                int64_t ldq, float* scale, int32_t* zero_point, void* stream) {
+  if (M < 0 || K <= 0 || ldx < K || ldq < K) return QG_ERR_INVALID_ARG;
+  if (M == 0) return QG_OK;
+  if (!x || !q || !scale || !zero_point) return QG_ERR_INVALID_ARG;
+  if (!aligned(x, 4) || !aligned(scale, 4) || !aligned(zero_point, 4)) return QG_ERR_MISALIGNED;
+  int rc = device_ready();
+  if (rc != QG_OK) return rc;
+  return launch_quantize_rows(M, K, x, ldx, q, ldq, scale, zero_point, (cudaStream_t)stream);
+}
+
+extern "C" size_t pack_w4_g32_bytes(int N, int K) {
+  if (N <= 0 || K <= 0 || K % 32) return 0;
+  return (size_t)N * (K / 2) + (size_t)N * (K / 32) * 4;
+}
+
+extern "C" int pack_w4_g32(int N, int K, const int8_t* w, int64_t ldw, const float* group_scales,
+                           void* packed, size_t packed_bytes, void* stream) {
+  if (N <= 0 || K <= 0 || ldw < K || !w || !group_scales || !packed) return QG_ERR_INVALID_ARG;
+  if (K % 32) return QG_ERR_UNSUPPORTED;
+  if (!aligned(packed, 16) || !aligned(group_scales, 4)) return QG_ERR_MISALIGNED;
+  if (packed_bytes < pack_w4_g32_bytes(N, K)) return QG_ERR_WORKSPACE;
+  int rc = device_ready();
+  if (rc != QG_OK) return rc;
+  return launch_pack_w4(N, K, w, ldw, group_scales, packed, (cudaStream_t)stream);
+}
+
+static const int kFusedGemvMaxK = 65536;   // activations held in shared memory
+static const int kSimtMaxK = 25600;        // 8 rows of activations in shared memory
+
+static size_t a8w4_ws_layout(int M, int K, size_t* off_scale, size_t* off_zp) {
+  const size_t q = round_up((int64_t)M * K, 256);
+  const size_t s = round_up((int64_t)M * 4, 256);
+  if (off_scale) *off_scale = q;
+  if (off_zp) *off_zp = q + s;
+  return q + s + round_up((int64_t)M * 4, 256);
+}
+
+extern "C" size_t qgemm_a8w4_workspace_bytes(int M, int K) {
+  if (M <= 0 || K <= 0) return 0;
+  if (M == 1 && K <= kFusedGemvMaxK) return 0;
+  return a8w4_ws_layout(M, K, nullptr, nullptr);
+}
+
+extern "C" int qgemm_a8w4_f32(int M, int N, int K, const float* x, int64_t ldx,
+                              const void* packed_w, const float* bias, float clamp_min,
+                              float clamp_max, float* y, int64_t ldy, int8_t* q_out,
+                              float* scale_out, int32_t* zp_out, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  if (M < 0 || N <= 0 || K <= 0 || ldx < K || ldy < N) return QG_ERR_INVALID_ARG;
+  if (K % 32) return QG_ERR_UNSUPPORTED;
+  if (!(clamp_min <= clamp_max)) return QG_ERR_INVALID_ARG;  // also rejects NaN
+  if (M == 0) return QG_OK;
+  if (!x || !packed_w || !y) return QG_ERR_INVALID_ARG;
+  if (!aligned(packed_w, 16)) return QG_ERR_MISALIGNED;
+  if (!aligned(x, 4) || !aligned(y, 4) || (bias && !aligned(bias, 4))) return QG_ERR_MISALIGNED;
+  if ((scale_out && !aligned(scale_out, 4)) || (zp_out && !aligned(zp_out, 4)))
+    return QG_ERR_MISALIGNED;
+  int rc = device_ready();
+  if (rc != QG_OK) return rc;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (M == 1 && K <= kFusedGemvMaxK)
+    return launch_a8w4_gemv(N, K, x, packed_w, bias, clamp_min, clamp_max, y, q_out, scale_out,
+                            zp_out, st);
+  if (K > kSimtMaxK) return QG_ERR_UNSUPPORTED;
+  size_t off_s = 0, off_z = 0;
+  const size_t need = a8w4_ws_layout(M, K, &off_s, &off_z);
+  if (!workspace || workspace_bytes < need) return QG_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return QG_ERR_MISALIGNED;
+  int8_t* q = (int8_t*)workspace;
+  float* sA = (float*)((char*)workspace + off_s);
+  int32_t* zA = (int32_t*)((char*)workspace + off_z);
+  rc = launch_quantize_rows(M, K, x, ldx, q, K, sA, zA, st);
+  if (rc != QG_OK) return rc;
+  if (q_out && cudaMemcpyAsync(q_out, q, (size_t)M * K, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    return QG_ERR_CUDA;
+  if (scale_out &&
+      cudaMemcpyAsync(scale_out, sA, (size_t)M * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    return QG_ERR_CUDA;
+  if (zp_out && cudaMemcpyAsync(zp_out, zA, (size_t)M * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    return QG_ERR_CUDA;
+  return launch_a8w4_gemm_simt(M, N, K, q, sA, zA, packed_w, bias, clamp_min, clamp_max, y, ldy,
+                               st);
+}

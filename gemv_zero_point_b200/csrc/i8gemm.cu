@@ -1,0 +1,612 @@
+// Affine INT8 GEMM on the 5th-generation tensor cores (tcgen05, kind::i8)
+// with the zero-point correction, bias, fixed-point requantization and clamp
+// fused into the epilogue; the INT8 convolution runs through the same kernel.
+//
+// Sources: xidianedu "量化 GEMM：数值契约、SRAM、DMA 与结果验证" section 1
+// (affine contract, int32 bias in accumulator scale, integer multiplier and
+// shift), section 2 (padding stands for real zero; logical vs physical
+// shape), section 4 (INT32 accumulator zeroed at the first K block, kept
+// across all of K, post-processing once after the last block), section 5
+// (element strides vs byte strides in copy descriptors; a double-buffer slot
+// is overwritten only after its last read); MNN ConvInt8TiledExecutor.cpp
+// (reorderWeight with per-column kernel sums; im2col padded with the input
+// zero-point; QuanPostTreatParameters clamp bounds).
+//
+// Expanded form of the accumulator computed here (exact in int32 under the
+// overflow bound the API enforces):
+//   acc[m,n] = S[m,n] - za*colsum[n] - zb*rowsum[m] + K*za*zb + bias[n]
+//   S = sum_k A[m,k]*B[k,n] (tensor cores), colsum[n] = sum_k B[k,n],
+//   rowsum[m] = sum_k A[m,k].
+// Padding of B beyond K is zero, so the padded K positions add nothing to S,
+// colsum or rowsum whatever A holds there.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+#include <stdint.h>
+
+#include "qg_internal.cuh"
+
+namespace qg {
+
+namespace {
+
+constexpr int BM = 128;          // tile rows (TMEM lanes)
+constexpr int BN = 256;          // tile columns (TMEM columns per accumulator)
+constexpr int BK = 128;          // bytes of K per pipeline stage (one 128B swizzle atom)
+constexpr int STAGES = 4;
+constexpr int A_STAGE = BM * BK;  // 16 KiB
+constexpr int B_STAGE = BN * BK;  // 32 KiB
+constexpr int TMEM_COLS = 2 * BN; // double-buffered accumulator
+constexpr int THREADS = 192;      // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
+constexpr size_t SMEM_BYTES = 1024 /*align slack*/ + STAGES * (A_STAGE + B_STAGE) + 4096;
+
+// Instruction descriptor for kind::i8: D s32, A s8, B s8, both K-major,
+// N = BN, M = BM.
+constexpr uint32_t IDESC = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                           ((uint32_t)(BM >> 4) << 24);
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
+// 1024 bytes apart (sm_100 descriptor version 1).
+__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr) {
+  uint64_t d = (uint64_t)((saddr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)1 << 16;            // leading byte offset (unused with 128B swizzle)
+  d |= (uint64_t)(1024 >> 4) << 32;  // stride byte offset between 8-row groups
+  d |= (uint64_t)1 << 46;            // descriptor version
+  d |= (uint64_t)2 << 61;            // SWIZZLE_128B
+  return d;
+}
+
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   smem_u32(dst)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void mma_i8(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(IDESC), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void epi_bar_sync() {
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+// Barrier over the 128 epilogue threads that also ANDs a predicate, so every
+// epilogue thread takes the same decision after a bounded wait.
+__device__ __forceinline__ bool epi_bar_and(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, 1, 128, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v)
+      : "memory");
+  return r != 0;
+}
+
+// y = clamp(zo + rne(acc*M0 / 2^(31+sh)), lo, hi).  With p = acc*M0 and
+// s = 31+sh: rne(p/2^s) = (p + 2^(s-1) - 1 + ((p >> s) & 1)) >> s.
+__device__ __forceinline__ int requant1(int acc, int m0, int sh, int zo, int lo, int hi) {
+  const int s = 31 + sh;
+  const long long p = (long long)acc * (long long)m0;
+  const long long q = (p + ((1LL << (s - 1)) - 1) + ((p >> s) & 1)) >> s;
+  long long v = q + zo;
+  v = v < lo ? lo : (v > hi ? hi : v);
+  return (int)v;
+}
+
+struct EpiArgs {
+  int M, N, K;
+  int za, zb, zo, lo, hi;
+  const int32_t* colsum;   // [>= N]
+  const int32_t* rowsum;   // [M] or NULL (zb == 0)
+  const int32_t* bias;     // [N] or NULL
+  int per_channel, m0, sh;
+  const int32_t* m0v;      // [N] when per_channel
+  const int32_t* shv;
+  int8_t* C;
+  int64_t ldc;
+  int32_t* acc_out;
+  int64_t ld_acc;
+};
+
+__global__ void __launch_bounds__(THREADS, 1)
+    i8gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     int num_kb, int tiles_m, int tiles_n, EpiArgs ep, int* status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * A_STAGE;
+  uint64_t* full = (uint64_t*)(sB + STAGES * B_STAGE);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint32_t* tmem_slot = (uint32_t*)(tempty + 2);
+  int32_t* c_term = (int32_t*)(tmem_slot + 4);  // [BN] per-column constant
+  int32_t* c_m0 = c_term + BN;                   // [BN]
+  int32_t* c_sh = c_m0 + BN;                     // [BN]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tiles = tiles_m * tiles_n;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 4);
+    }
+    fence_mbar_init();
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------- TMA producer -------------------------
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
+        const int tm = t % tiles_m, tn = t / tiles_m;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, status)) goto producer_done;
+          mbar_arrive_expect_tx(&full[stage], A_STAGE + B_STAGE);
+          tma_load_2d(sA + stage * A_STAGE, &tmA, kb * BK, tm * BM, &full[stage]);
+          tma_load_2d(sB + stage * B_STAGE, &tmB, kb * BK, tn * BN, &full[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+    producer_done:;
+    }
+  } else if (warp == 1) {
+    // ------------------------- MMA issuer -------------------------
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int local = 0;
+      for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++local) {
+        const int buf = local & 1;
+        const uint32_t use = (uint32_t)(local >> 1);
+        if (!mbar_wait(&tempty[buf], (use & 1) ^ 1, status)) goto mma_done;
+        tc_fence_after();
+        const uint32_t d = tmem_base + (uint32_t)(buf * BN);
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(&full[stage], phase, status)) goto mma_done;
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + stage * A_STAGE);
+          const uint32_t b0 = smem_u32(sB + stage * B_STAGE);
+#pragma unroll
+          for (int k = 0; k < BK / 32; ++k) {
+            mma_i8(d, sdesc_sw128(a0 + 32 * k), sdesc_sw128(b0 + 32 * k), (kb | k) != 0);
+          }
+          mma_commit(&empty[stage]);  // frees the stage when these MMAs finish
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        mma_commit(&tfull[buf]);  // accumulator ready for the epilogue
+      }
+    mma_done:;
+    }
+  } else {
+    // ------------------------- epilogue -------------------------
+    const int q = warp & 3;                 // TMEM lane quarter of this warp
+    const int etid = threadIdx.x - 64;      // 0..127
+    const int row_in_tile = 32 * q + lane;
+    const int64_t Kza_zb = (int64_t)ep.K * ep.za * ep.zb;
+    int local = 0;
+    for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++local) {
+      const int tm = t % tiles_m, tn = t / tiles_m;
+      const int buf = local & 1;
+      const uint32_t use = (uint32_t)(local >> 1);
+      epi_bar_sync();  // previous tile's column constants no longer read
+      for (int c = etid; c < BN; c += 128) {
+        const int n = tn * BN + c;
+        if (n < ep.N) {
+          const int64_t v = (ep.bias ? (int64_t)ep.bias[n] : 0) -
+                            (int64_t)ep.za * ep.colsum[n] + Kza_zb;
+          c_term[c] = (int32_t)v;  // wraps mod 2^32; the final sum is in range
+          c_m0[c] = ep.per_channel ? ep.m0v[n] : ep.m0;
+          c_sh[c] = ep.per_channel ? ep.shv[n] : ep.sh;
+        }
+      }
+      epi_bar_sync();
+      const int m = tm * BM + row_in_tile;
+      const bool row_ok = m < ep.M;
+      const int32_t r_term = (ep.rowsum && row_ok) ? -ep.zb * ep.rowsum[m] : 0;
+      const bool ok = epi_bar_and(mbar_wait(&tfull[buf], use & 1, status));
+      tc_fence_after();
+      if (ok) {
+        for (int ch = 0; ch < BN / 32; ++ch) {
+          const int nb = tn * BN + ch * 32;
+          if (nb >= ep.N) break;  // warp-uniform
+          uint32_t r[32];
+          tmem_ld32(tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * BN + ch * 32), r);
+          if (!row_ok) continue;
+          const bool full_chunk = nb + 32 <= ep.N;
+          int accv[32];
+          uint32_t packed[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int c = ch * 32 + j;
+            const int a = (int)((uint32_t)r[j] + (uint32_t)c_term[c] + (uint32_t)r_term);
+            accv[j] = a;
+            const int yv = requant1(a, c_m0[c], c_sh[c], ep.zo, ep.lo, ep.hi);
+            packed[j >> 2] |= ((uint32_t)yv & 0xFFu) << (8 * (j & 3));
+          }
+          int8_t* cp = ep.C + (int64_t)m * ep.ldc + nb;
+          if (full_chunk && (((uintptr_t)cp & 15) == 0)) {
+            reinterpret_cast<uint4*>(cp)[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+            reinterpret_cast<uint4*>(cp)[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (nb + j < ep.N) cp[j] = (int8_t)((packed[j >> 2] >> (8 * (j & 3))) & 0xFF);
+          }
+          if (ep.acc_out) {
+            int32_t* ap = ep.acc_out + (int64_t)m * ep.ld_acc + nb;
+            if (full_chunk && (((uintptr_t)ap & 15) == 0)) {
+#pragma unroll
+              for (int j = 0; j < 32; j += 4)
+                reinterpret_cast<int4*>(ap + j)[0] = make_int4(accv[j], accv[j + 1], accv[j + 2], accv[j + 3]);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (nb + j < ep.N) ap[j] = accv[j];
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[buf]);
+      if (!ok) break;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// B pack (row-major B[K][ldb] -> K-major Bp[Np][Kp], zero padded) with the
+// column sums colsum[n] = sum_{k<K} B[k,n].  64x64 tiles through shared memory.
+// ---------------------------------------------------------------------------
+__global__ void pack_b_rowmajor_kernel(int K, int N, const int8_t* __restrict__ B, int64_t ldb,
+                                       int8_t* __restrict__ Bp, int64_t Kp,
+                                       int32_t* __restrict__ colsum) {
+  __shared__ int8_t t[64][65];
+  const int k0 = blockIdx.x * 64, n0 = blockIdx.y * 64;
+  const int tx = threadIdx.x, ty = threadIdx.y;  // 32 x 8
+  for (int r = ty; r < 64; r += 8) {
+    const int k = k0 + r;
+    for (int c = tx; c < 64; c += 32) {
+      const int n = n0 + c;
+      t[r][c] = (k < K && n < N) ? B[(int64_t)k * ldb + n] : (int8_t)0;
+    }
+  }
+  __syncthreads();
+  for (int r = ty; r < 64; r += 8) {
+    const int n = n0 + r;
+    for (int c = tx; c < 64; c += 32) Bp[(int64_t)n * Kp + k0 + c] = t[c][r];
+  }
+  if (ty == 0) {
+    for (int c = tx; c < 64; c += 32) {
+      int s = 0;
+      for (int r = 0; r < 64; ++r) s += t[r][c];
+      if (n0 + c < N && s != 0) atomicAdd(&colsum[n0 + c], s);
+    }
+  }
+}
+
+// K-major source (w[N][ldw], K contiguous; conv weights [Cout][KH][KW][Cin]).
+__global__ void pack_b_kmajor_kernel(int K, int N, const int8_t* __restrict__ W, int64_t ldw,
+                                     int8_t* __restrict__ Bp, int64_t Kp,
+                                     int32_t* __restrict__ colsum) {
+  __shared__ int red[8];
+  const int n = blockIdx.x;
+  int s = 0;
+  for (int k = threadIdx.x; k < Kp; k += blockDim.x) {
+    int8_t v = (n < N && k < K) ? W[(int64_t)n * ldw + k] : (int8_t)0;
+    Bp[(int64_t)n * Kp + k] = v;
+    s += v;
+  }
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int tot = 0;
+    for (int i = 0; i < (int)(blockDim.x >> 5); ++i) tot += red[i];
+    colsum[n] = tot;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// A staging: copy rows into a 16-byte-aligned buffer (ld = ldw) when A's own
+// rows cannot be described to the tensor-copy engine, and/or compute
+// rowsum[m] = sum_k A[m,k] when zb != 0.  One CTA per row.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) stage_a_kernel(int K, const int8_t* __restrict__ A,
+                                                      int64_t lda, int8_t* __restrict__ Aw,
+                                                      int64_t ldw, int32_t* __restrict__ rowsum) {
+  __shared__ int red[8];
+  const int64_t m = blockIdx.x;
+  const int8_t* src = A + m * lda;
+  int8_t* dst = Aw ? Aw + m * ldw : nullptr;
+  int s = 0;
+  const bool vec = (((uintptr_t)src & 7) == 0);
+  const int K8 = vec ? (K & ~7) : 0;
+  for (int i = threadIdx.x * 8; i < K8; i += blockDim.x * 8) {
+    const uint2 v = *reinterpret_cast<const uint2*>(src + i);
+    if (dst) *reinterpret_cast<uint2*>(dst + i) = v;
+    s = __dp4a((int)v.x, 0x01010101, s);
+    s = __dp4a((int)v.y, 0x01010101, s);
+  }
+  for (int i = K8 + threadIdx.x; i < K; i += blockDim.x) {
+    const int8_t v = src[i];
+    if (dst) dst[i] = v;
+    s += v;
+  }
+  if (rowsum) {
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      int tot = 0;
+      for (int i = 0; i < 8; ++i) tot += red[i];
+      rowsum[m] = tot;
+    }
+  }
+}
+
+// Explicit im2col with the input zero-point in padded taps (conv).
+__global__ void im2col_zp_kernel(int Nb, int H, int W, int Cin, int KH, int KW, int sh, int sw,
+                                 int ph, int pw, int OH, int OW, const int8_t* __restrict__ x,
+                                 int8_t za, int8_t* __restrict__ A, int64_t lda) {
+  const int64_t K = (int64_t)KH * KW * Cin;
+  const int64_t total = (int64_t)Nb * OH * OW * K;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t m = i / K;
+    const int k = (int)(i % K);
+    const int ci = k % Cin, tap = k / Cin;
+    const int kw = tap % KW, kh = tap / KW;
+    const int ow = (int)(m % OW);
+    const int64_t t = m / OW;
+    const int oh = (int)(t % OH);
+    const int n = (int)(t / OH);
+    const int ih = oh * sh + kh - ph, iw = ow * sw + kw - pw;
+    int8_t v = za;
+    if (ih >= 0 && ih < H && iw >= 0 && iw < W) v = x[(((int64_t)n * H + ih) * W + iw) * Cin + ci];
+    A[m * lda + k] = v;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+int get_encode() {
+  if (g_encode) return QG_OK;
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult qr;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &qr) !=
+          cudaSuccess ||
+      qr != cudaDriverEntryPointSuccess || !fn)
+    return QG_ERR_CUDA;
+  g_encode = (PFN_cuTensorMapEncodeTiled_v12000)fn;
+  return QG_OK;
+}
+
+// 2-D uint8 tensor [rows][cols] with row pitch `pitch` bytes, box {128, box_rows}.
+int make_tmap(CUtensorMap* tm, const void* base, uint64_t cols, uint64_t rows, uint64_t pitch,
+              uint32_t box_rows) {
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {pitch};
+  cuuint32_t box[2] = {(cuuint32_t)BK, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? QG_OK : QG_ERR_CUDA;
+}
+
+struct PackDims {
+  int64_t Kp, Np;
+};
+PackDims pack_dims(int K, int N) { return {round_up(K, BK), round_up(N, BN)}; }
+
+}  // namespace
+
+size_t i8gemm_pack_b_bytes(int K, int N) {
+  PackDims d = pack_dims(K, N);
+  return (size_t)(d.Np * d.Kp + d.Np * 4);
+}
+
+static int pack_common(int K, int N, void* packed, cudaStream_t st, int32_t** colsum_out) {
+  PackDims d = pack_dims(K, N);
+  int32_t* colsum = (int32_t*)((int8_t*)packed + d.Np * d.Kp);
+  if (cudaMemsetAsync(colsum, 0, (size_t)d.Np * 4, st) != cudaSuccess) return QG_ERR_CUDA;
+  *colsum_out = colsum;
+  return QG_OK;
+}
+
+int i8gemm_pack_b(int K, int N, const int8_t* B, int64_t ldb, void* packed, cudaStream_t st) {
+  PackDims d = pack_dims(K, N);
+  int32_t* colsum = nullptr;
+  int rc = pack_common(K, N, packed, st, &colsum);
+  if (rc != QG_OK) return rc;
+  dim3 grid((unsigned)(d.Kp / 64), (unsigned)(d.Np / 64));
+  pack_b_rowmajor_kernel<<<grid, dim3(32, 8), 0, st>>>(K, N, B, ldb, (int8_t*)packed, d.Kp, colsum);
+  return launch_status();
+}
+
+int i8gemm_pack_b_kmajor(int K, int N, const int8_t* W, int64_t ldw, void* packed,
+                         cudaStream_t st) {
+  PackDims d = pack_dims(K, N);
+  int32_t* colsum = nullptr;
+  int rc = pack_common(K, N, packed, st, &colsum);
+  if (rc != QG_OK) return rc;
+  pack_b_kmajor_kernel<<<(unsigned)d.Np, 256, 0, st>>>(K, N, W, ldw, (int8_t*)packed, d.Kp, colsum);
+  return launch_status();
+}
+
+static int64_t staged_lda(int K) { return round_up(K, 16); }
+
+size_t i8gemm_packed_workspace_bytes(int M, int K) {
+  return (size_t)(round_up((int64_t)M * staged_lda(K), 256) + round_up((int64_t)M * 4, 256));
+}
+
+int i8gemm_setup() {
+  cudaError_t e = cudaFuncSetAttribute(i8gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)SMEM_BYTES);
+  if (e != cudaSuccess) return QG_ERR_CUDA;
+  return get_encode();
+}
+
+int i8gemm_run_packed(int M, int N, int K, const int8_t* A, int64_t lda, const void* packed_b,
+                      int8_t* C, int64_t ldc, const qg_requant_t& rq, int32_t* acc_out,
+                      int64_t ld_acc, void* ws, size_t ws_bytes, cudaStream_t st) {
+  const PackDims d = pack_dims(K, N);
+  const bool need_copy = (((uintptr_t)A & 15) != 0) || (lda % 16) != 0;
+  const bool need_rowsum = rq.b_zero_point != 0;
+  const int8_t* Aeff = A;
+  int64_t lda_eff = lda;
+  int32_t* rowsum = nullptr;
+  if (need_copy || need_rowsum) {
+    if (!ws || ws_bytes < i8gemm_packed_workspace_bytes(M, K)) return QG_ERR_WORKSPACE;
+    int8_t* Aw = (int8_t*)ws;
+    rowsum = need_rowsum ? (int32_t*)((int8_t*)ws + round_up((int64_t)M * staged_lda(K), 256))
+                         : nullptr;
+    stage_a_kernel<<<M, 256, 0, st>>>(K, A, lda, need_copy ? Aw : nullptr, staged_lda(K), rowsum);
+    int rc = launch_status();
+    if (rc != QG_OK) return rc;
+    if (need_copy) {
+      Aeff = Aw;
+      lda_eff = staged_lda(K);
+    }
+  }
+  CUtensorMap tmA, tmB;
+  int rc = make_tmap(&tmA, Aeff, (uint64_t)K, (uint64_t)M, (uint64_t)lda_eff, BM);
+  if (rc != QG_OK) return rc;
+  rc = make_tmap(&tmB, packed_b, (uint64_t)d.Kp, (uint64_t)d.Np, (uint64_t)d.Kp, BN);
+  if (rc != QG_OK) return rc;
+  EpiArgs ep;
+  ep.M = M; ep.N = N; ep.K = K;
+  ep.za = rq.a_zero_point; ep.zb = rq.b_zero_point; ep.zo = rq.out_zero_point;
+  ep.lo = rq.clamp_min; ep.hi = rq.clamp_max;
+  ep.colsum = (const int32_t*)((const int8_t*)packed_b + d.Np * d.Kp);
+  ep.rowsum = rowsum;
+  ep.bias = rq.bias;
+  ep.per_channel = rq.per_channel;
+  ep.m0 = rq.multiplier0; ep.sh = rq.shift0;
+  ep.m0v = rq.multiplier; ep.shv = rq.shift;
+  ep.C = C; ep.ldc = ldc; ep.acc_out = acc_out; ep.ld_acc = ld_acc;
+  const int tiles_m = (int)cdiv(M, BM), tiles_n = (int)cdiv(N, BN);
+  const int tiles = tiles_m * tiles_n;
+  const int grid = tiles < num_sms() ? tiles : num_sms();
+  const int num_kb = (int)(d.Kp / BK);
+  i8gemm_tc_kernel<<<grid, THREADS, SMEM_BYTES, st>>>(tmA, tmB, num_kb, tiles_m, tiles_n, ep,
+                                                      status_word());
+  return launch_status();
+}
+
+// ---------------------------------------------------------------------------
+// INT8 convolution: weights packed (K-major already, padded, column sums),
+// zero-point-padded im2col of x, then the GEMM above.
+// ---------------------------------------------------------------------------
+static void conv_geometry(int H, int W, int KH, int KW, int sh, int sw, int ph, int pw, int* OH,
+                          int* OW) {
+  *OH = (H + 2 * ph - KH) / sh + 1;
+  *OW = (W + 2 * pw - KW) / sw + 1;
+}
+
+size_t conv_workspace_bytes(int Nb, int H, int W, int Cin, int Cout, int KH, int KW, int sh,
+                            int sw, int ph, int pw) {
+  int OH, OW;
+  conv_geometry(H, W, KH, KW, sh, sw, ph, pw, &OH, &OW);
+  const int64_t K = (int64_t)KH * KW * Cin;
+  const int64_t M = (int64_t)Nb * OH * OW;
+  return (size_t)(round_up((int64_t)i8gemm_pack_b_bytes((int)K, Cout), 256) +
+                  round_up(M * staged_lda((int)K), 256));
+}
+
+int conv_run(int Nb, int H, int W, int Cin, int Cout, int KH, int KW, int sh, int sw, int ph,
+             int pw, const int8_t* x, const int8_t* w, int8_t* y, const qg_requant_t& rq,
+             int32_t* acc_out, void* ws, size_t ws_bytes, cudaStream_t st) {
+  int OH, OW;
+  conv_geometry(H, W, KH, KW, sh, sw, ph, pw, &OH, &OW);
+  const int K = KH * KW * Cin;
+  const int64_t M = (int64_t)Nb * OH * OW;
+  if (M > INT32_MAX) return QG_ERR_UNSUPPORTED;
+  const size_t pb = round_up((int64_t)i8gemm_pack_b_bytes(K, Cout), 256);
+  int8_t* packed = (int8_t*)ws;
+  int8_t* Aim = (int8_t*)ws + pb;
+  int rc = i8gemm_pack_b_kmajor(K, Cout, w, K, packed, st);
+  if (rc != QG_OK) return rc;
+  const int64_t lda = staged_lda(K);
+  const int64_t total = M * K;
+  int blocks = (int)min64(cdiv(total, 256), (int64_t)num_sms() * 16);
+  im2col_zp_kernel<<<blocks, 256, 0, st>>>(Nb, H, W, Cin, KH, KW, sh, sw, ph, pw, OH, OW, x,
+                                           (int8_t)rq.a_zero_point, Aim, lda);
+  rc = launch_status();
+  if (rc != QG_OK) return rc;
+  return i8gemm_run_packed((int)M, Cout, K, Aim, lda, packed, y, Cout, rq, acc_out, Cout, nullptr,
+                           0, st);
+}
+
+}  // namespace qg

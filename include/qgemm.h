@@ -1,0 +1,235 @@
+/*
+ * qgemm.h — C ABI of the B200 (sm_100a) quantized integer matmul library.
+ *
+ * Operations (sources cited by page title and section):
+ *   [QG]  xidianedu, "量化 GEMM：数值契约、SRAM、DMA 与结果验证" (quantized GEMM:
+ *         numeric contract, SRAM, DMA and result verification), sections 1-5.
+ *   [MNN] MNN source/backend/cpu/compute/ConvInt8TiledExecutor.cpp
+ *         (initializeConvInt8QuantInfo, reorderWeight, _computeReorderQuantInfo,
+ *          BatchAsyDynamicQuant, tileSplitFunction / QuanPostTreatParameters).
+ *   [KAI] pytorch/ao PR #997, "Kleidi 4b blockwise gemv prototype"
+ *         (matmul_clamp_f32_qai8dxp_qsi4c32p micro-kernels and their wrapper).
+ *
+ * Conventions shared by every entry point
+ *   - Pointers to tensors are DEVICE pointers unless a parameter says "host".
+ *     The caller owns and allocates every buffer; no entry point allocates
+ *     device memory.  Scratch space is passed as `workspace`, sized by the
+ *     matching *_workspace_bytes() query (0 means none is needed).
+ *   - Strides (ld*) count ELEMENTS, not bytes ([QG] section 5: row-major
+ *     A at base_A + (m*lda + k)*elem_bytes).  Logical sizes may be smaller
+ *     than physical ones (lda >= K, ...; [QG] section 2).  Inputs and outputs
+ *     must not alias.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream).  The return value reports argument checks and launch
+ *     errors.  Errors found on the device (a bounded wait that ran out, an
+ *     int4 weight out of range) are recorded in a per-device status word that
+ *     qg_device_status() reads after the work has finished.
+ *   - Every entry point returns QG_OK (0) or a negative qg_status.  It never
+ *     aborts the process and never traps on the GPU.
+ */
+#ifndef QGEMM_H_
+#define QGEMM_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define QG_API_VERSION 1
+
+typedef enum {
+  QG_OK = 0,
+  QG_ERR_INVALID_ARG = -1,     /* bad size, NULL pointer, stride < logical size, bad clamp */
+  QG_ERR_MISALIGNED = -2,      /* pointer alignment the operation requires is not met */
+  QG_ERR_OVERFLOW_BOUND = -3,  /* K*65025 + |bias| > INT32_MAX ([QG] section 4) */
+  QG_ERR_UNSUPPORTED = -4,     /* valid but not implemented (e.g. K % 32 != 0 for A8W4) */
+  QG_ERR_CUDA = -5,            /* a CUDA runtime call or kernel launch failed */
+  QG_ERR_TIMEOUT = -6,         /* a bounded device-side wait ran out (device status) */
+  QG_ERR_WORKSPACE = -7,       /* workspace missing or smaller than the query says */
+  QG_ERR_NO_DEVICE = -8        /* no sm_100 device is current */
+} qg_status;
+
+/* Human-readable name of a status code.  Never NULL. */
+const char* qg_status_string(int status);
+
+/* QG_API_VERSION of the built library. */
+int qg_version(void);
+
+/*
+ * Per-device error word.  Synchronises the current device, then returns
+ * QG_OK or the first qg_status a kernel recorded since the last reset; with
+ * reset != 0 the word is cleared afterwards.  Returns QG_ERR_CUDA if the
+ * synchronisation itself fails.
+ */
+int qg_device_status(int reset);
+
+/* ------------------------------------------------------------------------
+ * Requantization parameters of the affine INT8 contract.
+ *
+ * [QG] section 1: real = scale * (q - zero_point); the int32 bias lives in
+ * the accumulator scale sA*sB[n]; the ratio sA*sB[n]/sO is applied as an
+ * integer multiplier and shift.  [MNN] initializeConvInt8QuantInfo /
+ * QuanPostTreatParameters: output zero-point, clamp [clamp_min, clamp_max],
+ * fused ReLU expressed as clamp_min = out_zero_point.
+ *
+ * For every output element the library computes, exactly:
+ *   acc = sum_{k<K} (A[m,k]-a_zero_point)*(B[k,n]-b_zero_point) + bias[n]
+ *   y   = clamp(out_zero_point + rne(acc * M0 / 2^(31+shift)),
+ *               clamp_min, clamp_max)
+ * where rne rounds half to even on the exact 64-bit product and M0/shift are
+ * multiplier0/shift0 (per_channel == 0) or multiplier[n]/shift[n].
+ * ------------------------------------------------------------------------ */
+typedef struct {
+  int32_t a_zero_point;       /* za in [-128,127]; also the conv pad value */
+  int32_t b_zero_point;       /* zb in [-128,127]; 0 for symmetric weights */
+  const int32_t* bias;        /* device int32 [N], or NULL for no bias */
+  int32_t bias_abs_max;       /* host bound on |bias[n]| (>= 0) for the overflow check */
+  int32_t per_channel;        /* 0: multiplier0/shift0; 1: multiplier[N]/shift[N] */
+  int32_t multiplier0;        /* M0 in [2^30, 2^31) when per_channel == 0 */
+  int32_t shift0;             /* right shift in [0, 31] when per_channel == 0 */
+  const int32_t* multiplier;  /* device int32 [N] when per_channel == 1 */
+  const int32_t* shift;       /* device int32 [N] when per_channel == 1 */
+  int32_t out_zero_point;     /* zo in [-128,127] */
+  int32_t clamp_min;          /* int8 range, clamp_min <= clamp_max */
+  int32_t clamp_max;
+} qg_requant_t;
+
+/*
+ * Host helper: ratio = sA*sB/sO (0 < ratio < 1) -> (M0, shift) with
+ * ratio ~= M0 * 2^-(31+shift).  frexp(ratio) = f*2^e, M0 = round(f*2^31)
+ * (ties away from zero; 2^31 -> 2^30 and e+1), shift = -e.
+ * QG_ERR_UNSUPPORTED if ratio is outside (0,1) or shift would exceed 31;
+ * QG_ERR_INVALID_ARG for NULL outputs.
+ */
+int qg_requant_params(double ratio, int32_t* m0, int32_t* shift);
+
+/* ------------------------------------------------------------------------
+ * Affine INT8 GEMM with fused zero-point correction, bias, requant, clamp.
+ * [QG] sections 1 (contract), 2 (padding is real zero, logical vs physical
+ * shape), 4 (INT32 accumulator kept across all K blocks, requant once after
+ * the last block, overflow bound K*65025 + |bias|).
+ *
+ *   A: int8 row-major [M][lda], lda >= K.      B: int8 row-major [K][ldb], ldb >= N.
+ *   C: int8 row-major [M][ldc], ldc >= N (written).
+ *   acc_out: optional int32 row-major [M][ld_acc] (ld_acc >= N) receiving the
+ *            pre-requant accumulator including bias; NULL to skip.
+ *   rq: host pointer to the parameters above.
+ * Rejects (QG_ERR_OVERFLOW_BOUND) any call with K*65025 + bias_abs_max
+ * above INT32_MAX.  M, N, K >= 1.  Any alignment of A, B, C is accepted.
+ * ------------------------------------------------------------------------ */
+size_t qgemm_s8s8_workspace_bytes(int M, int N, int K);
+int qgemm_s8s8_requant(int M, int N, int K,
+                       const int8_t* A, int64_t lda,
+                       const int8_t* B, int64_t ldb,
+                       int8_t* C, int64_t ldc,
+                       const qg_requant_t* rq,
+                       int32_t* acc_out, int64_t ld_acc,
+                       void* workspace, size_t workspace_bytes,
+                       void* stream);
+
+/*
+ * Weight-stationary variant: B is packed once by qgemm_pack_b_s8 ([MNN]
+ * reorderWeight: weights reordered once at load, with per-column kernel
+ * sums) and reused.  The packed buffer is opaque; its size comes from
+ * qgemm_pack_b_s8_bytes and it must be 128-byte aligned.  The pack stores no
+ * zero-point: rq->b_zero_point is applied at GEMM time.  workspace is needed
+ * only when A's rows are not 16-byte aligned or b_zero_point != 0.
+ */
+size_t qgemm_pack_b_s8_bytes(int K, int N);
+int qgemm_pack_b_s8(int K, int N, const int8_t* B, int64_t ldb,
+                    void* packed_b, size_t packed_bytes, void* stream);
+size_t qgemm_s8s8_packed_workspace_bytes(int M, int K);
+int qgemm_s8s8_requant_packed(int M, int N, int K,
+                              const int8_t* A, int64_t lda,
+                              const void* packed_b,
+                              int8_t* C, int64_t ldc,
+                              const qg_requant_t* rq,
+                              int32_t* acc_out, int64_t ld_acc,
+                              void* workspace, size_t workspace_bytes,
+                              void* stream);
+
+/* ------------------------------------------------------------------------
+ * INT8 convolution as implicit-im2col GEMM.  [MNN] tileSplitFunction: the
+ * im2col buffer is filled with the input zero-point where a tap falls in the
+ * padding; [QG] section 2: padding must stand for real zero.
+ *
+ *   x: int8 NHWC [Nb][H][W][Cin]      w: int8 [Cout][KH][KW][Cin] (zw = 0)
+ *   y: int8 NHWC [Nb][OH][OW][Cout], OH = (H+2*pad_h-KH)/stride_h + 1 (same for W)
+ *   acc_out: optional int32 NHWC [Nb][OH][OW][Cout].
+ * GEMM view: M = Nb*OH*OW, N = Cout, K = KH*KW*Cin; pad value =
+ * rq->a_zero_point; rq->b_zero_point must be 0.  Per-Cout requant via
+ * rq->per_channel.  Fused ReLU: rq->clamp_min = rq->out_zero_point.
+ * ------------------------------------------------------------------------ */
+size_t qconv2d_s8_workspace_bytes(int Nb, int H, int W, int Cin, int Cout,
+                                  int KH, int KW, int stride_h, int stride_w,
+                                  int pad_h, int pad_w);
+int qconv2d_s8_im2col(int Nb, int H, int W, int Cin, int Cout, int KH, int KW,
+                      int stride_h, int stride_w, int pad_h, int pad_w,
+                      const int8_t* x, const int8_t* w, int8_t* y,
+                      const qg_requant_t* rq, int32_t* acc_out,
+                      void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Dynamic per-row asymmetric int8 activation quantization.  [MNN]
+ * BatchAsyDynamicQuant (min/max -> scale and zero-point, quantize with clamp
+ * to [-128,127]); [KAI] qai8dx (int8, dynamic, per row, asymmetric); [QG]
+ * section 1 (ONNX QuantizeLinear rounding: half to even).  All float32, one
+ * rounding per operation:
+ *   rmin = min(0, min_k x), rmax = max(0, max_k x)
+ *   scale = (rmax - rmin)/255, or 1 if that is 0;  inv = 1/scale
+ *   zero_point = clamp(rne(-128 - rmin*inv), -128, 127)
+ *   q[k] = clamp(rne(x[k]*inv) + zero_point, -128, 127)
+ *   x: f32 [M][ldx] (ldx >= K); q: int8 [M][ldq] (ldq >= K);
+ *   scale: f32 [M]; zero_point: int32 [M].  Non-finite x is out of contract.
+ * ------------------------------------------------------------------------ */
+int quantize_rows_a8(int M, int K, const float* x, int64_t ldx,
+                     int8_t* q, int64_t ldq, float* scale,
+                     int32_t* zero_point, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Int4 weights with one f32 scale per 32-wide K group.  [KAI] qsi4c32
+ * (symmetric int4, group 32; weight zero-points absent), [MNN]
+ * _computeReorderQuantInfo (int4 stored with an offset of 8).
+ *
+ *   w: int8 [N][ldw] (ldw >= K), values in [-8,7] (row n = output channel);
+ *   group_scales: f32 [N][K/32]; K % 32 == 0.
+ *   packed: opaque buffer of pack_w4_g32_bytes(N, K) bytes, 16-byte aligned:
+ *     N rows of K/2 bytes, where the little-endian 32-bit word j of a row
+ *     holds (w[8j+b]+8) in the low nibble and (w[8j+4+b]+8) in the high
+ *     nibble of byte b (b = 0..3), followed by the f32 scales [N][K/32].
+ * A weight outside [-8,7] records QG_ERR_INVALID_ARG in the device status.
+ * ------------------------------------------------------------------------ */
+size_t pack_w4_g32_bytes(int N, int K);
+int pack_w4_g32(int N, int K, const int8_t* w, int64_t ldw,
+                const float* group_scales, void* packed, size_t packed_bytes,
+                void* stream);
+
+/* ------------------------------------------------------------------------
+ * A8W4 linear: y = clamp(dequant(quantize_rows_a8(x)) @ dequant(W)^T + bias).
+ * [KAI] matmul_clamp_f32_qai8dxp_qsi4c32p: f32 out, clamp after bias
+ * (clamp_min = -INFINITY / clamp_max = +INFINITY for none).  Per element:
+ *   y[m,n] = clamp(sA[m] * sum_g sw[n,g] * I[m,n,g] + bias[n])
+ *   I[m,n,g] = sum_{k in g} (qA[m,k] - zA[m]) * w[n,k]   (exact integer)
+ * with the group combination in float32.
+ *   x: f32 [M][ldx] (ldx >= K); packed_w from pack_w4_g32; bias f32 [N] or
+ *   NULL; y: f32 [M][ldy] (ldy >= N).  K % 32 == 0 (else QG_ERR_UNSUPPORTED).
+ *   q_out [M][K] int8 / scale_out [M] / zp_out [M]: optional (each may be
+ *   NULL), receive the activation quantization for bit-exact checks.
+ * M == 1 runs one fused kernel (quantization inside); M > 1 quantizes into
+ * the workspace first.
+ * ------------------------------------------------------------------------ */
+size_t qgemm_a8w4_workspace_bytes(int M, int K);
+int qgemm_a8w4_f32(int M, int N, int K, const float* x, int64_t ldx,
+                   const void* packed_w, const float* bias,
+                   float clamp_min, float clamp_max,
+                   float* y, int64_t ldy,
+                   int8_t* q_out, float* scale_out, int32_t* zp_out,
+                   void* workspace, size_t workspace_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QGEMM_H_ */

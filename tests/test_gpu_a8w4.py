@@ -1,0 +1,162 @@
+"""GPU parity of the A8W4 path against the CPU oracle, through the C ABI.
+
+Quantized activations (q, scale, zero-point) and packed weights must match
+bit-exactly; f32 outputs within |y - y_ref| <= 1e-4 * max(|y_ref|, 1)
+(relative 1e-4 for |y| >= 1, absolute 1e-4 below; see the tolerance reading
+in the design notes)."""
+import numpy as np
+import pytest
+
+import oracle
+import workloads
+
+pytestmark = pytest.mark.gpu
+torch = pytest.importorskip("torch")
+
+TOL = 1e-4
+
+
+def _dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def assert_a8w4_close(y, y_ref):
+    err = np.abs(y.astype(np.float64) - y_ref.astype(np.float64)) / np.maximum(np.abs(y_ref), 1.0)
+    i = int(np.argmax(err))
+    assert err.flat[i] <= TOL, f"max err {err.flat[i]:.3e} at {np.unravel_index(i, y.shape)}: " \
+                               f"{y.flat[i]} vs {y_ref.flat[i]}"
+
+
+@pytest.fixture(autouse=True)
+def _clean_status(lib, cuda):
+    lib.qg_device_status(True)
+    yield
+    assert lib.qg_device_status(True) == 0
+
+
+# ---------------------------------------------------------------------------
+# dynamic quantization
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("M,K,pad", [(1, 4096, 0), (128, 4096, 0), (3, 33, 5), (5, 1, 0),
+                                     (2, 1000, 3), (7, 12345, 1)])
+def test_quantize_rows_bit_exact(lib, M, K, pad):
+    rng = np.random.default_rng(M * 1000 + K)
+    x = (rng.standard_normal((M, K + pad)) * rng.uniform(0.1, 10, (M, 1))).astype(np.float32)
+    if M >= 3:
+        x[1] = 0.0                       # all-zero row
+        x[2] = 3.25                      # constant positive row
+    q_ref, s_ref, z_ref = oracle.quantize_rows_a8(x[:, :K])
+    xd = _dev(x)
+    q = torch.full((M, K + 2), 99, dtype=torch.int8, device="cuda")
+    s = torch.empty(M, dtype=torch.float32, device="cuda")
+    z = torch.empty(M, dtype=torch.int32, device="cuda")
+    lib.quantize_rows_a8(xd[:, :K], q[:, :K], s, z)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(q[:, :K].cpu().numpy(), q_ref)
+    assert (q[:, K:].cpu().numpy() == 99).all()          # ldq padding untouched
+    np.testing.assert_array_equal(s.cpu().numpy().view(np.int32), s_ref.view(np.int32))
+    np.testing.assert_array_equal(z.cpu().numpy(), z_ref)
+
+
+def test_quantize_rows_golden_specials(lib):
+    import json, os
+    g = json.load(open(os.path.join(os.path.dirname(__file__), "golden",
+                                    "qg_dynamic_quant_specials.json")))
+    for case in g["cases"]:
+        x = np.array([case["x"]], np.float32)
+        xd = _dev(x)
+        q = torch.empty(x.shape, dtype=torch.int8, device="cuda")
+        s = torch.empty(1, dtype=torch.float32, device="cuda")
+        z = torch.empty(1, dtype=torch.int32, device="cuda")
+        lib.quantize_rows_a8(xd, q, s, z)
+        torch.cuda.synchronize()
+        assert s.item() == case["scale"] and z.item() == case["zp"]
+        assert q.cpu().numpy()[0].tolist() == case["q"]
+
+
+# ---------------------------------------------------------------------------
+# W4 pack
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("N,K,ldw", [(7, 96, 100), (300, 1024, 1024), (14336, 4096, 4096)])
+def test_pack_w4_bit_exact(lib, N, K, ldw):
+    w = workloads.a8w4(1, N, K, seed=N + K)
+    qw = np.zeros((N, ldw), np.int8)
+    qw[:, :K] = w["qw"]
+    packed = lib.pack_w4_g32(_dev(qw)[:, :K], _dev(w["sw"]))
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(packed.cpu().numpy(), oracle.pack_w4_g32(w["qw"], w["sw"]))
+
+
+def test_pack_w4_out_of_range_recorded(lib):
+    qw = np.zeros((2, 32), np.int8)
+    qw[1, 5] = 9                                       # not an int4 value
+    lib.pack_w4_g32(_dev(qw), _dev(np.ones((2, 1), np.float32)))
+    assert lib.qg_device_status(True) == -1
+
+
+# ---------------------------------------------------------------------------
+# A8W4 linear
+# ---------------------------------------------------------------------------
+def _run_a8w4(lib, w, ldy_pad=0, with_outputs=True):
+    M, N, K = w["M"], w["N"], w["K"]
+    packed = lib.pack_w4_g32(_dev(w["qw"]), _dev(w["sw"]))
+    x = _dev(w["x"])[:, :K]
+    y = torch.full((M, N + ldy_pad), 7.0, dtype=torch.float32, device="cuda")
+    q = torch.empty((M, K), dtype=torch.int8, device="cuda") if with_outputs else None
+    s = torch.empty(M, dtype=torch.float32, device="cuda") if with_outputs else None
+    z = torch.empty(M, dtype=torch.int32, device="cuda") if with_outputs else None
+    bias = None if w["bias"] is None else _dev(w["bias"])
+    lib.qgemm_a8w4_f32(x, packed, N, bias, w["clamp_min"], w["clamp_max"], y[:, :N], q, s, z)
+    torch.cuda.synchronize()
+    y_np = y.cpu().numpy()
+    if ldy_pad:
+        assert (y_np[:, N:] == 7.0).all()
+    out = (y_np[:, :N],)
+    if with_outputs:
+        out += (q.cpu().numpy(), s.cpu().numpy(), z.cpu().numpy())
+    return out
+
+
+def _check_a8w4(lib, w, **kw):
+    y, q, s, z = _run_a8w4(lib, w, **kw)
+    y_ref, q_ref, s_ref, z_ref = oracle.qgemm_a8w4_f32(w["x"][:, :w["K"]], w["qw"], w["sw"],
+                                                       w["bias"], w["clamp_min"], w["clamp_max"])
+    np.testing.assert_array_equal(q, q_ref)
+    np.testing.assert_array_equal(s.view(np.int32), s_ref.view(np.int32))
+    np.testing.assert_array_equal(z, z_ref)
+    assert_a8w4_close(y, y_ref)
+    return y, y_ref
+
+
+def test_gemv_full_size_cfg2(lib):
+    w = workloads.cfg2_gemv()
+    y, y_ref = _check_a8w4(lib, w)
+    # the clamp binds on a large share of outputs at this scale; both sides agree where it does
+    assert ((np.abs(y_ref) == 6.0) == (np.abs(y) == 6.0)).mean() > 0.999
+
+
+@pytest.mark.parametrize("N,K,bias,clamp", [
+    (1, 32, True, (-np.inf, np.inf)), (7, 96, False, (-np.inf, np.inf)),
+    (300, 1024, True, (-2.0, 2.0)), (1000, 2080, True, (-np.inf, np.inf)),
+    (33, 8192, True, (-np.inf, np.inf)), (17, 12288, False, (-np.inf, np.inf)),
+    (5000, 4096, True, (-6.0, 6.0))])
+def test_gemv_shapes(lib, N, K, bias, clamp):
+    w = workloads.a8w4(1, N, K, seed=N * 7 + K, clamp=clamp, with_bias=bias, ldx=K + 3)
+    _check_a8w4(lib, w, ldy_pad=2)
+
+
+@pytest.mark.parametrize("M,N,K", [(2, 64, 64), (9, 300, 1024), (17, 1000, 4096), (128, 256, 4096)])
+def test_a8w4_gemm_shapes(lib, M, N, K):
+    w = workloads.a8w4(M, N, K, seed=M * 31 + N + K, clamp=(-np.inf, np.inf), ldx=K + 1)
+    _check_a8w4(lib, w, ldy_pad=1)
+
+
+def test_a8w4_gemm_full_size_cfg3(lib):
+    _check_a8w4(lib, workloads.cfg3_gemm())
+
+
+def test_gemv_without_optional_outputs_matches(lib):
+    w = workloads.a8w4(1, 640, 4096, seed=3)
+    (y,) = _run_a8w4(lib, w, with_outputs=False)
+    y2, *_ = _run_a8w4(lib, w)
+    np.testing.assert_array_equal(y, y2)

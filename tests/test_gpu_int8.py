@@ -1,0 +1,168 @@
+"""GPU parity of the INT8 GEMM and INT8 convolution against the CPU oracle,
+through the C ABI.  Integer outputs (int8 C and the int32 accumulators) must
+match bit-exactly."""
+import numpy as np
+import pytest
+
+import oracle
+import workloads
+
+pytestmark = pytest.mark.gpu
+torch = pytest.importorskip("torch")
+
+
+def _dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+@pytest.fixture(autouse=True)
+def _clean_status(lib, cuda):
+    lib.qg_device_status(True)
+    yield
+    assert lib.qg_device_status(True) == 0
+
+
+def _params(lib, w):
+    """(library requant struct args, oracle m0/shift) from the workload's ratios."""
+    ratios = np.atleast_1d(w["ratio"])
+    lib_p = [lib.qg_requant_params(float(r)) for r in ratios]
+    ora_p = [oracle.requant_params(float(r)) for r in ratios]
+    assert lib_p == ora_p
+    m0 = np.array([p[0] for p in ora_p], np.int64)
+    sh = np.array([p[1] for p in ora_p], np.int64)
+    if w.get("per_channel", False) or ratios.size > 1:
+        mult = _dev(m0.astype(np.int32))
+        shift = _dev(sh.astype(np.int32))
+    else:
+        mult, shift, m0, sh = int(m0[0]), int(sh[0]), int(m0[0]), int(sh[0])
+    return mult, shift, m0, sh
+
+
+def run_gemm(lib, w, packed=False, with_acc=True, rows=None, ldc_pad=0):
+    M, N, K = w["M"], w["N"], w["K"]
+    A = _dev(w["A"])[:, :K]
+    B = _dev(w["B"])[:, :N]
+    mult, shift, m0, sh = _params(lib, w)
+    bias = None if w["bias"] is None else _dev(w["bias"])
+    rq = lib.make_requant(a_zero_point=w["za"], b_zero_point=w["zb"], bias=bias,
+                          multiplier=mult, shift=shift, out_zero_point=w["out_zp"],
+                          clamp_min=w["clamp_min"], clamp_max=w["clamp_max"])
+    C = torch.full((M, N + ldc_pad), 55, dtype=torch.int8, device="cuda")
+    acc = torch.full((M, N), 7, dtype=torch.int32, device="cuda") if with_acc else None
+    if packed:
+        pb = lib.qgemm_pack_b_s8(B)
+        lib.qgemm_s8s8_requant_packed(A, pb, N, C[:, :N], rq, K=K, acc_out=acc)
+    else:
+        lib.qgemm_s8s8_requant(A, B, C[:, :N], rq, K=K, N=N, acc_out=acc)
+    torch.cuda.synchronize()
+    Cn = C.cpu().numpy()
+    if ldc_pad:
+        assert (Cn[:, N:] == 55).all()
+    return Cn[:, :N], (acc.cpu().numpy() if with_acc else None), m0, sh
+
+
+def check_gemm(lib, w, rows=None, **kw):
+    C, acc, m0, sh = run_gemm(lib, w, **kw)
+    K, N = w["K"], w["N"]
+    Ar = w["A"][:, :K] if rows is None else w["A"][rows, :K]
+    C_ref, acc_ref = oracle.qgemm_s8s8_requant(Ar, w["B"][:, :N], w["za"], w["zb"], w["bias"],
+                                               m0, sh, w["out_zp"], w["clamp_min"],
+                                               w["clamp_max"])
+    Cg = C if rows is None else C[rows]
+    np.testing.assert_array_equal(Cg, C_ref)
+    if acc is not None:
+        np.testing.assert_array_equal(acc if rows is None else acc[rows], acc_ref)
+    return C, C_ref
+
+
+def test_gemm_cfg0_bit_exact(lib):
+    w = workloads.cfg0_gemm_small()
+    C, C_ref = check_gemm(lib, w)
+    # the outputs are not trivially saturated
+    assert 0.05 < np.mean(np.abs(C_ref.astype(int)) < 127)
+
+
+def test_gemm_cfg0_packed_bit_exact(lib):
+    check_gemm(lib, workloads.cfg0_gemm_small(), packed=True, ldc_pad=3)
+
+
+SHAPES = [(1, 1, 1), (2, 16, 31), (127, 70, 129), (128, 256, 128), (129, 257, 256),
+          (300, 600, 300), (64, 40, 1000), (257, 513, 130)]
+
+
+@pytest.mark.parametrize("M,N,K", SHAPES)
+@pytest.mark.parametrize("per_channel,zb", [(False, None), (True, 0)])
+def test_gemm_shapes(lib, M, N, K, per_channel, zb):
+    seed = M * 10007 + N * 101 + K + (1 if per_channel else 0)
+    w = workloads.int8_gemm(M, N, K, seed, per_channel=per_channel, zb=zb,
+                            lda=K + (seed % 5), ldb=N + (seed % 3))
+    check_gemm(lib, w)
+
+
+def test_gemm_relu_clamp_and_no_bias(lib):
+    w = workloads.int8_gemm(200, 96, 200, seed=77, with_bias=False, out_zp=-10,
+                            clamp=(-10, 127))
+    check_gemm(lib, w)
+
+
+def test_gemm_extreme_bound(lib):
+    # all terms at the worst magnitude 255*255 with K at the page's example size
+    K = 129
+    w = workloads.int8_gemm(130, 70, K, seed=1, za=-128, zb=127, with_bias=False)
+    w["A"][:] = 127
+    w["B"][:] = -128
+    w["ratio"] = np.array([1e-7])
+    C, acc, m0, sh = run_gemm(lib, w)
+    assert (acc == -K * 65025).all()
+
+
+def test_gemm_deterministic(lib):
+    w = workloads.int8_gemm(300, 300, 500, seed=9)
+    C1, a1, *_ = run_gemm(lib, w)
+    C2, a2, *_ = run_gemm(lib, w)
+    np.testing.assert_array_equal(C1, C2)
+    np.testing.assert_array_equal(a1, a2)
+
+
+def test_gemm_cfg4_full_size_sampled_rows(lib):
+    w = workloads.cfg4_gemm_large()
+    rows = np.array([0, 1, 127, 128, 129, 2047, 4096, 5000, 8063, 8064, 8190, 8191])
+    C, C_ref = check_gemm(lib, w, packed=True, rows=rows)
+    # every column of the sampled rows is checked; outputs are not all saturated
+    assert np.mean(np.abs(C_ref.astype(int)) < 127) > 0.05
+
+
+# ---------------------------------------------------------------------------
+# convolution
+# ---------------------------------------------------------------------------
+def run_conv(lib, w, with_acc=True):
+    mult, shift, m0, sh = _params(lib, dict(ratio=w["ratio"], per_channel=True))
+    bias = None if w["bias"] is None else _dev(w["bias"])
+    rq = lib.make_requant(a_zero_point=w["za"], bias=bias, multiplier=mult, shift=shift,
+                          out_zero_point=w["out_zp"], clamp_min=w["clamp_min"],
+                          clamp_max=w["clamp_max"])
+    OH, OW = lib.conv_out_hw(w["H"], w["W"], w["KH"], w["KW"], w["stride"], w["pad"])
+    y = torch.empty((w["Nb"], OH, OW, w["Cout"]), dtype=torch.int8, device="cuda")
+    acc = torch.empty((w["Nb"], OH, OW, w["Cout"]), dtype=torch.int32, device="cuda") if with_acc else None
+    lib.qconv2d_s8_im2col(_dev(w["x"]), _dev(w["w"]), y, rq, w["stride"], w["pad"], acc_out=acc)
+    torch.cuda.synchronize()
+    y_ref, acc_ref = oracle.qconv2d_s8(w["x"], w["w"], w["stride"], w["pad"], w["za"], w["bias"],
+                                       m0, sh, w["out_zp"], w["clamp_min"], w["clamp_max"])
+    np.testing.assert_array_equal(y.cpu().numpy(), y_ref)
+    if with_acc:
+        np.testing.assert_array_equal(acc.cpu().numpy(), acc_ref)
+    return y_ref
+
+
+def test_conv_cfg1_bit_exact(lib):
+    y_ref = run_conv(lib, workloads.cfg1_conv())
+    assert (y_ref == -10).mean() > 0.05      # the ReLU floor at the out zero-point binds
+
+
+@pytest.mark.parametrize("Nb,H,W,Cin,Cout,KH,KW,s,p", [
+    (1, 9, 7, 8, 5, 3, 3, 1, 1), (2, 15, 16, 3, 33, 3, 3, 2, 1), (1, 8, 8, 64, 300, 1, 1, 1, 0),
+    (3, 11, 13, 20, 64, 5, 3, 2, 2), (1, 30, 30, 130, 17, 3, 3, 1, 0)])
+def test_conv_shapes(lib, Nb, H, W, Cin, Cout, KH, KW, s, p):
+    w = workloads.int8_conv(Nb, H, W, Cin, Cout, KH, KW, (s, s), (p, p), seed=H * W + Cin + Cout,
+                            relu=(Cout % 2 == 1))
+    run_conv(lib, w)
