@@ -1,0 +1,601 @@
+#!/usr/bin/env python3
+"""Benchmark of the quantized-matmul hot path on B200.
+
+One step = one pass over the two headline workloads, each through the C ABI
+with its inputs resident in HBM:
+  * INT8 GEMM 8192x8192x8200 (row-major A with lda 8200, za = 7; B pre-packed
+    once, symmetric, per-column Q31 requant, bias, clamp) -> int8 C
+  * A8W4 GEMV 1x14336x4096 (f32 x quantized per row inside the kernel, int4
+    group-32 weights pre-packed once) -> f32 y
+value = integer ops of both (2 per MAC) / step time, in TOPS, whole job.
+Per-part numbers (GEMM TOPS, GEMV HBM GB/s) and each kernel's fraction of the
+measured roofline are on the same JSON line.
+
+Timing: W untimed warm-up steps, then exactly K steps bracketed by a barrier
+and cudaDeviceSynchronize on both sides, CUDA events on the launching stream,
+max over ranks.  L2 (126 MB) is defeated by rotating input sets larger than
+it: 2 GEMM sets (A + packed B = 135 MB each) and 8 GEMV weight sets (36.8 MB
+each, 295 MB in all).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+                  [--workload headline|cfg0|cfg1|cfg2|cfg3|cfg4] [--no-cpu-baseline]
+Under torchrun each rank runs the same work on its own GPU (replicas: the
+path has no exchange step), and value sums all ranks' work.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "INT8 GEMM TOPS and A8W4 GEMV HBM GB/s, as % of B200 roofline"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+INT8_OVER_BF16 = 2.0  # nominal dense ratio (4.5 POPS int8 vs 2.25 PFLOPS bf16)
+
+
+def load_peaks():
+    if os.path.exists(PEAKS_FILE):
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return p, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# Algorithmic work per call (what the method must move / compute)
+# ---------------------------------------------------------------------------
+def gemm_ops(M, N, K):
+    return 2.0 * M * N * K
+
+
+def gemm_bytes(M, N, K):
+    # A, B, C int8 + bias/multiplier/shift int32 per column
+    return M * K + K * N + M * N + 3 * 4 * N
+
+
+def a8w4_bytes(M, N, K):
+    # int4 nibbles + f32 group scales + f32 x + f32 bias + f32 y
+    return N * K // 2 + N * (K // 32) * 4 + M * K * 4 + N * 4 + M * N * 4
+
+
+def a8w4_ops(M, N, K):
+    return 2.0 * M * N * K
+
+
+# ---------------------------------------------------------------------------
+# Distributed plumbing (replicas; one process per GPU)
+# ---------------------------------------------------------------------------
+class Dist:
+    def __init__(self, want):
+        import torch
+        self.torch = torch
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+        if self.world > 1:
+            import datetime
+            import torch.distributed as dist
+            backend = "nccl" if torch.cuda.is_available() else "gloo"
+            if backend == "nccl":
+                torch.cuda.set_device(self.local)
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+            self.pg = dist
+        if want and want != self.world and self.rank == 0:
+            print(f"# note: --gpus {want} but WORLD_SIZE={self.world}", file=sys.stderr)
+
+    def barrier(self):
+        if self.pg:
+            if self.torch.cuda.is_available():
+                self.pg.barrier(device_ids=[self.local])
+            else:
+                self.pg.barrier()
+
+    def max(self, v):
+        if not self.pg:
+            return v
+        dev = "cuda" if self.torch.cuda.is_available() else "cpu"
+        t = self.torch.tensor([float(v)], dtype=self.torch.float64, device=dev)
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            self.pg.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------
+# Clock sampling during the timed region
+# ---------------------------------------------------------------------------
+class Clocks:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.idx = str(gpu_index)
+        self.proc = None
+        self.path = os.path.join("/tmp", f"qg_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.idx, f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if not self.proc:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                rows.append((float(f[1]), float(f[2]), float(f[3]), f[5:9]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        load = [r for r in rows if r[2] > 200.0] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in load for i, v in enumerate(r[3]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in load), "sm_max_mhz": max(r[1] for r in rows),
+                "samples": len(load), "power_w_max": max(r[2] for r in rows), "reasons": reasons}
+
+
+# ---------------------------------------------------------------------------
+# Workload setup on the GPU
+# ---------------------------------------------------------------------------
+def dev(a, torch):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+class GemmCase:
+    """INT8 GEMM (weights pre-packed), `sets` rotating input sets."""
+
+    def __init__(self, qg, torch, w, sets):
+        self.M, self.N, self.K = w["M"], w["N"], w["K"]
+        self.qg, self.torch = qg, torch
+        ratios = np.atleast_1d(w["ratio"])
+        params = [qg.qg_requant_params(float(r)) for r in ratios]
+        per_channel = ratios.size > 1
+        self.inputs = []
+        B0 = dev(w["B"], torch)[:, :self.N]
+        for s in range(sets):
+            # distinct sets (same distributions): rotate A along K and B along K
+            A = dev(w["A"], torch)[:, :self.K] if s == 0 else torch.roll(self.inputs[0][0], shifts=s, dims=1)
+            B = B0 if s == 0 else torch.roll(B0, shifts=s, dims=0)
+            self.inputs.append((A, qg.qgemm_pack_b_s8(B)))
+        del B0, B
+        if per_channel:
+            mult = dev(np.array([p[0] for p in params], np.int32), torch)
+            shift = dev(np.array([p[1] for p in params], np.int32), torch)
+        else:
+            mult, shift = params[0]
+        self.bias = None if w["bias"] is None else dev(w["bias"], torch)
+        self.rq = qg.make_requant(a_zero_point=w["za"], b_zero_point=w["zb"], bias=self.bias,
+                                  multiplier=mult, shift=shift, out_zero_point=w["out_zp"],
+                                  clamp_min=w["clamp_min"], clamp_max=w["clamp_max"])
+        self.C = torch.empty((self.M, self.N), dtype=torch.int8, device="cuda")
+        self.ws = torch.empty(max(qg.qgemm_s8s8_packed_workspace_bytes(self.M, self.K), 1),
+                              dtype=torch.uint8, device="cuda")
+        self.launches = 1 + (1 if (w["lda"] % 16 or w["zb"]) else 0)
+        self.h2d_host = torch.from_numpy(np.ascontiguousarray(w["A"])).pin_memory()
+        self.d2h_host = torch.empty((self.M, self.N), dtype=torch.int8).pin_memory()
+
+    def run(self, i, stream=None):
+        A, pb = self.inputs[i % len(self.inputs)]
+        self.qg.qgemm_s8s8_requant_packed(A, pb, self.N, self.C, self.rq, K=self.K,
+                                          workspace=self.ws, stream=stream)
+
+    def run_e2e(self, i):
+        A, pb = self.inputs[0]
+        dst = self.e2e_A
+        dst.copy_(self.h2d_host, non_blocking=True)
+        self.qg.qgemm_s8s8_requant_packed(dst[:, :self.K], pb, self.N, self.C, self.rq, K=self.K,
+                                          workspace=self.ws)
+        self.d2h_host.copy_(self.C, non_blocking=True)
+
+    def prep_e2e(self):
+        self.e2e_A = self.torch.empty(tuple(self.h2d_host.shape), dtype=self.torch.int8, device="cuda")
+
+    def ops(self):
+        return gemm_ops(self.M, self.N, self.K)
+
+    def bytes(self):
+        return gemm_bytes(self.M, self.N, self.K)
+
+    def h2d(self):
+        return self.h2d_host.numel()
+
+    def d2h(self):
+        return self.d2h_host.numel()
+
+
+class A8W4Case:
+    def __init__(self, qg, torch, w, sets):
+        self.M, self.N, self.K = w["M"], w["N"], w["K"]
+        self.qg, self.torch = qg, torch
+        qw = dev(w["qw"], torch)
+        sw = dev(w["sw"], torch)
+        self.packed = []
+        for s in range(sets):
+            # distinct weight sets: rotate the int4 codes along K (still in [-8,7])
+            src = qw if s == 0 else torch.roll(qw, shifts=32 * s, dims=1)
+            self.packed.append(qg.pack_w4_g32(src, sw))
+        del qw
+        self.x = dev(w["x"], torch)
+        self.bias = None if w["bias"] is None else dev(w["bias"], torch)
+        self.lo, self.hi = w["clamp_min"], w["clamp_max"]
+        self.y = torch.empty((self.M, self.N), dtype=torch.float32, device="cuda")
+        wsb = qg.qgemm_a8w4_workspace_bytes(self.M, self.K)
+        self.ws = torch.empty(max(wsb, 1), dtype=torch.uint8, device="cuda") if wsb else None
+        self.launches = 1 if self.M == 1 else 2
+        self.h2d_host = torch.from_numpy(np.ascontiguousarray(w["x"])).pin_memory()
+        self.d2h_host = torch.empty((self.M, self.N), dtype=torch.float32).pin_memory()
+
+    def run(self, i, stream=None):
+        self.qg.qgemm_a8w4_f32(self.x, self.packed[i % len(self.packed)], self.N, self.bias,
+                               self.lo, self.hi, self.y, workspace=self.ws, stream=stream)
+
+    def prep_e2e(self):
+        self.e2e_x = self.torch.empty(tuple(self.h2d_host.shape), dtype=self.torch.float32, device="cuda")
+
+    def run_e2e(self, i):
+        self.e2e_x.copy_(self.h2d_host, non_blocking=True)
+        self.qg.qgemm_a8w4_f32(self.e2e_x, self.packed[0], self.N, self.bias, self.lo, self.hi,
+                               self.y, workspace=self.ws)
+        self.d2h_host.copy_(self.y, non_blocking=True)
+
+    def ops(self):
+        return a8w4_ops(self.M, self.N, self.K)
+
+    def bytes(self):
+        return a8w4_bytes(self.M, self.N, self.K)
+
+    def h2d(self):
+        return self.h2d_host.numel() * 4
+
+    def d2h(self):
+        return self.d2h_host.numel() * 4
+
+
+class ConvCase:
+    def __init__(self, qg, torch, w, sets):
+        self.qg, self.torch, self.w = qg, torch, w
+        ratios = w["ratio"]
+        params = [qg.qg_requant_params(float(r)) for r in ratios]
+        self.mult = dev(np.array([p[0] for p in params], np.int32), torch)
+        self.shift = dev(np.array([p[1] for p in params], np.int32), torch)
+        self.bias = dev(w["bias"], torch)
+        self.rq = qg.make_requant(a_zero_point=w["za"], bias=self.bias, multiplier=self.mult,
+                                  shift=self.shift, out_zero_point=w["out_zp"],
+                                  clamp_min=w["clamp_min"], clamp_max=w["clamp_max"])
+        self.x = dev(w["x"], torch)
+        self.wt = dev(w["w"], torch)
+        OH, OW = qg.conv_out_hw(w["H"], w["W"], w["KH"], w["KW"], w["stride"], w["pad"])
+        self.y = torch.empty((w["Nb"], OH, OW, w["Cout"]), dtype=torch.int8, device="cuda")
+        self.M, self.N, self.K = w["Nb"] * OH * OW, w["Cout"], w["KH"] * w["KW"] * w["Cin"]
+        self.ws = torch.empty(max(qg.qconv2d_s8_workspace_bytes(self.x.shape, self.wt.shape, w["stride"], w["pad"]), 1),
+                              dtype=torch.uint8, device="cuda")
+        self.launches = 3
+        self.h2d_host = torch.from_numpy(np.ascontiguousarray(w["x"])).pin_memory()
+        self.d2h_host = torch.empty(tuple(self.y.shape), dtype=torch.int8).pin_memory()
+
+    def run(self, i, stream=None):
+        self.qg.qconv2d_s8_im2col(self.x, self.wt, self.y, self.rq, self.w["stride"], self.w["pad"],
+                                  workspace=self.ws, stream=stream)
+
+    def prep_e2e(self):
+        self.e2e_x = self.torch.empty_like(self.x)
+
+    def run_e2e(self, i):
+        self.e2e_x.copy_(self.h2d_host, non_blocking=True)
+        self.qg.qconv2d_s8_im2col(self.e2e_x, self.wt, self.y, self.rq, self.w["stride"],
+                                  self.w["pad"], workspace=self.ws)
+        self.d2h_host.copy_(self.y, non_blocking=True)
+
+    def ops(self):
+        return gemm_ops(self.M, self.N, self.K)
+
+    def bytes(self):
+        w = self.w
+        return self.x.numel() + self.wt.numel() + self.y.numel() + 3 * 4 * self.N
+
+    def h2d(self):
+        return self.h2d_host.numel()
+
+    def d2h(self):
+        return self.d2h_host.numel()
+
+
+def build_cases(workload, qg, torch):
+    import workloads as W
+    if workload == "headline":
+        return [("int8_gemm_8192x8192x8200", GemmCase(qg, torch, W.cfg4_gemm_large(), 2), "tensor"),
+                ("a8w4_gemv_1x14336x4096", A8W4Case(qg, torch, W.cfg2_gemv(), 8), "hbm")]
+    if workload == "cfg0":
+        return [("int8_gemm_130x70x129", GemmCase(qg, torch, W.cfg0_gemm_small(), 1), "latency")]
+    if workload == "cfg1":
+        return [("int8_conv_56x56x64_3x3", ConvCase(qg, torch, W.cfg1_conv(), 1), "latency")]
+    if workload == "cfg2":
+        return [("a8w4_gemv_1x14336x4096", A8W4Case(qg, torch, W.cfg2_gemv(), 8), "hbm")]
+    if workload == "cfg3":
+        return [("a8w4_gemm_128x4096x4096", A8W4Case(qg, torch, W.cfg3_gemm(), 16), "hbm")]
+    if workload == "cfg4":
+        return [("int8_gemm_8192x8192x8200", GemmCase(qg, torch, W.cfg4_gemm_large(), 2), "tensor")]
+    raise SystemExit(f"unknown workload {workload}")
+
+
+# ---------------------------------------------------------------------------
+# ncu traffic figure (committed summary), valid only for the same kernel source
+# ---------------------------------------------------------------------------
+def source_digest():
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "gemv_zero_point_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kernel):
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    digest = source_digest()
+    for line in open(path):
+        f = dict(kv.split("=", 1) for kv in line.split() if "=" in kv)
+        if f.get("kernel") == kernel and f.get("src") == digest:
+            return float(f["bytes_per_launch"])
+    return None
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (bounded sample)
+# ---------------------------------------------------------------------------
+def oracle_sample(workload, budget_s=12.0, rows_gemm=None, small=False):
+    """Time the CPU oracle, as it stands, on a bounded sample of the workload.
+    Returns (ops per second, seconds spent, description)."""
+    import oracle
+    import workloads as W
+    ops, spent, parts = 0.0, 0.0, []
+    if workload in ("headline", "cfg4"):
+        w = W.cfg4_gemm_large()
+        m0 = np.array([oracle.requant_params(float(r))[0] for r in w["ratio"]])
+        sh = np.array([oracle.requant_params(float(r))[1] for r in w["ratio"]])
+        cols = 512 if small else w["N"]
+        rows = 1 if small else (rows_gemm or 2)
+        t = time.perf_counter()
+        oracle.qgemm_s8s8_requant(w["A"][:rows, :w["K"]], w["B"][:, :cols], w["za"], w["zb"],
+                                  w["bias"][:cols], m0[:cols], sh[:cols], w["out_zp"],
+                                  w["clamp_min"], w["clamp_max"])
+        dt = time.perf_counter() - t
+        ops += gemm_ops(rows, cols, w["K"]); spent += dt
+        parts.append(f"int8 GEMM {rows} row(s) x {cols} cols of 8192x8192x8200")
+    if workload in ("headline", "cfg2"):
+        w = W.cfg2_gemv()
+        n = 512 if small else w["N"]
+        t = time.perf_counter()
+        oracle.qgemm_a8w4_f32(w["x"], w["qw"][:n], w["sw"][:n], w["bias"][:n], -6.0, 6.0)
+        dt = time.perf_counter() - t
+        ops += a8w4_ops(1, n, w["K"]); spent += dt
+        parts.append(f"A8W4 GEMV {n} of 14336 rows")
+    if workload == "cfg3":
+        w = W.cfg3_gemm()
+        rows = 1 if small else 4
+        t = time.perf_counter()
+        oracle.qgemm_a8w4_f32(w["x"][:rows], w["qw"], w["sw"], w["bias"], -6.0, 6.0)
+        dt = time.perf_counter() - t
+        ops += a8w4_ops(rows, w["N"], w["K"]); spent += dt
+        parts.append(f"A8W4 GEMM {rows} of 128 rows")
+    if workload == "cfg0":
+        w = W.cfg0_gemm_small()
+        m0, sh = oracle.requant_params(float(w["ratio"][0]))
+        t = time.perf_counter()
+        oracle.qgemm_s8s8_requant(w["A"], w["B"], w["za"], w["zb"], w["bias"], m0, sh,
+                                  w["out_zp"], w["clamp_min"], w["clamp_max"])
+        dt = time.perf_counter() - t
+        ops += gemm_ops(130, 70, 129); spent += dt
+        parts.append("int8 GEMM 130x70x129 (whole)")
+    if workload == "cfg1":
+        w = W.cfg1_conv()
+        pr = [oracle.requant_params(float(r)) for r in w["ratio"]]
+        m0 = np.array([p[0] for p in pr]); sh = np.array([p[1] for p in pr])
+        t = time.perf_counter()
+        oracle.qconv2d_s8(w["x"], w["w"], w["stride"], w["pad"], w["za"], w["bias"], m0, sh,
+                          w["out_zp"], w["clamp_min"], w["clamp_max"])
+        dt = time.perf_counter() - t
+        ops += gemm_ops(3136, 64, 576); spent += dt
+        parts.append("int8 conv 1x56x56x64 3x3 (whole)")
+    return ops / spent, spent, "; ".join(parts)
+
+
+def reference_arm(args, dist):
+    """--impl reference: the oracle as it stands on the host cores, one bounded
+    sample per step, same metric/unit as the GPU arm.  Rank 0 only."""
+    if dist.rank != 0:
+        return
+    total_ops, total_s = 0.0, 0.0
+    desc = ""
+    for i in range(args.warmup + args.steps):
+        rate, spent, desc = oracle_sample(args.workload, small=True)
+        if i >= args.warmup:
+            total_ops += rate * spent
+            total_s += spent
+    value = total_ops / total_s / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TOPS",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * total_s / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+            "config": {"workload": args.workload, "l2": "n/a (CPU)"},
+            "cpu_baseline": {"kind": "oracle", "cores": 1, "value": value, "unit": "TOPS",
+                             "sample": "per step: " + desc},
+            "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="headline",
+                    choices=["headline", "cfg0", "cfg1", "cfg2", "cfg3", "cfg4"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    dist = Dist(args.gpus)
+    if args.impl == "reference":
+        reference_arm(args, dist)
+        dist.close()
+        return
+
+    import torch
+    import gemv_zero_point_b200 as qg
+    torch.cuda.set_device(dist.local)
+    qg.qg_device_status(True)
+    cases = build_cases(args.workload, qg, torch)
+    stream = torch.cuda.current_stream()
+    torch.cuda.synchronize()
+
+    # warm-up
+    for i in range(args.warmup):
+        for _, c, _ in cases:
+            c.run(i)
+    torch.cuda.synchronize()
+
+    # timed region: per-call events plus whole-region events
+    n_calls = len(cases)
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(n_calls)] for _ in range(args.steps)]
+    clocks = Clocks(dist.local)
+    clocks.start()
+    time.sleep(0.3)
+    dist.barrier()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(args.steps):
+        for j, (_, c, _) in enumerate(cases):
+            ev[i][j][0].record(stream)
+            c.run(i + args.warmup)
+            ev[i][j][1].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    dist.barrier()
+    clk = clocks.stop()
+    region_ms = t0.elapsed_time(t1)
+    region_ms = dist.max(region_ms)
+    per_call_ms = [statistics.mean(ev[i][j][0].elapsed_time(ev[i][j][1]) for i in range(args.steps))
+                   for j in range(n_calls)]
+    status = qg.qg_device_status(True)
+    if status != 0:
+        raise SystemExit(f"device status after timed region: {qg.lib.qg_status_string(status).decode()}")
+
+    # end-to-end through the same C ABI with host buffers (pinned), copies timed
+    for _, c, _ in cases:
+        c.prep_e2e()
+    for i in range(2):
+        for _, c, _ in cases:
+            c.run_e2e(i)
+    torch.cuda.synchronize()
+    dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.e2e_steps):
+        for _, c, _ in cases:
+            c.run_e2e(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = dist.max(e0.elapsed_time(e1)) / args.e2e_steps
+
+    step_ops = sum(c.ops() for _, c, _ in cases)
+    ms_per_step = region_ms / args.steps
+    value = dist.world * step_ops / (ms_per_step * 1e-3) / 1e12
+    peaks, peak_src = load_peaks()
+    sustained = region_ms > 1000.0
+    tensor_peak_tops = INT8_OVER_BF16 * (peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"])
+    parts = {}
+    rooflines = {}
+    for j, (name, c, bound) in enumerate(cases):
+        t = per_call_ms[j] * 1e-3
+        part = {"ms": per_call_ms[j], "TOPS": c.ops() / t / 1e12, "GB/s": c.bytes() / t / 1e9,
+                "launches_per_call": c.launches}
+        if bound == "tensor":
+            part["frac_of_int8_peak"] = part["TOPS"] / tensor_peak_tops
+            rooflines[name] = {"bound": "tensor", "achieved": part["TOPS"], "peak": tensor_peak_tops,
+                               "unit": "TOPS", "frac": part["TOPS"] / tensor_peak_tops,
+                               "traffic": traffic_for(name),
+                               "peak_source": f"{peak_src} bf16 {'sustained' if sustained else 'burst'} x {INT8_OVER_BF16:g} (int8/bf16 nominal)"}
+        else:
+            part["frac_of_hbm"] = part["GB/s"] / peaks["hbm_gbs"]
+            rooflines[name] = {"bound": "hbm", "achieved": part["GB/s"], "peak": peaks["hbm_gbs"],
+                               "unit": "GB/s", "frac": part["GB/s"] / peaks["hbm_gbs"],
+                               "traffic": traffic_for(name), "peak_source": f"{peak_src} copy bandwidth"}
+        parts[name] = part
+    dominant = max(range(n_calls), key=lambda j: per_call_ms[j])
+    dom_name = cases[dominant][0]
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": dist.world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
+        "data": "synthetic",
+        "config": {"workload": " + ".join(n for n, _, _ in cases),
+                   "l2": "inputs larger than L2: rotating input sets "
+                         + ", ".join(f"{n}: {len(getattr(c, 'inputs', getattr(c, 'packed', [0])))}"
+                                     for n, c, _ in cases),
+                   "parallelism": f"replicas x{dist.world}"},
+        "parts": parts,
+        "roofline": dict(rooflines[dom_name], kernel=dom_name),
+        "rooflines": rooflines,
+        "gpu_launches": args.steps * sum(c.launches for _, c, _ in cases),
+        "e2e": {"value": dist.world * step_ops / (e2e_ms * 1e-3) / 1e12, "unit": "TOPS",
+                "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": sum(c.h2d() for _, c, _ in cases),
+                "d2h_bytes_per_step": sum(c.d2h() for _, c, _ in cases)},
+        "clocks": clk,
+    }
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        rate, spent, desc = oracle_sample(args.workload)
+        line["cpu_baseline"] = {"value": rate / 1e12, "unit": "TOPS", "cores": 1, "kind": "oracle",
+                                "seconds": spent, "sample": desc}
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+    dist.close()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,67 @@
+"""World-size-2 gloo ranks on CPU exercise the benchmark's multi-rank host
+plumbing (rendezvous, barrier, max-over-ranks timing, reference arm printing
+on rank 0 only).  The hot path itself has no exchange step."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+WORKER = r"""
+import os, sys, json
+sys.path.insert(0, sys.argv[1])
+import bench
+d = bench.Dist(2)
+d.barrier()
+m = d.max(10.0 * (d.rank + 1))
+d.barrier()
+print(json.dumps({"rank": d.rank, "world": d.world, "max": m}), flush=True)
+d.close()
+"""
+
+
+def test_two_rank_barrier_and_max():
+    port = _free_port()
+    procs = []
+    for r in range(2):
+        env = dict(os.environ, RANK=str(r), LOCAL_RANK=str(r), WORLD_SIZE="2",
+                   MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), CUDA_VISIBLE_DEVICES="")
+        procs.append(subprocess.Popen([sys.executable, "-c", WORKER, ROOT], env=env,
+                                      stdout=subprocess.PIPE, stderr=subprocess.PIPE, text=True))
+    outs = [p.communicate(timeout=120) for p in procs]
+    for p, (o, e) in zip(procs, outs):
+        assert p.returncode == 0, e
+    res = sorted((json.loads(o.strip().splitlines()[-1]) for o, _ in outs), key=lambda x: x["rank"])
+    assert [x["world"] for x in res] == [2, 2]
+    assert [x["max"] for x in res] == [20.0, 20.0]
+
+
+def test_reference_arm_prints_on_rank0_only():
+    port = _free_port()
+    procs = []
+    for r in range(2):
+        env = dict(os.environ, RANK=str(r), LOCAL_RANK=str(r), WORLD_SIZE="2",
+                   MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), CUDA_VISIBLE_DEVICES="")
+        procs.append(subprocess.Popen(
+            [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2",
+             "--steps", "1", "--warmup", "3", "--workload", "cfg0"],
+            env=env, stdout=subprocess.PIPE, stderr=subprocess.PIPE, text=True))
+    outs = [p.communicate(timeout=300) for p in procs]
+    for p, (o, e) in zip(procs, outs):
+        assert p.returncode == 0, e
+    line = json.loads(outs[0][0].strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["value"] > 0 and line["unit"] == "TOPS"
+    assert outs[1][0].strip() == ""
