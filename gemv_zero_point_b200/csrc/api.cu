@@ -95,6 +95,9 @@ static int device_ready() {
   return s->setup_rc;
 }
 
+// Per-device set-up status for entry points defined in other files.
+int device_setup_status() { return device_ready(); }
+
 }  // namespace qg
 
 using namespace qg;

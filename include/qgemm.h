@@ -228,6 +228,33 @@ int qgemm_a8w4_f32(int M, int N, int K, const float* x, int64_t ldx,
                    int8_t* q_out, float* scale_out, int32_t* zp_out,
                    void* workspace, size_t workspace_bytes, void* stream);
 
+/* ------------------------------------------------------------------------
+ * qgemm_a8w4_f32 without a workspace.  The pages have no counterpart: this
+ * entry point exists for callers that cannot allocate device memory for
+ * scratch — a plugin inside a host framework that owns the allocator and
+ * exposes none, or a serving loop that must not call cudaMalloc after
+ * start-up because it can synchronise the device.
+ *
+ * Same arguments and results as qgemm_a8w4_f32 (without the optional
+ * quantization outputs).  The scratch (per-row int8 activations, scales and
+ * zero-points) lives in a fixed array in device global memory owned by the
+ * library: 4 MiB + 64 KiB, held on every GPU that loads the library until
+ * the process exits.  Limits: M <= 8192 and M*K <= 4194304 when M > 1;
+ * larger calls return QG_ERR_WORKSPACE and launch nothing.  It never calls
+ * cudaMalloc/cudaFree or any allocating routine.
+ *
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  Every call on a device shares the one array
+ * and each call overwrites every scratch byte it later reads, so nothing
+ * needs clearing — but calls whose work overlaps on the GPU (different
+ * streams, no ordering between them) race on it: order them.
+ * ------------------------------------------------------------------------ */
+int qgemm_a8w4_f32_noalloc(int M, int N, int K, const float* x, int64_t ldx,
+                           const void* packed_w, const float* bias,
+                           float clamp_min, float clamp_max,
+                           float* y, int64_t ldy, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
