@@ -252,7 +252,7 @@ class A8W4Case:
         self.bias = None if w["bias"] is None else dev(w["bias"], torch)
         self.lo, self.hi = w["clamp_min"], w["clamp_max"]
         self.y = torch.empty((self.M, self.N), dtype=torch.float32, device="cuda")
-        wsb = qg.qgemm_a8w4_workspace_bytes(self.M, self.K)
+        wsb = qg.qgemm_a8w4_workspace_bytes(self.M, self.N, self.K)
         self.ws = torch.empty(max(wsb, 1), dtype=torch.uint8, device="cuda") if wsb else None
         self.launches = 1 if self.M == 1 else 2
         self.h2d_host = torch.from_numpy(np.ascontiguousarray(w["x"])).pin_memory()

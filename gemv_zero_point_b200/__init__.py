@@ -85,7 +85,7 @@ _sig("qconv2d_s8_im2col", _i32, [_i32] * 11 + [_vp, _vp, _vp, ctypes.POINTER(Req
 _sig("quantize_rows_a8", _i32, [_i32, _i32, _vp, _i64, _vp, _i64, _vp, _vp, _vp])
 _sig("pack_w4_g32_bytes", _sz, [_i32, _i32])
 _sig("pack_w4_g32", _i32, [_i32, _i32, _vp, _i64, _vp, _vp, _sz, _vp])
-_sig("qgemm_a8w4_workspace_bytes", _sz, [_i32, _i32])
+_sig("qgemm_a8w4_workspace_bytes", _sz, [_i32, _i32, _i32])
 _sig("qgemm_a8w4_f32", _i32, [_i32, _i32, _i32, _vp, _i64, _vp, _vp, _f32, _f32, _vp, _i64,
                               _vp, _vp, _vp, _vp, _sz, _vp])
 
@@ -178,14 +178,14 @@ def pack_w4_g32(w, group_scales, packed=None, stream=None):
     return packed
 
 
-def qgemm_a8w4_workspace_bytes(M, K):
-    return lib.qgemm_a8w4_workspace_bytes(M, K)
+def qgemm_a8w4_workspace_bytes(M, N, K):
+    return lib.qgemm_a8w4_workspace_bytes(M, N, K)
 
 
 def qgemm_a8w4_f32(x, packed_w, N, bias, clamp_min, clamp_max, y, q_out=None, scale_out=None,
                    zp_out=None, workspace=None, stream=None):
     M, K = x.shape
-    wsb = lib.qgemm_a8w4_workspace_bytes(M, K)
+    wsb = lib.qgemm_a8w4_workspace_bytes(M, N, K)
     if wsb and workspace is None:
         workspace = _empty_bytes(wsb, x.device)
     _check(lib.qgemm_a8w4_f32(M, N, K, _p(x), _ld(x), _p(packed_w), _p(bias),

@@ -25,6 +25,13 @@ int launch_a8w4_gemm_simt(int M, int N, int K, const int8_t* q, const float* sA,
 int setup_a8w4_gemv();
 int setup_a8w4_gemm_simt();
 int i8gemm_setup();
+int a8w4_tc_setup();
+bool a8w4_tc_supported(int M, int N, int K);
+int a8w4_tc_splits(int M, int N, int K, int sms);
+size_t a8w4_tc_workspace_bytes(int M, int N, int K, int splits);
+int launch_a8w4_tc(int M, int N, int K, const float* x, int64_t ldx, const void* packed,
+                   const float* bias, float lo, float hi, float* y, int64_t ldy, int8_t* q_out,
+                   float* scale_out, int32_t* zp_out, void* ws, size_t ws_bytes, cudaStream_t st);
 
 int i8gemm_pack_b(int K, int N, const int8_t* B, int64_t ldb, void* packed, cudaStream_t st);
 size_t i8gemm_pack_b_bytes(int K, int N);
@@ -71,6 +78,7 @@ DeviceState* current_state() {
       int rc = setup_a8w4_gemv();
       if (rc == QG_OK) rc = setup_a8w4_gemm_simt();
       if (rc == QG_OK) rc = i8gemm_setup();
+      if (rc == QG_OK) rc = a8w4_tc_setup();
       s.setup_rc = rc;
     }
     s.ready = true;
@@ -333,9 +341,11 @@ static size_t a8w4_ws_layout(int M, int K, size_t* off_scale, size_t* off_zp) {
   return q + s + round_up((int64_t)M * 4, 256);
 }
 
-extern "C" size_t qgemm_a8w4_workspace_bytes(int M, int K) {
-  if (M <= 0 || K <= 0) return 0;
+extern "C" size_t qgemm_a8w4_workspace_bytes(int M, int N, int K) {
+  if (M <= 0 || N <= 0 || K <= 0) return 0;
   if (M == 1 && K <= kFusedGemvMaxK) return 0;
+  if (a8w4_tc_supported(M, N, K))
+    return a8w4_tc_workspace_bytes(M, N, K, a8w4_tc_splits(M, N, K, num_sms()));
   return a8w4_ws_layout(M, K, nullptr, nullptr);
 }
 
@@ -359,6 +369,12 @@ extern "C" int qgemm_a8w4_f32(int M, int N, int K, const float* x, int64_t ldx,
   if (M == 1 && K <= kFusedGemvMaxK)
     return launch_a8w4_gemv(N, K, x, packed_w, bias, clamp_min, clamp_max, y, q_out, scale_out,
                             zp_out, st);
+  if (a8w4_tc_supported(M, N, K)) {
+    if (!workspace) return QG_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return QG_ERR_MISALIGNED;
+    return launch_a8w4_tc(M, N, K, x, ldx, packed_w, bias, clamp_min, clamp_max, y, ldy, q_out,
+                          scale_out, zp_out, workspace, workspace_bytes, st);
+  }
   if (K > kSimtMaxK) return QG_ERR_UNSUPPORTED;
   size_t off_s = 0, off_z = 0;
   const size_t need = a8w4_ws_layout(M, K, &off_s, &off_z);

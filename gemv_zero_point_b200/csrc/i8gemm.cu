@@ -312,6 +312,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   }
 
+  // Reconverge every warp (lane 0 of the TMA and MMA warps ran their loops
+  // alone) so the CTA barrier below counts complete warps only after all
+  // of their work, in particular before TMEM is freed.
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -464,6 +468,25 @@ int make_tmap(CUtensorMap* tm, const void* base, uint64_t cols, uint64_t rows, u
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? QG_OK : QG_ERR_CUDA;
 }
+
+}  // namespace
+
+// Generic 2-D tensor map (any element type), used by the A8W4 tensor-core path.
+int make_tmap_generic(CUtensorMap* tm, CUtensorMapDataType dt, const void* base, uint64_t inner,
+                      uint64_t rows, uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_rows,
+                      CUtensorMapSwizzle swz) {
+  if (get_encode() != QG_OK) return QG_ERR_CUDA;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {pitch_bytes};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(tm, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? QG_OK : QG_ERR_CUDA;
+}
+
+namespace {
 
 struct PackDims {
   int64_t Kp, Np;

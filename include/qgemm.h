@@ -217,10 +217,13 @@ int pack_w4_g32(int N, int K, const int8_t* w, int64_t ldw,
  *   NULL; y: f32 [M][ldy] (ldy >= N).  K % 32 == 0 (else QG_ERR_UNSUPPORTED).
  *   q_out [M][K] int8 / scale_out [M] / zp_out [M]: optional (each may be
  *   NULL), receive the activation quantization for bit-exact checks.
- * M == 1 runs one fused kernel (quantization inside); M > 1 quantizes into
- * the workspace first.
+ * M == 1 runs one fused kernel (quantization inside, no workspace).  M > 1
+ * quantizes into the workspace, then runs the tensor-core kernel (K % 128 == 0
+ * and N % 4 == 0; exact per-group integer dots from bf16 MMAs, f32 group
+ * combination, split-K partials reduced in a fixed order), otherwise a
+ * CUDA-core kernel.
  * ------------------------------------------------------------------------ */
-size_t qgemm_a8w4_workspace_bytes(int M, int K);
+size_t qgemm_a8w4_workspace_bytes(int M, int N, int K);
 int qgemm_a8w4_f32(int M, int N, int K, const float* x, int64_t ldx,
                    const void* packed_w, const float* bias,
                    float clamp_min, float clamp_max,

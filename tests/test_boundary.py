@@ -52,8 +52,8 @@ def test_requant_params_match_oracle_bit_exact():
 def test_workspace_queries():
     assert qg.pack_w4_g32_bytes(14336, 4096) == 14336 * 2048 + 14336 * 128 * 4
     assert qg.pack_w4_g32_bytes(10, 33) == 0          # K % 32 != 0
-    assert qg.qgemm_a8w4_workspace_bytes(1, 4096) == 0  # fused GEMV needs none
-    assert qg.qgemm_a8w4_workspace_bytes(128, 4096) >= 128 * 4096 + 2 * 128 * 4
+    assert qg.qgemm_a8w4_workspace_bytes(1, 14336, 4096) == 0  # fused GEMV needs none
+    assert qg.qgemm_a8w4_workspace_bytes(128, 4096, 4096) >= 128 * 4096 + 2 * 128 * 4
     assert qg.qgemm_pack_b_s8_bytes(129, 70) >= 256 * 256 + 256 * 4
     assert qg.qgemm_s8s8_workspace_bytes(130, 70, 129) >= qg.qgemm_pack_b_s8_bytes(129, 70)
     assert qg.qgemm_pack_b_s8_bytes(0, 5) == 0

@@ -145,7 +145,9 @@ def test_gemv_shapes(lib, N, K, bias, clamp):
     _check_a8w4(lib, w, ldy_pad=2)
 
 
-@pytest.mark.parametrize("M,N,K", [(2, 64, 64), (9, 300, 1024), (17, 1000, 4096), (128, 256, 4096)])
+@pytest.mark.parametrize("M,N,K", [(2, 64, 64), (9, 300, 1024), (17, 1000, 4096), (128, 256, 4096),
+                                   (129, 520, 384), (200, 132, 128), (3, 4096, 8192),
+                                   (256, 8, 2048), (5, 96, 96)])
 def test_a8w4_gemm_shapes(lib, M, N, K):
     w = workloads.a8w4(M, N, K, seed=M * 31 + N + K, clamp=(-np.inf, np.inf), ldx=K + 1)
     _check_a8w4(lib, w, ldy_pad=1)
