@@ -564,8 +564,12 @@ def main():
     ms_per_step = region_ms / args.steps
     value = dist.world * step_ops / (ms_per_step * 1e-3) / 1e12
     peaks, peak_src = load_peaks()
-    sustained = region_ms > 1000.0
-    tensor_peak_tops = INT8_OVER_BF16 * (peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"])
+    # The burst peak describes a GEMM timed alone; once the 1 kW cap engages
+    # (sw_power_cap seen while timing) the sustained figure is the fair one.
+    sustained = region_ms > 1000.0 or bool(clk and "sw_power_cap" in clk.get("reasons", []))
+    tensor_peak_burst = INT8_OVER_BF16 * peaks["bf16_tflops"]
+    tensor_peak_sust = INT8_OVER_BF16 * peaks["bf16_tflops_sustained"]
+    tensor_peak_tops = tensor_peak_sust if sustained else tensor_peak_burst
     parts = {}
     rooflines = {}
     for j, (name, c, bound) in enumerate(cases):
@@ -574,6 +578,8 @@ def main():
                 "launches_per_call": c.launches}
         if bound == "tensor":
             part["frac_of_int8_peak"] = part["TOPS"] / tensor_peak_tops
+            part["frac_of_int8_peak_burst"] = part["TOPS"] / tensor_peak_burst
+            part["frac_of_int8_peak_sustained"] = part["TOPS"] / tensor_peak_sust
             rooflines[name] = {"bound": "tensor", "achieved": part["TOPS"], "peak": tensor_peak_tops,
                                "unit": "TOPS", "frac": part["TOPS"] / tensor_peak_tops,
                                "traffic": traffic_for(name),

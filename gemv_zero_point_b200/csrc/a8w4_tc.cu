@@ -235,7 +235,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       tma_load_2d(sN, &tmW, k0 / 8, n0, nib_full);
       for (int s = 0; s < nstages; ++s) {
         const int slot = s % STAGES;
-        if (s >= STAGES && !mbar_wait(&empty[slot], ((s / STAGES) - 1) & 1, status)) break;
+        if (s >= STAGES && !mbar_poll(&empty[slot], ((s / STAGES) - 1) & 1, status)) break;
         const int kb = (s + rot) % nstages;
         mbar_arrive_expect_tx(&ld_full[slot], (uint32_t)A_STAGE);
         tma_load_2d(sA + slot * A_STAGE, &tmA, k0 + KS * kb, m0, &ld_full[slot]);
@@ -248,7 +248,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int s = 0; s < nstages && ok; ++s) {
         const int slot = s % STAGES;
         const uint32_t par = (uint32_t)(s / STAGES) & 1;
-        if (!mbar_wait(&ld_full[slot], par, status) || !mbar_wait(&cv_full[slot], par, status)) break;
+        if (!mbar_poll(&ld_full[slot], par, status) || !mbar_poll(&cv_full[slot], par, status)) break;
         tc_fence_after();
         const uint32_t a0 = smem_u32(sA + slot * A_STAGE);
         const uint32_t b0 = smem_u32(sB + slot * B_STAGE);
@@ -257,7 +257,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           const int g = 2 * s + gi;
           const int buf = g % NBUF;
           const uint32_t use = (uint32_t)(g / NBUF);
-          if (!mbar_wait(&tempty[buf], (use & 1) ^ 1, status)) {
+          if (!mbar_poll(&tempty[buf], (use & 1) ^ 1, status)) {
             ok = false;
             break;
           }

@@ -193,7 +193,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
         const int tm = t % tiles_m, tn = t / tiles_m;
         for (int kb = 0; kb < num_kb; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1, status)) goto producer_done;
+          if (!mbar_poll(&empty[stage], phase ^ 1, status)) goto producer_done;
           mbar_arrive_expect_tx(&full[stage], A_STAGE + B_STAGE);
           tma_load_2d(sA + stage * A_STAGE, &tmA, kb * BK, tm * BM, &full[stage]);
           tma_load_2d(sB + stage * B_STAGE, &tmB, kb * BK, tn * BN, &full[stage]);
@@ -214,11 +214,11 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++local) {
         const int buf = local & 1;
         const uint32_t use = (uint32_t)(local >> 1);
-        if (!mbar_wait(&tempty[buf], (use & 1) ^ 1, status)) goto mma_done;
+        if (!mbar_poll(&tempty[buf], (use & 1) ^ 1, status)) goto mma_done;
         tc_fence_after();
         const uint32_t d = tmem_base + (uint32_t)(buf * BN);
         for (int kb = 0; kb < num_kb; ++kb) {
-          if (!mbar_wait(&full[stage], phase, status)) goto mma_done;
+          if (!mbar_poll(&full[stage], phase, status)) goto mma_done;
           tc_fence_after();
           const uint32_t a0 = smem_u32(sA + stage * A_STAGE);
           const uint32_t b0 = smem_u32(sB + stage * B_STAGE);

@@ -87,6 +87,29 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* s
   return false;
 }
 
+// Non-blocking variant for single-thread roles (TMA producer, MMA issuer):
+// polls with mbarrier.test_wait, so the thread reacts as soon as the phase
+// completes instead of after a suspension; bounded like mbar_wait.
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ bool mbar_poll(uint64_t* bar, uint32_t parity, int* status) {
+  for (uint32_t i = 0; i < (kSpinLimit << 4); ++i) {
+    if (mbar_test(bar, parity)) return true;
+  }
+  record_error(status, QG_ERR_TIMEOUT);
+  return false;
+}
+
 // ---------------------------------------------------------------------------
 // Bulk copies (TMA engine)
 // ---------------------------------------------------------------------------
