@@ -325,6 +325,270 @@ __global__ void __launch_bounds__(THREADS, 1)
 }
 
 // ---------------------------------------------------------------------------
+// 2-CTA version (cta_group::2).  A cluster of two CTAs on two SMs computes a
+// 256 x 256 tile: CTA rank r stages rows [128r, 128r+128) of the A tile and
+// columns [128r, 128r+128) of the B tile (32 KiB per stage, so 6 stages fit),
+// and its TMEM receives rows [128r, 128r+128) x all 256 columns.  Rank 0 (the
+// leader) issues tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 32); both
+// CTAs' tensor copies complete on the leader's `full` barrier, the leader's
+// commits arrive on both CTAs' `empty` / `tfull` barriers, and both epilogues
+// hand the accumulator back on the leader's `tempty` barrier.  No cluster
+// multicast load is used.
+// ---------------------------------------------------------------------------
+constexpr int P_STAGES = 6;
+constexpr int P_STAGE = BM * BK;  // 16 KiB for the A half, same for the B half
+constexpr size_t P_SMEM_BYTES = 1024 + (size_t)P_STAGES * 2 * P_STAGE + 4096;
+constexpr int P_GROUP_M = 16;     // pair-tile rows per raster group (A slice stays in L2)
+// kind::i8, D s32, A/B s8 K-major, N = 256, M = 256 (the pair)
+constexpr uint32_t IDESC2 = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(256 >> 3) << 17) |
+                            ((uint32_t)(256 >> 4) << 24);
+
+__device__ __forceinline__ uint32_t cluster_rank_u32() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
+__device__ __forceinline__ uint32_t mapa_u32(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+// Tensor copy into this CTA's shared memory whose completion is counted on the
+// (leader's) barrier at cluster address `bar_cluster`.
+__device__ __forceinline__ void tma_load_2d_pair(void* dst_smem, const void* tmap, int32_t x,
+                                                 int32_t y, uint32_t bar_cluster) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst_smem)),
+      "l"(tmap), "r"(x), "r"(y), "r"(bar_cluster)
+      : "memory");
+}
+__device__ __forceinline__ void mma_i8_pair(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(IDESC2), "r"(accumulate)
+      : "memory");
+}
+// Arrive on the barrier at the same offset in both CTAs of the pair once the
+// leader's prior MMAs complete.
+__device__ __forceinline__ void mma_commit_pair(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(smem_u32(bar)),
+      "h"((uint16_t)0x3)
+      : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster)
+               : "memory");
+}
+
+__device__ __forceinline__ void pair_tile_coords(int t, int tiles_m, int tiles_n, int& tm, int& tn) {
+  const int per_group = P_GROUP_M * tiles_n;
+  const int g = t / per_group, r = t % per_group;
+  const int rows = min(P_GROUP_M, tiles_m - g * P_GROUP_M);
+  tm = g * P_GROUP_M + r % rows;
+  tn = r / rows;
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+    i8gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                      int num_kb, int tiles_m, int tiles_n, EpiArgs ep, int* status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + P_STAGES * P_STAGE;
+  uint64_t* full = (uint64_t*)(sB + P_STAGES * P_STAGE);
+  uint64_t* empty = full + P_STAGES;
+  uint64_t* tfull = empty + P_STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint32_t* tmem_slot = (uint32_t*)(tempty + 2);
+  int32_t* c_term = (int32_t*)(tmem_slot + 4);
+  int32_t* c_m0 = c_term + 256;
+  int32_t* c_sh = c_m0 + 256;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank_u32();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int tiles = tiles_m * tiles_n;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < P_STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 8);  // 4 epilogue warps in each CTA of the pair
+    }
+    fence_mbar_init();
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  cluster_sync_all();  // both CTAs' barriers exist before any cross-CTA signal
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------- TMA producer (both CTAs) -------------------------
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int t = pair; t < tiles; t += npairs) {
+        int tm, tn;
+        pair_tile_coords(t, tiles_m, tiles_n, tm, tn);
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_poll(&empty[stage], phase ^ 1, status)) goto producer_done;
+          const uint32_t fb = mapa_u32(smem_u32(&full[stage]), 0);
+          if (leader) mbar_arrive_expect_tx(&full[stage], 2u * 2u * P_STAGE);
+          tma_load_2d_pair(sA + stage * P_STAGE, &tmA, kb * BK, tm * 256 + (int)rank * BM, fb);
+          tma_load_2d_pair(sB + stage * P_STAGE, &tmB, kb * BK, tn * 256 + (int)rank * BM, fb);
+          if (++stage == P_STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+    producer_done:;
+    }
+  } else if (warp == 1) {
+    // ------------------------- MMA issuer (leader only) -------------------------
+    if (leader && lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int local = 0;
+      for (int t = pair; t < tiles; t += npairs, ++local) {
+        const int buf = local & 1;
+        const uint32_t use = (uint32_t)(local >> 1);
+        if (!mbar_poll(&tempty[buf], (use & 1) ^ 1, status)) goto mma_done;
+        tc_fence_after();
+        const uint32_t d = tmem_base + (uint32_t)(buf * BN);
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_poll(&full[stage], phase, status)) goto mma_done;
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + stage * P_STAGE);
+          const uint32_t b0 = smem_u32(sB + stage * P_STAGE);
+#pragma unroll
+          for (int k = 0; k < BK / 32; ++k)
+            mma_i8_pair(d, sdesc_sw128(a0 + 32 * k), sdesc_sw128(b0 + 32 * k), (kb | k) != 0);
+          mma_commit_pair(&empty[stage]);
+          if (++stage == P_STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        mma_commit_pair(&tfull[buf]);
+      }
+    mma_done:;
+    }
+  } else {
+    // ------------------------- epilogue (both CTAs) -------------------------
+    const int q = warp & 3;
+    const int etid = threadIdx.x - 64;
+    const int row_in_tile = 32 * q + lane;
+    const int64_t Kza_zb = (int64_t)ep.K * ep.za * ep.zb;
+    const uint32_t tempty_leader0 = mapa_u32(smem_u32(&tempty[0]), 0);
+    const uint32_t tempty_leader1 = mapa_u32(smem_u32(&tempty[1]), 0);
+    int local = 0;
+    for (int t = pair; t < tiles; t += npairs, ++local) {
+      int tm, tn;
+      pair_tile_coords(t, tiles_m, tiles_n, tm, tn);
+      const int buf = local & 1;
+      const uint32_t use = (uint32_t)(local >> 1);
+      epi_bar_sync();
+      for (int c = etid; c < BN; c += 128) {
+        const int n = tn * BN + c;
+        if (n < ep.N) {
+          const int64_t v = (ep.bias ? (int64_t)ep.bias[n] : 0) -
+                            (int64_t)ep.za * ep.colsum[n] + Kza_zb;
+          c_term[c] = (int32_t)v;
+          c_m0[c] = ep.per_channel ? ep.m0v[n] : ep.m0;
+          c_sh[c] = ep.per_channel ? ep.shv[n] : ep.sh;
+        }
+      }
+      epi_bar_sync();
+      const int m = tm * 256 + (int)rank * BM + row_in_tile;
+      const bool row_ok = m < ep.M;
+      const int32_t r_term = (ep.rowsum && row_ok) ? -ep.zb * ep.rowsum[m] : 0;
+      const bool ok = epi_bar_and(mbar_wait(&tfull[buf], use & 1, status));
+      tc_fence_after();
+      if (ok) {
+        for (int ch = 0; ch < BN / 32; ++ch) {
+          const int nb = tn * BN + ch * 32;
+          if (nb >= ep.N) break;  // warp-uniform
+          uint32_t r[32];
+          tmem_ld32(tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * BN + ch * 32), r);
+          if (!row_ok) continue;
+          const bool full_chunk = nb + 32 <= ep.N;
+          int accv[32];
+          uint32_t packed[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int c = ch * 32 + j;
+            const int a = (int)((uint32_t)r[j] + (uint32_t)c_term[c] + (uint32_t)r_term);
+            accv[j] = a;
+            const int yv = requant1(a, c_m0[c], c_sh[c], ep.zo, ep.lo, ep.hi);
+            packed[j >> 2] |= ((uint32_t)yv & 0xFFu) << (8 * (j & 3));
+          }
+          int8_t* cp = ep.C + (int64_t)m * ep.ldc + nb;
+          if (full_chunk && (((uintptr_t)cp & 15) == 0)) {
+            reinterpret_cast<uint4*>(cp)[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+            reinterpret_cast<uint4*>(cp)[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (nb + j < ep.N) cp[j] = (int8_t)((packed[j >> 2] >> (8 * (j & 3))) & 0xFF);
+          }
+          if (ep.acc_out) {
+            int32_t* ap = ep.acc_out + (int64_t)m * ep.ld_acc + nb;
+            if (full_chunk && (((uintptr_t)ap & 15) == 0)) {
+#pragma unroll
+              for (int j = 0; j < 32; j += 4)
+                reinterpret_cast<int4*>(ap + j)[0] = make_int4(accv[j], accv[j + 1], accv[j + 2], accv[j + 3]);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (nb + j < ep.N) ap[j] = accv[j];
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(buf ? tempty_leader1 : tempty_leader0);
+      if (!ok) break;
+    }
+  }
+
+  // Reconverge every warp, then the whole pair: no CTA leaves while its peer
+  // may still signal its barriers or read its shared memory; then free TMEM.
+  __syncwarp();
+  tc_fence_before();
+  cluster_sync_all();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(TMEM_COLS)
+                 : "memory");
+  }
+}
+
+// ---------------------------------------------------------------------------
 // B pack (row-major B[K][ldb] -> K-major Bp[Np][Kp], zero padded) with the
 // column sums colsum[n] = sum_{k<K} B[k,n].  64x64 tiles through shared memory.
 // ---------------------------------------------------------------------------
@@ -488,6 +752,9 @@ int make_tmap_generic(CUtensorMap* tm, CUtensorMapDataType dt, const void* base,
 
 namespace {
 
+constexpr int kMaxDevices = 64;
+int g_max_pairs[kMaxDevices];  // resident CTA pairs per device, set by i8gemm_setup
+
 struct PackDims {
   int64_t Kp, Np;
 };
@@ -538,6 +805,29 @@ int i8gemm_setup() {
   cudaError_t e = cudaFuncSetAttribute(i8gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)SMEM_BYTES);
   if (e != cudaSuccess) return QG_ERR_CUDA;
+  e = cudaFuncSetAttribute(i8gemm_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)P_SMEM_BYTES);
+  if (e != cudaSuccess) return QG_ERR_CUDA;
+  // how many CTA pairs can be resident at once (SM pairs with a disabled
+  // partner cannot host one)
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return QG_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2);
+  cfg.blockDim = dim3(THREADS);
+  cfg.dynamicSmemBytes = P_SMEM_BYTES;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int clusters = 0;
+  if (cudaOccupancyMaxActiveClusters(&clusters, i8gemm_tc2_kernel, &cfg) != cudaSuccess ||
+      clusters < 1)
+    return QG_ERR_CUDA;
+  g_max_pairs[dev] = clusters;
   return get_encode();
 }
 
@@ -563,10 +853,13 @@ int i8gemm_run_packed(int M, int N, int K, const int8_t* A, int64_t lda, const v
       lda_eff = staged_lda(K);
     }
   }
+  // A pair of CTAs (M > 128) stages half of the B tile per CTA: box of BM rows.
+  const bool pair_path = M > BM;
   CUtensorMap tmA, tmB;
   int rc = make_tmap(&tmA, Aeff, (uint64_t)K, (uint64_t)M, (uint64_t)lda_eff, BM);
   if (rc != QG_OK) return rc;
-  rc = make_tmap(&tmB, packed_b, (uint64_t)d.Kp, (uint64_t)d.Np, (uint64_t)d.Kp, BN);
+  rc = make_tmap(&tmB, packed_b, (uint64_t)d.Kp, (uint64_t)d.Np, (uint64_t)d.Kp,
+                 pair_path ? BM : BN);
   if (rc != QG_OK) return rc;
   EpiArgs ep;
   ep.M = M; ep.N = N; ep.K = K;
@@ -579,10 +872,34 @@ int i8gemm_run_packed(int M, int N, int K, const int8_t* A, int64_t lda, const v
   ep.m0 = rq.multiplier0; ep.sh = rq.shift0;
   ep.m0v = rq.multiplier; ep.shv = rq.shift;
   ep.C = C; ep.ldc = ldc; ep.acc_out = acc_out; ep.ld_acc = ld_acc;
+  const int num_kb = (int)(d.Kp / BK);
+  if (pair_path) {
+    // 2-CTA pairs on 256 x 256 tiles, one resident pair per SM pair
+    const int tiles_m = (int)cdiv(M, 256), tiles_n = (int)cdiv(N, BN);
+    const int tiles = tiles_m * tiles_n;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return QG_ERR_CUDA;
+    int pairs = g_max_pairs[dev] > 0 ? g_max_pairs[dev] : num_sms() / 2;
+    if (pairs > tiles) pairs = tiles;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(2 * pairs));
+    cfg.blockDim = dim3(THREADS);
+    cfg.dynamicSmemBytes = P_SMEM_BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, i8gemm_tc2_kernel, tmA, tmB, num_kb, tiles_m, tiles_n,
+                                       ep, status_word());
+    return e == cudaSuccess ? QG_OK : QG_ERR_CUDA;
+  }
   const int tiles_m = (int)cdiv(M, BM), tiles_n = (int)cdiv(N, BN);
   const int tiles = tiles_m * tiles_n;
   const int grid = tiles < num_sms() ? tiles : num_sms();
-  const int num_kb = (int)(d.Kp / BK);
   i8gemm_tc_kernel<<<grid, THREADS, SMEM_BYTES, st>>>(tmA, tmB, num_kb, tiles_m, tiles_n, ep,
                                                       status_word());
   return launch_status();
