@@ -344,122 +344,122 @@ __global__ void __launch_bounds__(256) a8w4_gemv_kernel(
 }
 
 // ---------------------------------------------------------------------------
-// Fused A8W4 GEMV (M = 1), bulk-copy ring version (K % 128 == 0, K <= 8192).
+// Fused A8W4 GEMV (M = 1), register-pipelined row streaming (K % 128 == 0,
+// K <= 8192).
 //
-// One CTA per SM owns the contiguous rows [n0, n1).  Its producer warp asks
-// the copy engine for whole stages of 16 rows (nibbles and scales, two bulk
-// copies) into a ring of shared-memory slots, so most of the CTA's weight
-// bytes are requested at kernel start and HBM streams at full rate while the
-// 16 consumer warps quantize x.  Consumer warp w then takes row w of every
-// stage: lane l holds the activations of groups l, l+32, ... in registers and
-// reads its 16-byte nibble chunk and scale per group from shared memory.
-// Slots are handed back through per-slot `empty` barriers.
+// One CTA per SM owns the contiguous rows [n0, n1); warp w of W takes rows
+// n0 + w, n0 + w + W, ...  Lane l holds the quantized activations of groups
+// l, l+32, ... in registers and, for every row, loads the matching 16-byte
+// nibble chunk and f32 scale of each of its groups with 128-bit / 32-bit
+// non-coherent loads: each warp instruction reads 512 contiguous bytes.  Each
+// warp keeps D rows of loads in flight in registers: after computing a row it
+// issues the loads of its row D further on into the registers just freed.
+// The weight stream therefore never passes through the copy engine (whose
+// per-request cost bounds small copies) nor through shared memory.
+//
+// Launch overlap.  Launches use programmatic dependent launch.  Packed
+// weights and scales are inputs of the call alone, so every warp issues the
+// loads of its first D rows before waiting for the previous grid; x and bias
+// may be outputs of that grid, so before the wait they are only prefetched
+// into L2 (a prefetch cannot return stale data: L2 is where every write
+// lands).  After the wait one thread copies x into shared memory, where the
+// CTA quantizes it while those weight rows are in flight, and prefetches the
+// rest of the CTA's slice into L2.
 // ---------------------------------------------------------------------------
-constexpr int kRingWarps = 16;  // consumer warps = rows per stage
-constexpr int kRingThreads = (kRingWarps + 1) * 32;
-constexpr int kRingSmemMax = 220 * 1024;
+constexpr int kStreamSmemMax = 96 * 1024;  // x_s + bias_s
 
-__device__ __forceinline__ void consumer_bar() {
-  asm volatile("bar.sync 1, %0;" ::"n"(kRingWarps * 32) : "memory");
+template <int W>
+__device__ __forceinline__ void gemv_bar() {
+  asm volatile("bar.sync 1, %0;" ::"n"(W * 32) : "memory");
 }
 
-template <int GPL>
-__global__ void __launch_bounds__(kRingThreads, 1) a8w4_gemv_ring_kernel(
-    int N, int K, int slots, int max_rows, const float* __restrict__ x,
-    const uint8_t* __restrict__ wq, const float* __restrict__ wscale,
-    const float* __restrict__ bias, float clamp_lo, float clamp_hi, float* __restrict__ y,
-    int8_t* __restrict__ q_out, float* __restrict__ scale_out, int32_t* __restrict__ zp_out,
-    int* status) {
+// L2 prefetch of the 16-byte-aligned interior of [p, p + bytes).
+__device__ __forceinline__ void prefetch_l2_interior(const void* p, int64_t bytes) {
+  uintptr_t a = ((uintptr_t)p + 15) & ~(uintptr_t)15;
+  const uintptr_t e = ((uintptr_t)p + (uintptr_t)bytes) & ~(uintptr_t)15;
+  while (a < e) {
+    const uint32_t c = (uint32_t)min64((int64_t)(e - a), 1 << 20);
+    bulk_prefetch_l2((const void*)a, c);
+    a += c;
+  }
+}
+
+template <int GPL, int W, int D>
+__global__ void __launch_bounds__(W * 32, 1) a8w4_gemv_stream_kernel(
+    int N, int K, int max_rows, const float* __restrict__ x, const uint8_t* __restrict__ wq,
+    const float* __restrict__ wscale, const float* __restrict__ bias, float clamp_lo,
+    float clamp_hi, float* __restrict__ y, int8_t* __restrict__ q_out,
+    float* __restrict__ scale_out, int32_t* __restrict__ zp_out, int* status) {
   extern __shared__ __align__(128) uint8_t sm[];
-  __shared__ float red[2 * kRingWarps];
+  __shared__ float red[2 * W];
+  __shared__ __align__(8) uint64_t xfull;  // x has landed in x_s
   const int G = K >> 5;
   const int rowbytes = K >> 1;
-  const int sclbytes = G * 4;
-  const int stage_bytes = kRingWarps * (rowbytes + sclbytes);
-  int8_t* qa_s = reinterpret_cast<int8_t*>(sm);
-  float* bias_s = reinterpret_cast<float*>(sm + ((K + 127) & ~127));  // [max_rows]
-  uint8_t* ring = sm + ((K + 127) & ~127) + ((max_rows * 4 + 127) & ~127);
-  uint64_t* full = reinterpret_cast<uint64_t*>(ring + (size_t)slots * stage_bytes);
-  uint64_t* empty = full + slots;
-  uint64_t* xfull = empty + slots;   // x has landed in x_s
-  uint64_t* xfree = xfull + 1;       // every consumer warp has read x_s
-  // x (4K bytes) borrows the last ring slot until the consumers hold it in
-  // registers; that slot's first stage is requested afterwards.
-  const int xslot = slots - 1;
-  const float* x_s = reinterpret_cast<const float*>(ring + (size_t)xslot * stage_bytes);
+  float* x_s = reinterpret_cast<float*>(sm);             // [K] f32 as copied in
+  int8_t* qa_s = reinterpret_cast<int8_t*>(sm);          // [K] quantized x, over x_s
+  float* bias_s = reinterpret_cast<float*>(sm + 4 * K);  // [max_rows]
 
   const int n0 = (int)((int64_t)blockIdx.x * N / gridDim.x);
   const int n1 = (int)((int64_t)(blockIdx.x + 1) * N / gridDim.x);
-  const int nstages = (n1 - n0 + kRingWarps - 1) / kRingWarps;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nrows = n1 - n0 > warp ? (n1 - n0 - warp + W - 1) / W : 0;  // this warp's rows
+
+  uint4 wbuf[D][GPL];
+  float sbuf[D][GPL];
+  // loads of this warp's row j into buffer u (nothing past the last row)
+  auto load_row = [&](int u, int j) {
+    if (j < nrows) {
+      const int r = n0 + warp + W * j;
+#pragma unroll
+      for (int i = 0; i < GPL; ++i) {
+        const int g = lane + 32 * i;
+        if (g < G) {
+          wbuf[u][i] = ld_stream_u4(wq + (int64_t)r * rowbytes + 16 * g);
+          sbuf[u][i] = ld_stream_f32(wscale + (int64_t)r * G + g);
+        }
+      }
+    }
+  };
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < slots; ++i) {
-      mbar_init(&full[i], 1);
-      mbar_init(&empty[i], kRingWarps);
-    }
-    mbar_init(xfull, 1);
-    mbar_init(xfree, kRingWarps);
+    mbar_init(&xfull, 1);
     fence_mbar_init();
-    // Stage this CTA's weight slice into L2 before waiting on the previous
-    // grid: a prefetch cannot return stale data (L2 is where every write
-    // lands), and the copies that feed the math are issued after the wait.
-    if (n1 > n0) {
-      const uint8_t* p = wq + (int64_t)n0 * rowbytes;
-      int64_t bytes = (int64_t)(n1 - n0) * rowbytes;
-      while (bytes > 0) {
-        const uint32_t c = (uint32_t)min64(bytes, 1 << 20);
-        bulk_prefetch_l2(p, c);
-        p += c;
-        bytes -= c;
-      }
-      bulk_prefetch_l2(wscale + (int64_t)n0 * G, (uint32_t)((n1 - n0) * sclbytes));
-    }
+    prefetch_l2_interior(x, (int64_t)K * 4);
+    if (bias && n1 > n0) prefetch_l2_interior(bias + n0, (int64_t)(n1 - n0) * 4);
   }
+#pragma unroll
+  for (int u = 0; u < D; ++u) load_row(u, u);
+  __syncthreads();
   // Programmatic dependent launch: let the next grid in the stream start its
   // own prologue, then wait until the previous grid's writes are visible.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  __syncthreads();
 
-  if (warp == kRingWarps) {
-    // ---------------- producer ----------------
-    if (lane == 0) {
-      mbar_arrive_expect_tx(xfull, (uint32_t)(K * 4));
-      bulk_g2s(const_cast<float*>(x_s), x, (uint32_t)(K * 4), xfull);
-      for (int s = 0; s < nstages; ++s) {
-        const int slot = s % slots;
-        if (s == xslot && !mbar_wait(xfree, 0, status)) break;
-        if (s >= slots && !mbar_wait(&empty[slot], ((s / slots) - 1) & 1, status)) break;
-        const int r0 = n0 + kRingWarps * s;
-        const int rows = min(kRingWarps, n1 - r0);
-        uint8_t* dst = ring + (size_t)slot * stage_bytes;
-        mbar_arrive_expect_tx(&full[slot], (uint32_t)(rows * (rowbytes + sclbytes)));
-        bulk_g2s(dst, wq + (int64_t)r0 * rowbytes, (uint32_t)(rows * rowbytes), &full[slot]);
-        bulk_g2s(dst + kRingWarps * rowbytes, wscale + (int64_t)r0 * G,
-                 (uint32_t)(rows * sclbytes), &full[slot]);
-      }
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(&xfull, (uint32_t)(K * 4));
+    bulk_g2s(x_s, x, (uint32_t)(K * 4), &xfull);
+    const int r_rest = n0 + W * D;  // rows beyond the ones already requested
+    if (r_rest < n1) {
+      prefetch_l2_interior(wq + (int64_t)r_rest * rowbytes, (int64_t)(n1 - r_rest) * rowbytes);
+      prefetch_l2_interior(wscale + (int64_t)r_rest * G, (int64_t)(n1 - r_rest) * G * 4);
     }
-    return;
   }
 
-  // ---------------- consumers: quantize x ----------------
-  for (int i = threadIdx.x; i < n1 - n0; i += kRingWarps * 32)
+  // ---------------- quantize x ----------------
+  for (int i = threadIdx.x; i < n1 - n0; i += W * 32)
     bias_s[i] = bias ? bias[n0 + i] : 0.0f;
   // Each thread takes its float4 chunks of x from shared memory once and keeps
   // them in registers for both passes (K <= 1024*GPL).
-  constexpr int XV = (GPL * 1024 + 4 * kRingWarps * 32 - 1) / (4 * kRingWarps * 32);
+  constexpr int XV = (GPL * 1024 + 4 * W * 32 - 1) / (4 * W * 32);
   float4 xv[XV];
   float mn = 0.0f, mx = 0.0f;
-  const bool x_ok = mbar_wait(xfull, 0, status);
+  const bool x_ok = mbar_wait(&xfull, 0, status);
 #pragma unroll
   for (int j = 0; j < XV; ++j) {
-    const int c = threadIdx.x + j * kRingWarps * 32;  // float4 chunk index
+    const int c = threadIdx.x + j * W * 32;  // float4 chunk index
     xv[j] = (x_ok && 4 * c < K) ? reinterpret_cast<const float4*>(x_s)[c]
                                 : make_float4(0.f, 0.f, 0.f, 0.f);
   }
-  __syncwarp();
-  if (lane == 0) mbar_arrive(xfree);   // x_s may now be overwritten by its stage
 #pragma unroll
   for (int j = 0; j < XV; ++j) {
     mn = fminf(mn, fminf(fminf(xv[j].x, xv[j].y), fminf(xv[j].z, xv[j].w)));
@@ -471,20 +471,20 @@ __global__ void __launch_bounds__(kRingThreads, 1) a8w4_gemv_ring_kernel(
   }
   if (lane == 0) {
     red[warp] = mn;
-    red[kRingWarps + warp] = mx;
+    red[W + warp] = mx;
   }
-  consumer_bar();
+  gemv_bar<W>();  // also: every x_s read is done before qa_s overwrites it
   mn = red[0];
-  mx = red[kRingWarps];
+  mx = red[W];
 #pragma unroll
-  for (int i = 1; i < kRingWarps; ++i) {
+  for (int i = 1; i < W; ++i) {
     mn = fminf(mn, red[i]);
-    mx = fmaxf(mx, red[kRingWarps + i]);
+    mx = fmaxf(mx, red[W + i]);
   }
   const RowQuant rq = row_quant_params(mn, mx);
 #pragma unroll
   for (int j = 0; j < XV; ++j) {
-    const int c = threadIdx.x + j * kRingWarps * 32;
+    const int c = threadIdx.x + j * W * 32;
     if (4 * c < K) {
       const uint32_t b0 = (uint32_t)quant_one(xv[j].x, rq) & 0xFFu;
       const uint32_t b1 = (uint32_t)quant_one(xv[j].y, rq) & 0xFFu;
@@ -501,7 +501,7 @@ __global__ void __launch_bounds__(kRingThreads, 1) a8w4_gemv_ring_kernel(
     if (scale_out) scale_out[0] = rq.scale;
     if (zp_out) zp_out[0] = rq.zp;
   }
-  consumer_bar();
+  gemv_bar<W>();
 
   const int za = rq.zp;
   int a[GPL][8];
@@ -522,56 +522,44 @@ __global__ void __launch_bounds__(kRingThreads, 1) a8w4_gemv_ring_kernel(
     }
   }
 
-  // ---------------- consumers: stream rows ----------------
-  for (int s = 0; s < nstages; ++s) {
-    const int slot = s % slots;
-    if (!mbar_wait(&full[slot], (s / slots) & 1, status)) break;
-    const int r = n0 + kRingWarps * s + warp;
-    if (r < n1) {
-      const uint8_t* nib = ring + (size_t)slot * stage_bytes + warp * rowbytes;
-      const float* scl = reinterpret_cast<const float*>(ring + (size_t)slot * stage_bytes +
-                                                        kRingWarps * rowbytes + warp * sclbytes);
-      float acc = 0.0f;
+  // ---------------- stream this warp's rows ----------------
+  for (int j0 = 0; j0 < nrows; j0 += D) {
 #pragma unroll
-      for (int i = 0; i < GPL; ++i) {
-        const int g = lane + 32 * i;
-        if (g < G) {
-          const uint4 wv = *reinterpret_cast<const uint4*>(nib + 16 * g);
-          acc = fmaf(scl[g], (float)group_dot(wv, a[i], cseed[i], za), acc);
+    for (int u = 0; u < D; ++u) {
+      const int j = j0 + u;
+      if (j < nrows) {
+        float acc = 0.0f;
+#pragma unroll
+        for (int i = 0; i < GPL; ++i) {
+          const int g = lane + 32 * i;
+          if (g < G) acc = fmaf(sbuf[u][i], (float)group_dot(wbuf[u][i], a[i], cseed[i], za), acc);
+        }
+        load_row(u, j + D);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (lane == 0) {
+          const int r = n0 + warp + W * j;
+          float v = __fmul_rn(rq.scale, acc);
+          if (bias) v = __fadd_rn(v, bias_s[r - n0]);
+          y[r] = fminf(fmaxf(v, clamp_lo), clamp_hi);
         }
       }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-      if (lane == 0) {
-        float v = __fmul_rn(rq.scale, acc);
-        if (bias) v = __fadd_rn(v, bias_s[r - n0]);
-        y[r] = fminf(fmaxf(v, clamp_lo), clamp_hi);
-      }
     }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[slot]);
   }
 }
 
-template <int GPL>
-static int launch_ring(int N, int K, const float* x, const uint8_t* wq, const float* ws,
-                       const float* bias, float lo, float hi, float* y, int8_t* q_out,
-                       float* scale_out, int32_t* zp_out, cudaStream_t st) {
-  const int G = K / 32;
-  const int stage_bytes = kRingWarps * (K / 2 + G * 4);
+template <int GPL, int W, int D>
+static int launch_stream(int N, int K, const float* x, const uint8_t* wq, const float* ws,
+                         const float* bias, float lo, float hi, float* y, int8_t* q_out,
+                         float* scale_out, int32_t* zp_out, cudaStream_t st) {
   int grid = num_sms();
-  const int max_grid = (N + kRingWarps - 1) / kRingWarps;
-  if (grid > max_grid) grid = max_grid;
+  if (grid > N) grid = N;
   const int rows_per_cta = (N + grid - 1) / grid;
-  const int nstages = (rows_per_cta + kRingWarps - 1) / kRingWarps;
-  const int base = ((K + 127) & ~127) + ((rows_per_cta * 4 + 127) & ~127);
-  int slots = (kRingSmemMax - base - 16) / (stage_bytes + 16);
-  if (slots > nstages) slots = nstages;
-  if (slots < 1) return 1;  // does not fit: caller uses the register-streaming kernel
-  const size_t smem = (size_t)base + (size_t)slots * (stage_bytes + 16) + 16;
+  const size_t smem = (size_t)4 * K + (size_t)rows_per_cta * 4;  // x_s, bias_s
+  if (smem > (size_t)kStreamSmemMax) return 1;  // caller uses the plain kernel
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kRingThreads);
+  cfg.blockDim = dim3(W * 32);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -579,8 +567,8 @@ static int launch_ring(int N, int K, const float* x, const uint8_t* wq, const fl
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, a8w4_gemv_ring_kernel<GPL>, N, K, slots, rows_per_cta, x,
-                                     wq, ws, bias, lo, hi, y, q_out, scale_out, zp_out,
+  cudaError_t e = cudaLaunchKernelEx(&cfg, a8w4_gemv_stream_kernel<GPL, W, D>, N, K, rows_per_cta,
+                                     x, wq, ws, bias, lo, hi, y, q_out, scale_out, zp_out,
                                      status_word());
   return e == cudaSuccess ? QG_OK : QG_ERR_CUDA;
 }
@@ -595,10 +583,10 @@ int launch_a8w4_gemv(int N, int K, const float* x, const void* packed, const flo
   if (grid > N) grid = N;
   if (K % 128 == 0 && K <= 8192 && ((uintptr_t)x & 15) == 0) {
     int rc;
-    if (G <= 32) rc = launch_ring<1>(N, K, x, wq, ws, bias, lo, hi, y, q_out, scale_out, zp_out, st);
-    else if (G <= 64) rc = launch_ring<2>(N, K, x, wq, ws, bias, lo, hi, y, q_out, scale_out, zp_out, st);
-    else if (G <= 128) rc = launch_ring<4>(N, K, x, wq, ws, bias, lo, hi, y, q_out, scale_out, zp_out, st);
-    else rc = launch_ring<8>(N, K, x, wq, ws, bias, lo, hi, y, q_out, scale_out, zp_out, st);
+    if (G <= 32) rc = launch_stream<1, 16, 3>(N, K, x, wq, ws, bias, lo, hi, y, q_out, scale_out, zp_out, st);
+    else if (G <= 64) rc = launch_stream<2, 16, 3>(N, K, x, wq, ws, bias, lo, hi, y, q_out, scale_out, zp_out, st);
+    else if (G <= 128) rc = launch_stream<4, 16, 3>(N, K, x, wq, ws, bias, lo, hi, y, q_out, scale_out, zp_out, st);
+    else rc = launch_stream<8, 8, 3>(N, K, x, wq, ws, bias, lo, hi, y, q_out, scale_out, zp_out, st);
     if (rc <= 0) return rc;
   }
   const size_t smem = (size_t)K;
@@ -623,14 +611,14 @@ int setup_a8w4_gemv() {
                                         cudaFuncAttributeMaxDynamicSharedMemorySize, 65536);
   cudaError_t e3 = cudaFuncSetAttribute(a8w4_gemv_kernel<4>,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize, 65536);
-  cudaError_t e4 = cudaFuncSetAttribute(a8w4_gemv_ring_kernel<1>,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kRingSmemMax);
-  cudaError_t e5 = cudaFuncSetAttribute(a8w4_gemv_ring_kernel<2>,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kRingSmemMax);
-  cudaError_t e6 = cudaFuncSetAttribute(a8w4_gemv_ring_kernel<4>,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kRingSmemMax);
-  cudaError_t e7 = cudaFuncSetAttribute(a8w4_gemv_ring_kernel<8>,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kRingSmemMax);
+  cudaError_t e4 = cudaFuncSetAttribute(a8w4_gemv_stream_kernel<1, 16, 3>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmemMax);
+  cudaError_t e5 = cudaFuncSetAttribute(a8w4_gemv_stream_kernel<2, 16, 3>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmemMax);
+  cudaError_t e6 = cudaFuncSetAttribute(a8w4_gemv_stream_kernel<4, 16, 3>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmemMax);
+  cudaError_t e7 = cudaFuncSetAttribute(a8w4_gemv_stream_kernel<8, 8, 3>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmemMax);
   return (e1 == cudaSuccess && e2 == cudaSuccess && e3 == cudaSuccess && e4 == cudaSuccess &&
           e5 == cudaSuccess && e6 == cudaSuccess && e7 == cudaSuccess)
              ? QG_OK

@@ -217,7 +217,11 @@ int pack_w4_g32(int N, int K, const int8_t* w, int64_t ldw,
  *   NULL; y: f32 [M][ldy] (ldy >= N).  K % 32 == 0 (else QG_ERR_UNSUPPORTED).
  *   q_out [M][K] int8 / scale_out [M] / zp_out [M]: optional (each may be
  *   NULL), receive the activation quantization for bit-exact checks.
- * M == 1 runs one fused kernel (quantization inside, no workspace).  M > 1
+ * M == 1 runs one fused kernel (quantization inside, no workspace), launched
+ * so that it may start while the previous M == 1 call on the same stream is
+ * still finishing: it reads packed_w (never x or bias) before that call has
+ * completed.  So packed_w must not be written by the M == 1 call just before
+ * it on the stream; every other ordering is kept as usual.  M > 1
  * quantizes into the workspace, then runs the tensor-core kernel (K % 128 == 0
  * and N % 4 == 0; exact per-group integer dots from bf16 MMAs, f32 group
  * combination, split-K partials reduced in a fixed order), otherwise a
