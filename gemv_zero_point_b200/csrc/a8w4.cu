@@ -347,8 +347,12 @@ __global__ void __launch_bounds__(256) a8w4_gemv_kernel(
 // Fused A8W4 GEMV (M = 1), register-pipelined row streaming (K % 128 == 0,
 // K <= 8192).
 //
-// One CTA per SM owns the contiguous rows [n0, n1); warp w of W takes rows
-// n0 + w, n0 + w + W, ...  Lane l holds the quantized activations of groups
+// One CTA per SM owns the contiguous rows [n0, n1).  The first W * nfull
+// rows (nfull = (n1 - n0) / W) go round-robin to the W warps; each of the
+// L < W rows left over is split by groups across GPL warps (warp w takes
+// slot w % GPL of every lane) and their partial sums meet in shared memory,
+// so no warp finishes a whole extra row alone (14336 rows over 148 SMs give
+// 96 or 97 rows per CTA: 6 per warp plus at most one split row).  Lane l holds the quantized activations of groups
 // l, l+32, ... in registers and, for every row, loads the matching 16-byte
 // nibble chunk and f32 scale of each of its groups with 128-bit / 32-bit
 // non-coherent loads: each warp instruction reads 512 contiguous bytes.  Each
@@ -392,6 +396,7 @@ __global__ void __launch_bounds__(W * 32, 1) a8w4_gemv_stream_kernel(
     float* __restrict__ scale_out, int32_t* __restrict__ zp_out, int* status) {
   extern __shared__ __align__(128) uint8_t sm[];
   __shared__ float red[2 * W];
+  __shared__ float part_s[W * GPL];        // partial sums of the split rows
   __shared__ __align__(8) uint64_t xfull;  // x has landed in x_s
   const int G = K >> 5;
   const int rowbytes = K >> 1;
@@ -402,7 +407,10 @@ __global__ void __launch_bounds__(W * 32, 1) a8w4_gemv_stream_kernel(
   const int n0 = (int)((int64_t)blockIdx.x * N / gridDim.x);
   const int n1 = (int)((int64_t)(blockIdx.x + 1) * N / gridDim.x);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nrows = n1 - n0 > warp ? (n1 - n0 - warp + W - 1) / W : 0;  // this warp's rows
+  const int nrows = (n1 - n0) / W;         // whole rows per warp
+  const int nleft = n1 - n0 - W * nrows;   // rows split across warps
+  const int slot = warp % GPL;             // this warp's slot in a split row
+  static_assert(W % GPL == 0, "split rows need W to be a multiple of GPL");
 
   uint4 wbuf[D][GPL];
   float sbuf[D][GPL];
@@ -429,6 +437,18 @@ __global__ void __launch_bounds__(W * 32, 1) a8w4_gemv_stream_kernel(
   }
 #pragma unroll
   for (int u = 0; u < D; ++u) load_row(u, u);
+  // the first split row this warp takes part in
+  uint4 wsplit = make_uint4(0, 0, 0, 0);
+  float ssplit = 0.0f;
+  auto load_split = [&](int k) {
+    const int r = n0 + W * nrows + k;
+    const int g = lane + 32 * slot;
+    if (g < G) {
+      wsplit = ld_stream_u4(wq + (int64_t)r * rowbytes + 16 * g);
+      ssplit = ld_stream_f32(wscale + (int64_t)r * G + g);
+    }
+  };
+  if (warp / GPL < nleft) load_split(warp / GPL);
   __syncthreads();
   // Programmatic dependent launch: let the next grid in the stream start its
   // own prologue, then wait until the previous grid's writes are visible.
@@ -436,9 +456,14 @@ __global__ void __launch_bounds__(W * 32, 1) a8w4_gemv_stream_kernel(
   asm volatile("griddepcontrol.wait;" ::: "memory");
 
   if (threadIdx.x == 0) {
+    // x in four chunks, in an order rotated by CTA, so that the CTAs do not
+    // all ask the same L2 lines for x at the same moment
     mbar_arrive_expect_tx(&xfull, (uint32_t)(K * 4));
-    bulk_g2s(x_s, x, (uint32_t)(K * 4), &xfull);
-    const int r_rest = n0 + W * D;  // rows beyond the ones already requested
+    for (int c = 0; c < 4; ++c) {
+      const int q = (c + blockIdx.x) & 3;
+      bulk_g2s(x_s + q * (K / 4), x + q * (K / 4), (uint32_t)K, &xfull);
+    }
+    const int r_rest = n0 + W * min(D, nrows);  // rows beyond the ones already requested
     if (r_rest < n1) {
       prefetch_l2_interior(wq + (int64_t)r_rest * rowbytes, (int64_t)(n1 - r_rest) * rowbytes);
       prefetch_l2_interior(wscale + (int64_t)r_rest * G, (int64_t)(n1 - r_rest) * G * 4);
@@ -546,6 +571,32 @@ __global__ void __launch_bounds__(W * 32, 1) a8w4_gemv_stream_kernel(
       }
     }
   }
+
+  // ---------------- split rows ----------------
+  if (nleft > 0) {  // uniform across the CTA
+    for (int k = warp / GPL; k < nleft; k += W / GPL) {
+      if (k != warp / GPL) load_split(k);
+      float part = 0.0f;
+      const int g = lane + 32 * slot;
+#pragma unroll
+      for (int i = 0; i < GPL; ++i)  // static register indexing of a[slot]
+        if (i == slot && g < G) part = __fmul_rn(ssplit, (float)group_dot(wsplit, a[i], cseed[i], za));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+      if (lane == 0) part_s[k * GPL + slot] = part;
+    }
+    gemv_bar<W>();
+    if (threadIdx.x < nleft) {
+      const int k = threadIdx.x;
+      float acc = part_s[k * GPL];
+#pragma unroll
+      for (int i = 1; i < GPL; ++i) acc += part_s[k * GPL + i];
+      const int r = n0 + W * nrows + k;
+      float v = __fmul_rn(rq.scale, acc);
+      if (bias) v = __fadd_rn(v, bias_s[r - n0]);
+      y[r] = fminf(fmaxf(v, clamp_lo), clamp_hi);
+    }
+  }
 }
 
 template <int GPL, int W, int D>
@@ -585,7 +636,7 @@ int launch_a8w4_gemv(int N, int K, const float* x, const void* packed, const flo
     int rc;
     if (G <= 32) rc = launch_stream<1, 16, 3>(N, K, x, wq, ws, bias, lo, hi, y, q_out, scale_out, zp_out, st);
     else if (G <= 64) rc = launch_stream<2, 16, 3>(N, K, x, wq, ws, bias, lo, hi, y, q_out, scale_out, zp_out, st);
-    else if (G <= 128) rc = launch_stream<4, 16, 3>(N, K, x, wq, ws, bias, lo, hi, y, q_out, scale_out, zp_out, st);
+    else if (G <= 128) rc = launch_stream<4, 16, 2>(N, K, x, wq, ws, bias, lo, hi, y, q_out, scale_out, zp_out, st);
     else rc = launch_stream<8, 8, 3>(N, K, x, wq, ws, bias, lo, hi, y, q_out, scale_out, zp_out, st);
     if (rc <= 0) return rc;
   }
@@ -615,7 +666,7 @@ int setup_a8w4_gemv() {
                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmemMax);
   cudaError_t e5 = cudaFuncSetAttribute(a8w4_gemv_stream_kernel<2, 16, 3>,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmemMax);
-  cudaError_t e6 = cudaFuncSetAttribute(a8w4_gemv_stream_kernel<4, 16, 3>,
+  cudaError_t e6 = cudaFuncSetAttribute(a8w4_gemv_stream_kernel<4, 16, 2>,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmemMax);
   cudaError_t e7 = cudaFuncSetAttribute(a8w4_gemv_stream_kernel<8, 8, 3>,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmemMax);
