@@ -372,6 +372,18 @@ __global__ void __launch_bounds__(256) a8w4_gemv_kernel(
 // ---------------------------------------------------------------------------
 constexpr int kStreamSmemMax = 96 * 1024;  // x_s + bias_s
 
+// Warp-wide float min / max (NaN inputs ignored, as fminf / fmaxf do).
+__device__ __forceinline__ float warp_min(float v) {
+  float r;
+  asm volatile("redux.sync.min.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+  return r;
+}
+__device__ __forceinline__ float warp_max(float v) {
+  float r;
+  asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+  return r;
+}
+
 template <int W>
 __device__ __forceinline__ void gemv_bar() {
   asm volatile("bar.sync 1, %0;" ::"n"(W * 32) : "memory");
@@ -490,22 +502,16 @@ __global__ void __launch_bounds__(W * 32, 1) a8w4_gemv_stream_kernel(
     mn = fminf(mn, fminf(fminf(xv[j].x, xv[j].y), fminf(xv[j].z, xv[j].w)));
     mx = fmaxf(mx, fmaxf(fmaxf(xv[j].x, xv[j].y), fmaxf(xv[j].z, xv[j].w)));
   }
-  for (int o = 16; o > 0; o >>= 1) {
-    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  }
+  mn = warp_min(mn);
+  mx = warp_max(mx);
   if (lane == 0) {
     red[warp] = mn;
     red[W + warp] = mx;
   }
   gemv_bar<W>();  // also: every x_s read is done before qa_s overwrites it
-  mn = red[0];
-  mx = red[W];
-#pragma unroll
-  for (int i = 1; i < W; ++i) {
-    mn = fminf(mn, red[i]);
-    mx = fmaxf(mx, red[W + i]);
-  }
+  // every warp combines the W per-warp results (lanes past W repeat warp 0's)
+  mn = warp_min(red[lane < W ? lane : 0]);
+  mx = warp_max(red[W + (lane < W ? lane : 0)]);
   const RowQuant rq = row_quant_params(mn, mx);
 #pragma unroll
   for (int j = 0; j < XV; ++j) {
