@@ -367,8 +367,8 @@ __global__ void __launch_bounds__(256) a8w4_gemv_kernel(
 // may be outputs of that grid, so before the wait they are only prefetched
 // into L2 (a prefetch cannot return stale data: L2 is where every write
 // lands).  After the wait one thread copies x into shared memory, where the
-// CTA quantizes it while those weight rows are in flight, and prefetches the
-// rest of the CTA's slice into L2.
+// CTA quantizes it while those weight rows are in flight; once x has landed
+// the rest of the CTA's slice is prefetched into L2.
 // ---------------------------------------------------------------------------
 constexpr int kStreamSmemMax = 96 * 1024;  // x_s + bias_s
 
@@ -475,11 +475,6 @@ __global__ void __launch_bounds__(W * 32, 1) a8w4_gemv_stream_kernel(
       const int q = (c + blockIdx.x) & 3;
       bulk_g2s(x_s + q * (K / 4), x + q * (K / 4), (uint32_t)K, &xfull);
     }
-    const int r_rest = n0 + W * min(D, nrows);  // rows beyond the ones already requested
-    if (r_rest < n1) {
-      prefetch_l2_interior(wq + (int64_t)r_rest * rowbytes, (int64_t)(n1 - r_rest) * rowbytes);
-      prefetch_l2_interior(wscale + (int64_t)r_rest * G, (int64_t)(n1 - r_rest) * G * 4);
-    }
   }
 
   // ---------------- quantize x ----------------
@@ -491,6 +486,15 @@ __global__ void __launch_bounds__(W * 32, 1) a8w4_gemv_stream_kernel(
   float4 xv[XV];
   float mn = 0.0f, mx = 0.0f;
   const bool x_ok = mbar_wait(&xfull, 0, status);
+  if (threadIdx.x == 0) {
+    // the rest of the slice into L2, queued only once x (on the critical
+    // path) has landed
+    const int r_rest = n0 + W * min(D, nrows);  // rows beyond the ones already requested
+    if (r_rest < n1) {
+      prefetch_l2_interior(wq + (int64_t)r_rest * rowbytes, (int64_t)(n1 - r_rest) * rowbytes);
+      prefetch_l2_interior(wscale + (int64_t)r_rest * G, (int64_t)(n1 - r_rest) * G * 4);
+    }
+  }
 #pragma unroll
   for (int j = 0; j < XV; ++j) {
     const int c = threadIdx.x + j * W * 32;  // float4 chunk index
