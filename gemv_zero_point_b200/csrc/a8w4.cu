@@ -203,6 +203,15 @@ __device__ __forceinline__ uint4 ld_stream_u4(const void* p) {
   return v;
 }
 
+// 16 bytes through L2 only (coherent with writes of a preceding grid).
+__device__ __forceinline__ float4 ld_cg_f4(const float* p) {
+  float4 v;
+  asm volatile("ld.global.cg.v4.f32 {%0,%1,%2,%3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "l"(p));
+  return v;
+}
+
 __device__ __forceinline__ float ld_stream_f32(const float* p) {
   float v;
   asm volatile("ld.global.nc.L1::no_allocate.f32 %0, [%1];" : "=f"(v) : "l"(p));
@@ -366,11 +375,12 @@ __global__ void __launch_bounds__(256) a8w4_gemv_kernel(
 // loads of its first D rows before waiting for the previous grid; x and bias
 // may be outputs of that grid, so before the wait they are only prefetched
 // into L2 (a prefetch cannot return stale data: L2 is where every write
-// lands).  After the wait one thread copies x into shared memory, where the
-// CTA quantizes it while those weight rows are in flight; once x has landed
-// the rest of the CTA's slice is prefetched into L2.
+// lands).  After the wait every thread loads its share of x into registers
+// (through L2) and the CTA quantizes it while those weight rows are in
+// flight; once x has landed the rest of the CTA's slice is prefetched into
+// L2.
 // ---------------------------------------------------------------------------
-constexpr int kStreamSmemMax = 96 * 1024;  // x_s + bias_s
+constexpr int kStreamSmemMax = 96 * 1024;  // qa_s + bias_s
 
 // Warp-wide float min / max (NaN inputs ignored, as fminf / fmaxf do).
 __device__ __forceinline__ float warp_min(float v) {
@@ -409,12 +419,10 @@ __global__ void __launch_bounds__(W * 32, 1) a8w4_gemv_stream_kernel(
   extern __shared__ __align__(128) uint8_t sm[];
   __shared__ float red[2 * W];
   __shared__ float part_s[W * GPL];        // partial sums of the split rows
-  __shared__ __align__(8) uint64_t xfull;  // x has landed in x_s
   const int G = K >> 5;
   const int rowbytes = K >> 1;
-  float* x_s = reinterpret_cast<float*>(sm);             // [K] f32 as copied in
-  int8_t* qa_s = reinterpret_cast<int8_t*>(sm);          // [K] quantized x, over x_s
-  float* bias_s = reinterpret_cast<float*>(sm + 4 * K);  // [max_rows]
+  int8_t* qa_s = reinterpret_cast<int8_t*>(sm);      // [K] quantized x
+  float* bias_s = reinterpret_cast<float*>(sm + K);  // [max_rows]
 
   const int n0 = (int)((int64_t)blockIdx.x * N / gridDim.x);
   const int n1 = (int)((int64_t)(blockIdx.x + 1) * N / gridDim.x);
@@ -442,8 +450,6 @@ __global__ void __launch_bounds__(W * 32, 1) a8w4_gemv_stream_kernel(
   };
 
   if (threadIdx.x == 0) {
-    mbar_init(&xfull, 1);
-    fence_mbar_init();
     prefetch_l2_interior(x, (int64_t)K * 4);
     if (bias && n1 > n0) prefetch_l2_interior(bias + n0, (int64_t)(n1 - n0) * 4);
   }
@@ -467,44 +473,35 @@ __global__ void __launch_bounds__(W * 32, 1) a8w4_gemv_stream_kernel(
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
 
-  if (threadIdx.x == 0) {
-    // x in four chunks, in an order rotated by CTA, so that the CTAs do not
-    // all ask the same L2 lines for x at the same moment
-    mbar_arrive_expect_tx(&xfull, (uint32_t)(K * 4));
-    for (int c = 0; c < 4; ++c) {
-      const int q = (c + blockIdx.x) & 3;
-      bulk_g2s(x_s + q * (K / 4), x + q * (K / 4), (uint32_t)K, &xfull);
-    }
-  }
-
   // ---------------- quantize x ----------------
   for (int i = threadIdx.x; i < n1 - n0; i += W * 32)
     bias_s[i] = bias ? bias[n0 + i] : 0.0f;
-  // Each thread takes its float4 chunks of x from shared memory once and keeps
-  // them in registers for both passes (K <= 1024*GPL).
+  // Each thread loads its float4 chunks of x once (through L2, coherent with
+  // the previous grid's writes) and keeps them in registers for both passes
+  // (K <= 1024*GPL).
   constexpr int XV = (GPL * 1024 + 4 * W * 32 - 1) / (4 * W * 32);
   float4 xv[XV];
   float mn = 0.0f, mx = 0.0f;
-  const bool x_ok = mbar_wait(&xfull, 0, status);
-  if (threadIdx.x == 0) {
-    // the rest of the slice into L2, queued only once x (on the critical
-    // path) has landed
-    const int r_rest = n0 + W * min(D, nrows);  // rows beyond the ones already requested
-    if (r_rest < n1) {
-      prefetch_l2_interior(wq + (int64_t)r_rest * rowbytes, (int64_t)(n1 - r_rest) * rowbytes);
-      prefetch_l2_interior(wscale + (int64_t)r_rest * G, (int64_t)(n1 - r_rest) * G * 4);
-    }
-  }
 #pragma unroll
   for (int j = 0; j < XV; ++j) {
     const int c = threadIdx.x + j * W * 32;  // float4 chunk index
-    xv[j] = (x_ok && 4 * c < K) ? reinterpret_cast<const float4*>(x_s)[c]
-                                : make_float4(0.f, 0.f, 0.f, 0.f);
+    xv[j] = 4 * c < K ? ld_cg_f4(x + 4 * c) : make_float4(0.f, 0.f, 0.f, 0.f);
   }
 #pragma unroll
   for (int j = 0; j < XV; ++j) {
     mn = fminf(mn, fminf(fminf(xv[j].x, xv[j].y), fminf(xv[j].z, xv[j].w)));
     mx = fmaxf(mx, fmaxf(fmaxf(xv[j].x, xv[j].y), fmaxf(xv[j].z, xv[j].w)));
+  }
+  // The rest of the slice into L2, queued only once x (on the critical path)
+  // has landed: mn <= 0 always holds (the running minimum starts at 0, and
+  // fminf ignores NaN), but testing it makes the prefetch wait for this
+  // thread's x loads.
+  if (threadIdx.x == 0 && mn <= 0.0f) {
+    const int r_rest = n0 + W * min(D, nrows);  // rows beyond the ones already requested
+    if (r_rest < n1) {
+      prefetch_l2_interior(wq + (int64_t)r_rest * rowbytes, (int64_t)(n1 - r_rest) * rowbytes);
+      prefetch_l2_interior(wscale + (int64_t)r_rest * G, (int64_t)(n1 - r_rest) * G * 4);
+    }
   }
   mn = warp_min(mn);
   mx = warp_max(mx);
@@ -512,7 +509,7 @@ __global__ void __launch_bounds__(W * 32, 1) a8w4_gemv_stream_kernel(
     red[warp] = mn;
     red[W + warp] = mx;
   }
-  gemv_bar<W>();  // also: every x_s read is done before qa_s overwrites it
+  gemv_bar<W>();
   // every warp combines the W per-warp results (lanes past W repeat warp 0's)
   mn = warp_min(red[lane < W ? lane : 0]);
   mx = warp_max(red[W + (lane < W ? lane : 0)]);
@@ -616,7 +613,7 @@ static int launch_stream(int N, int K, const float* x, const uint8_t* wq, const 
   int grid = num_sms();
   if (grid > N) grid = N;
   const int rows_per_cta = (N + grid - 1) / grid;
-  const size_t smem = (size_t)4 * K + (size_t)rows_per_cta * 4;  // x_s, bias_s
+  const size_t smem = (size_t)K + (size_t)rows_per_cta * 4;  // qa_s, bias_s
   if (smem > (size_t)kStreamSmemMax) return 1;  // caller uses the plain kernel
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
