@@ -14,8 +14,9 @@
 // f32 TMEM accumulator.  Only the combination over groups is rounded (f32).
 //
 // Roles (448 threads, one CTA per SM, tile 128 x 128 over a K range):
-//   warp 0      TMA: bf16 A' stages (128 rows x 64 K, 128B swizzle), nibble
-//               stage tiles (128 rows x 32 bytes), the CTA's scale tile once
+//   warp 0      TMA: the CTA's nibble slice once, then (after waiting for the
+//               quantization grid) bf16 A' stages (128 rows x 64 K, 128B
+//               swizzle)
 //   warp 1      TMEM allocation; MMA issue, one 128-column TMEM buffer per
 //               group, 4 buffers
 //   warps 2..5  expand nibbles into the swizzled bf16 B' stage
@@ -233,6 +234,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       // this CTA's whole nibble slice (BN rows x Kr/2 bytes) in one box
       mbar_arrive_expect_tx(nib_full, (uint32_t)(BN * a.Kr / 2));
       tma_load_2d(sN, &tmW, k0 / 8, n0, nib_full);
+      // The activation codes come from the quantization grid just before
+      // this one (programmatic dependent launch): wait for it from here on.
+      asm volatile("griddepcontrol.wait;" ::: "memory");
       for (int s = 0; s < nstages; ++s) {
         const int slot = s % STAGES;
         if (s >= STAGES && !mbar_poll(&empty[slot], ((s / STAGES) - 1) & 1, status)) break;
@@ -322,6 +326,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
     }
     epi_sync(1);
+    // sA (read after the mainloop) comes from the quantization grid
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     unsigned long long acc[16];
 #pragma unroll
     for (int j = 0; j < 16; ++j) acc[j] = 0ull;
@@ -459,6 +465,8 @@ __global__ void __launch_bounds__(256) quantize_rows_centered_kernel(
     int8_t* __restrict__ q_opt, float* __restrict__ scale, int32_t* __restrict__ zero_point) {
   __shared__ float red[16];
   const int64_t m = blockIdx.x;
+  // let the GEMM grid start its prologue (it waits before reading our outputs)
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const float* xr = x + m * ldx;
   float mn = 0.0f, mx = 0.0f;
   int k = threadIdx.x;
@@ -594,13 +602,17 @@ int launch_a8w4_tc(int M, int N, int K, const float* x, int64_t ldx, const void*
   cfg.blockDim = dim3(THREADS);
   cfg.dynamicSmemBytes = SMEM_BYTES;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = (unsigned)splits;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  // programmatic dependent launch: the prologue (barriers, TMEM, the weight
+  // nibbles and scales) overlaps the quantization grid
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   cudaError_t e = cudaLaunchKernelEx(&cfg, a8w4_tc_kernel, tmA, tmW, a, status_word());
   return e == cudaSuccess ? QG_OK : QG_ERR_CUDA;
 }
