@@ -162,3 +162,25 @@ def test_gemv_without_optional_outputs_matches(lib):
     (y,) = _run_a8w4(lib, w, with_outputs=False)
     y2, *_ = _run_a8w4(lib, w)
     np.testing.assert_array_equal(y, y2)
+
+
+def test_gemv_chain_on_one_stream(lib):
+    """Back-to-back M = 1 calls on one stream, each reading the previous call's
+    y as its x.  A call may start while the previous one finishes (it fetches
+    its weights early); it must still quantize the finished y."""
+    K = 4096
+    ws = [workloads.a8w4(1, K, K, seed=40 + i) for i in range(3)]
+    packed = [lib.pack_w4_g32(_dev(w["qw"]), _dev(w["sw"])) for w in ws]
+    ys = [torch.empty((1, K), dtype=torch.float32, device="cuda") for _ in ws]
+    cur = _dev(ws[0]["x"])[:, :K]
+    for w, p, y in zip(ws, packed, ys):
+        lib.qgemm_a8w4_f32(cur, p, K, _dev(w["bias"]), w["clamp_min"], w["clamp_max"], y)
+        cur = y
+    torch.cuda.synchronize()
+    xin = ws[0]["x"][:, :K]
+    for w, y in zip(ws, ys):
+        y_ref = oracle.qgemm_a8w4_f32(xin, w["qw"], w["sw"], w["bias"], w["clamp_min"],
+                                      w["clamp_max"])[0]
+        y_np = y.cpu().numpy()
+        assert_a8w4_close(y_np, y_ref)
+        xin = y_np

@@ -116,6 +116,21 @@ def test_gemm_extreme_bound(lib):
     assert (acc == -K * 65025).all()
 
 
+@pytest.mark.parametrize("M", [64, 200])
+def test_gemm_k_at_the_overflow_bound(lib, M):
+    # K = 33025 is the largest K with K*65025 <= 2^31 - 1 (no bias): every term
+    # at the worst magnitude gives an accumulator of -2,147,450,625, inside
+    # int32 by 33,022.  M = 64 runs the one-CTA kernel, M = 200 the CTA pairs.
+    K = 33025
+    w = workloads.int8_gemm(M, 64, K, seed=3, za=-128, zb=127, with_bias=False)
+    w["A"][:] = 127
+    w["B"][:] = -128
+    w["ratio"] = np.array([1e-9])
+    C, acc, m0, sh = run_gemm(lib, w)
+    assert (acc == -K * 65025).all()
+    assert (C == w["out_zp"] + np.int64(oracle.rq_round(np.int64(-K * 65025), m0, sh))).all()
+
+
 def test_gemm_deterministic(lib):
     w = workloads.int8_gemm(300, 300, 500, seed=9)
     C1, a1, *_ = run_gemm(lib, w)
