@@ -356,6 +356,51 @@ def unpack_w4_g32(packed, N, K):
 
 
 # ---------------------------------------------------------------------------
+# O5: bf16 group scales ([KAI] review of the packing call: the Kleidi packing
+# is passed a bf16 type for the group scales, kept as bf16 to save space).
+# READING R12: f32 -> bf16 rounds to nearest, ties to even; the method then
+# uses that bf16 value as the group scale.
+# ---------------------------------------------------------------------------
+def f32_to_bf16_bits(a):
+    """bfloat16 bit patterns (uint16) of finite float32 values, rounded to
+    nearest with ties to even.  bf16 keeps the top 16 bits of the f32 pattern.
+    Patterns order like magnitudes within one sign, so adding 0x7FFF plus the
+    lowest kept bit and dropping the low 16 bits rounds the magnitude to
+    nearest, a tie (low half exactly 0x8000) going to the even pattern."""
+    a = np.ascontiguousarray(np.asarray(a, dtype=np.float32))
+    assert np.isfinite(a).all()
+    u = a.view(np.uint32).astype(np.uint64)
+    kept_lsb = (u >> 16) & 1
+    return ((u + 0x7FFF + kept_lsb) >> 16).astype(np.uint16)
+
+
+def bf16_bits_to_f32(b):
+    """bf16 bit patterns -> the float32 values they denote (exact)."""
+    b = np.ascontiguousarray(np.asarray(b, dtype=np.uint16))
+    return (b.astype(np.uint32) << 16).view(np.float32)
+
+
+def pack_w4_g32_bf16_bytes(N, K):
+    return N * (K // 2) + N * (K // GROUP) * 2
+
+
+def pack_w4_g32_bf16(qw, sw):
+    """As pack_w4_g32, with region 2 the bf16 patterns of sw[N][K/32] (R12),
+    little-endian, row-major."""
+    qw = np.asarray(qw)
+    N, K = qw.shape
+    nib = pack_w4_g32(qw, sw)[:N * (K // 2)]
+    bits = f32_to_bf16_bits(np.asarray(sw, np.float32).reshape(N, K // GROUP))
+    return np.concatenate([nib, bits.reshape(-1).astype("<u2").view(np.uint8)])
+
+
+def bf16_scales(sw):
+    """The group scales the bf16-scale method uses: sw rounded to bf16 (R12)."""
+    sw = np.asarray(sw, np.float32)
+    return bf16_bits_to_f32(f32_to_bf16_bits(sw)).reshape(sw.shape)
+
+
+# ---------------------------------------------------------------------------
 # O4: A8W4 blockwise GEMV/GEMM  ([KAI] matmul_clamp_f32_qai8dxp_qsi4c32p:
 # f32 out = clamp(dequant(int8 dyn act) x dequant(int4 g32 weights) + bias);
 # weight zero-points are absent (nullptr or all zero); bias before clamp R8)
@@ -383,3 +428,8 @@ def qgemm_a8w4_f32(x, qw, sw, bias, clamp_min, clamp_max):
             comb = comb + np.asarray(bias, np.float64)
         y[m] = np.minimum(np.maximum(comb.astype(np.float32), lo), hi)
     return y, qA, sA, za
+
+
+def qgemm_a8w4_f32_bf16s(x, qw, sw, bias, clamp_min, clamp_max):
+    """O4 with every group scale replaced by its bf16 value (O5, R12)."""
+    return qgemm_a8w4_f32(x, qw, bf16_scales(sw), bias, clamp_min, clamp_max)

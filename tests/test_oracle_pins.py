@@ -344,3 +344,66 @@ def test_p8_w4_pack_round_trip_and_bytes():
             expect.append(lo | (hi << 4))
     np.testing.assert_array_equal(p[:16], expect)
     assert p[16:20].view(np.float32)[0] == 1.0
+
+
+# ---------------------------------------------------------------------------
+# P9: bf16 group scales (reading R12: f32 -> bf16 round to nearest, ties to
+# even; the method uses the bf16 value)
+# ---------------------------------------------------------------------------
+def test_p9_bf16_rounding_hand_derived_cases():
+    # bf16 keeps 7 fraction bits: around 1.0 the spacing is 2^-7
+    cases = [
+        (1.0, 0x3F80),
+        (1 + 2 ** -8, 0x3F80),              # exactly half way: tie -> even (0x3F80)
+        (1 + 3 * 2 ** -8, 0x3F82),          # half way between 0x3F81 and 0x3F82 -> even
+        (1 + 2 ** -8 + 2 ** -23, 0x3F81),   # just above half way -> up
+        (1 + 2 ** -8 - 2 ** -23, 0x3F80),   # just below half way -> down
+        (-(1 + 2 ** -8), 0xBF80),           # the sign does not change the rounding
+        (2.0 ** -126, 0x0080),              # smallest normal, exact
+        (0.1, 0x3DCD),                      # 0x3DCCCCCD: low half 0xCCCD > 0x8000 -> up
+        (65280.0, 0x477F),                  # 255 * 256 exact
+    ]
+    x = np.array([c[0] for c in cases], np.float32)
+    got = oracle.f32_to_bf16_bits(x)
+    assert [int(v) for v in got] == [c[1] for c in cases]
+    # round trip of exact bf16 values is the identity
+    np.testing.assert_array_equal(oracle.bf16_bits_to_f32(got)[[0, 6, 8]],
+                                  np.array([1.0, 2.0 ** -126, 65280.0], np.float32))
+
+
+def test_p9_bf16_rounding_matches_library_conversion():
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(12)
+    x = rng.standard_normal(20000).astype(np.float32) * np.float32(10.0) ** rng.integers(-6, 6, 20000)
+    # exact ties: an f32 whose low 16 bits are 0x8000, both parities of bit 16
+    ties = (rng.integers(0x3000, 0x4F00, 4000).astype(np.uint32) << 16) | 0x8000
+    x = np.concatenate([x, ties.view(np.float32)])
+    lib = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    np.testing.assert_array_equal(oracle.f32_to_bf16_bits(x), lib)
+
+
+def test_p9_bf16_pack_layout_and_scales():
+    w = workloads.a8w4(1, 5, 64, seed=4)
+    p = oracle.pack_w4_g32_bf16(w["qw"], w["sw"])
+    assert p.size == oracle.pack_w4_g32_bf16_bytes(5, 64) == 5 * 32 + 5 * 2 * 2
+    # the nibble region is the f32 packing's, byte for byte
+    np.testing.assert_array_equal(p[:160], oracle.pack_w4_g32(w["qw"], w["sw"])[:160])
+    bits = p[160:].view("<u2").reshape(5, 2)
+    np.testing.assert_array_equal(bits, oracle.f32_to_bf16_bits(w["sw"]))
+    # the rounded scale is within half a bf16 step (2^-8 relative) of the f32 scale
+    rel = np.abs(oracle.bf16_scales(w["sw"]) - w["sw"]) / w["sw"]
+    assert rel.max() <= 2.0 ** -8
+
+
+def test_p9_bf16_linear_equals_f32_linear_on_representable_scales():
+    # with scales that are exact in bf16 (powers of two) the two methods agree
+    w = workloads.a8w4(3, 40, 128, seed=5)
+    sw = (2.0 ** np.round(np.log2(w["sw"]))).astype(np.float32)
+    np.testing.assert_array_equal(oracle.bf16_scales(sw), sw)
+    y16 = oracle.qgemm_a8w4_f32_bf16s(w["x"], w["qw"], sw, w["bias"], -6.0, 6.0)[0]
+    y32 = oracle.qgemm_a8w4_f32(w["x"], w["qw"], sw, w["bias"], -6.0, 6.0)[0]
+    np.testing.assert_array_equal(y16, y32)
+    # and with general scales they differ only through the rounded scales
+    y16g = oracle.qgemm_a8w4_f32_bf16s(w["x"], w["qw"], w["sw"], w["bias"], -6.0, 6.0)[0]
+    y32r = oracle.qgemm_a8w4_f32(w["x"], w["qw"], oracle.bf16_scales(w["sw"]), w["bias"], -6.0, 6.0)[0]
+    np.testing.assert_array_equal(y16g, y32r)
