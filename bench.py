@@ -21,7 +21,8 @@ it: 2 GEMM sets (A + packed B = 135 MB each) and 8 GEMV weight sets (36.8 MB
 each, 295 MB in all).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
-                  [--workload headline|cfg0|cfg1|cfg2|cfg3|cfg4] [--no-cpu-baseline]
+                  [--workload headline|cfg0|cfg1|cfg2|cfg2b|cfg3|cfg4] [--no-cpu-baseline]
+(cfg2b: the A8W4 GEMV with bf16 group scales.)
 Under torchrun each rank runs the same work on its own GPU (replicas: the
 path has no exchange step), and value sums all ranks' work.
 """
@@ -67,9 +68,9 @@ def gemm_bytes(M, N, K):
     return M * K + K * N + M * N + 3 * 4 * N
 
 
-def a8w4_bytes(M, N, K):
-    # int4 nibbles + f32 group scales + f32 x + f32 bias + f32 y
-    return N * K // 2 + N * (K // 32) * 4 + M * K * 4 + N * 4 + M * N * 4
+def a8w4_bytes(M, N, K, scale_bytes=4):
+    # int4 nibbles + group scales (f32, or bf16) + f32 x + f32 bias + f32 y
+    return N * K // 2 + N * (K // 32) * scale_bytes + M * K * 4 + N * 4 + M * N * 4
 
 
 def a8w4_ops(M, N, K):
@@ -261,16 +262,17 @@ class GemmCase:
 
 
 class A8W4Case:
-    def __init__(self, qg, torch, w, sets):
+    def __init__(self, qg, torch, w, sets, bf16_scales=False):
         self.M, self.N, self.K = w["M"], w["N"], w["K"]
         self.qg, self.torch = qg, torch
+        self.bf16 = bf16_scales
         qw = dev(w["qw"], torch)
         sw = dev(w["sw"], torch)
         self.packed = []
         for s in range(sets):
             # distinct weight sets: rotate the int4 codes along K (still in [-8,7])
             src = qw if s == 0 else torch.roll(qw, shifts=32 * s, dims=1)
-            self.packed.append(qg.pack_w4_g32(src, sw))
+            self.packed.append(qg.pack_w4_g32(src, sw, bf16_scales=bf16_scales))
         del qw
         self.x = dev(w["x"], torch)
         self.bias = None if w["bias"] is None else dev(w["bias"], torch)
@@ -285,7 +287,8 @@ class A8W4Case:
 
     def run(self, i, stream=None):
         self.qg.qgemm_a8w4_f32(self.x, self.packed[i % len(self.packed)], self.N, self.bias,
-                               self.lo, self.hi, self.y, workspace=self.ws, stream=stream)
+                               self.lo, self.hi, self.y, workspace=self.ws, stream=stream,
+                               bf16_scales=self.bf16)
 
     def prep_e2e(self):
         self.e2e_x = self.torch.empty(tuple(self.h2d_host.shape), dtype=self.torch.float32, device="cuda")
@@ -293,14 +296,14 @@ class A8W4Case:
     def run_e2e(self, i):
         self.e2e_x.copy_(self.h2d_host, non_blocking=True)
         self.qg.qgemm_a8w4_f32(self.e2e_x, self.packed[0], self.N, self.bias, self.lo, self.hi,
-                               self.y, workspace=self.ws)
+                               self.y, workspace=self.ws, bf16_scales=self.bf16)
         self.d2h_host.copy_(self.y, non_blocking=True)
 
     def ops(self):
         return a8w4_ops(self.M, self.N, self.K)
 
     def bytes(self):
-        return a8w4_bytes(self.M, self.N, self.K)
+        return a8w4_bytes(self.M, self.N, self.K, 2 if self.bf16 else 4)
 
     def h2d(self):
         return self.h2d_host.numel() * 4
@@ -372,6 +375,8 @@ def build_cases(workload, qg, torch):
         return [("a8w4_gemv_1x14336x4096", A8W4Case(qg, torch, W.cfg2_gemv(), 8), "hbm")]
     if workload == "cfg3":
         return [("a8w4_gemm_128x4096x4096", A8W4Case(qg, torch, W.cfg3_gemm(), 16), "hbm")]
+    if workload == "cfg2b":   # the GEMV with bf16 group scales (9 sets: 298 MB > L2)
+        return [("a8w4_gemv_bf16s_1x14336x4096", A8W4Case(qg, torch, W.cfg2_gemv(), 9, True), "hbm")]
     if workload == "cfg4":
         return [("int8_gemm_8192x8192x8200", GemmCase(qg, torch, W.cfg4_gemm_large(), 2), "tensor")]
     raise SystemExit(f"unknown workload {workload}")
@@ -387,6 +392,7 @@ KERNEL_SOURCES = {
     "int8_conv_56x56x64_3x3": "i8gemm.cu",
     "a8w4_gemv_1x14336x4096": "a8w4.cu",
     "a8w4_gemm_128x4096x4096": "a8w4_tc.cu",
+    "a8w4_gemv_bf16s_1x14336x4096": "a8w4.cu",
 }
 
 
@@ -437,14 +443,15 @@ def oracle_sample(workload, budget_s=12.0, rows_gemm=None, small=False):
         dt = time.perf_counter() - t
         ops += gemm_ops(rows, cols, w["K"]); spent += dt
         parts.append(f"int8 GEMM {rows} row(s) x {cols} cols of 8192x8192x8200")
-    if workload in ("headline", "cfg2"):
+    if workload in ("headline", "cfg2", "cfg2b"):
         w = W.cfg2_gemv()
         n = 512 if small else w["N"]
         t = time.perf_counter()
-        oracle.qgemm_a8w4_f32(w["x"], w["qw"][:n], w["sw"][:n], w["bias"][:n], -6.0, 6.0)
+        fn = oracle.qgemm_a8w4_f32_bf16s if workload == "cfg2b" else oracle.qgemm_a8w4_f32
+        fn(w["x"], w["qw"][:n], w["sw"][:n], w["bias"][:n], -6.0, 6.0)
         dt = time.perf_counter() - t
         ops += a8w4_ops(1, n, w["K"]); spent += dt
-        parts.append(f"A8W4 GEMV {n} of 14336 rows")
+        parts.append(f"A8W4 GEMV{' (bf16 scales)' if workload == 'cfg2b' else ''} {n} of 14336 rows")
     if workload == "cfg3":
         w = W.cfg3_gemm()
         rows = 1 if small else 4
@@ -510,7 +517,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="headline",
-                    choices=["headline", "cfg0", "cfg1", "cfg2", "cfg3", "cfg4"])
+                    choices=["headline", "cfg0", "cfg1", "cfg2", "cfg2b", "cfg3", "cfg4"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=10)
     args = ap.parse_args()

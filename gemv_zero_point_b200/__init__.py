@@ -88,6 +88,10 @@ _sig("pack_w4_g32", _i32, [_i32, _i32, _vp, _i64, _vp, _vp, _sz, _vp])
 _sig("qgemm_a8w4_workspace_bytes", _sz, [_i32, _i32, _i32])
 _sig("qgemm_a8w4_f32", _i32, [_i32, _i32, _i32, _vp, _i64, _vp, _vp, _f32, _f32, _vp, _i64,
                               _vp, _vp, _vp, _vp, _sz, _vp])
+_sig("pack_w4_g32_bf16_bytes", _sz, [_i32, _i32])
+_sig("pack_w4_g32_bf16", _i32, [_i32, _i32, _vp, _i64, _vp, _vp, _sz, _vp])
+_sig("qgemm_a8w4_f32_bf16s", _i32, [_i32, _i32, _i32, _vp, _i64, _vp, _vp, _f32, _f32, _vp,
+                                    _i64, _vp, _vp, _vp, _vp, _sz, _vp])
 
 
 def _check(rc, where):
@@ -168,14 +172,22 @@ def pack_w4_g32_bytes(N, K):
     return lib.pack_w4_g32_bytes(N, K)
 
 
-def pack_w4_g32(w, group_scales, packed=None, stream=None):
+def pack_w4_g32(w, group_scales, packed=None, stream=None, bf16_scales=False):
+    """Pack int4 weights [N][K] and f32 group scales; with bf16_scales the
+    scales are stored rounded to bf16 (use with qgemm_a8w4_f32_bf16s)."""
     N, K = w.shape
-    nbytes = lib.pack_w4_g32_bytes(N, K)
+    bytes_fn = lib.pack_w4_g32_bf16_bytes if bf16_scales else lib.pack_w4_g32_bytes
+    pack_fn = lib.pack_w4_g32_bf16 if bf16_scales else lib.pack_w4_g32
+    nbytes = bytes_fn(N, K)
     if packed is None:
         packed = _empty_bytes(nbytes, w.device)
-    _check(lib.pack_w4_g32(N, K, _p(w), _ld(w), _p(group_scales), _p(packed), packed.numel(),
-                           _stream(stream)), "pack_w4_g32")
+    _check(pack_fn(N, K, _p(w), _ld(w), _p(group_scales), _p(packed), packed.numel(),
+                   _stream(stream)), pack_fn.__name__)
     return packed
+
+
+def pack_w4_g32_bf16(w, group_scales, packed=None, stream=None):
+    return pack_w4_g32(w, group_scales, packed, stream, bf16_scales=True)
 
 
 def qgemm_a8w4_workspace_bytes(M, N, K):
@@ -183,16 +195,21 @@ def qgemm_a8w4_workspace_bytes(M, N, K):
 
 
 def qgemm_a8w4_f32(x, packed_w, N, bias, clamp_min, clamp_max, y, q_out=None, scale_out=None,
-                   zp_out=None, workspace=None, stream=None):
+                   zp_out=None, workspace=None, stream=None, bf16_scales=False):
+    """A8W4 linear; bf16_scales selects weights packed by pack_w4_g32_bf16."""
     M, K = x.shape
     wsb = lib.qgemm_a8w4_workspace_bytes(M, N, K)
     if wsb and workspace is None:
         workspace = _empty_bytes(wsb, x.device)
-    _check(lib.qgemm_a8w4_f32(M, N, K, _p(x), _ld(x), _p(packed_w), _p(bias),
-                              float(clamp_min), float(clamp_max), _p(y), _ld(y), _p(q_out),
-                              _p(scale_out), _p(zp_out), _p(workspace),
-                              0 if workspace is None else workspace.numel(), _stream(stream)),
-           "qgemm_a8w4_f32")
+    fn = lib.qgemm_a8w4_f32_bf16s if bf16_scales else lib.qgemm_a8w4_f32
+    _check(fn(M, N, K, _p(x), _ld(x), _p(packed_w), _p(bias),
+              float(clamp_min), float(clamp_max), _p(y), _ld(y), _p(q_out),
+              _p(scale_out), _p(zp_out), _p(workspace),
+              0 if workspace is None else workspace.numel(), _stream(stream)), fn.__name__)
+
+
+def qgemm_a8w4_f32_bf16s(x, packed_w, N, bias, clamp_min, clamp_max, y, **kw):
+    return qgemm_a8w4_f32(x, packed_w, N, bias, clamp_min, clamp_max, y, bf16_scales=True, **kw)
 
 
 # ---------------------------------------------------------------------------

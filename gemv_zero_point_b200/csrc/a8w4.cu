@@ -7,6 +7,7 @@
 // clamped after the bias); MNN ConvInt8TiledExecutor.cpp
 // (BatchAsyDynamicQuant min/max quantization; int4 weights stored with an
 // offset of 8 in _computeReorderQuantInfo).
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
@@ -121,12 +122,12 @@ int launch_quantize_rows(int M, int K, const float* x, int64_t ldx, int8_t* q, i
 // ---------------------------------------------------------------------------
 __global__ void pack_w4_kernel(int N, int K, const int8_t* __restrict__ w, int64_t ldw,
                                const float* __restrict__ sw, uint8_t* __restrict__ packed,
-                               int* status) {
+                               int scale_bf16, int* status) {
   const int64_t words_per_row = K / 8;
   const int64_t total = (int64_t)N * words_per_row;
   const int G = K / 32;
   uint32_t* out = reinterpret_cast<uint32_t*>(packed);
-  float* sout = reinterpret_cast<float*>(packed + (size_t)N * (K / 2));
+  uint8_t* sout = packed + (size_t)N * (K / 2);  // f32 or bf16 scales [N][K/32]
   bool bad = false;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
        i += (int64_t)gridDim.x * blockDim.x) {
@@ -142,17 +143,22 @@ __global__ void pack_w4_kernel(int N, int K, const int8_t* __restrict__ w, int64
     out[i] = word;
   }
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < (int64_t)N * G;
-       i += (int64_t)gridDim.x * blockDim.x)
-    sout[i] = sw[i];
+       i += (int64_t)gridDim.x * blockDim.x) {
+    if (scale_bf16)  // round to nearest even
+      reinterpret_cast<unsigned short*>(sout)[i] = __bfloat16_as_ushort(__float2bfloat16_rn(sw[i]));
+    else
+      reinterpret_cast<float*>(sout)[i] = sw[i];
+  }
   if (bad) record_error(status, QG_ERR_INVALID_ARG);
 }
 
 int launch_pack_w4(int N, int K, const int8_t* w, int64_t ldw, const float* sw, void* packed,
-                   cudaStream_t st) {
+                   bool scale_bf16, cudaStream_t st) {
   const int64_t words = (int64_t)N * (K / 8);
   int blocks = (int)min64(cdiv(words, 256), (int64_t)num_sms() * 8);
   if (blocks < 1) blocks = 1;
-  pack_w4_kernel<<<blocks, 256, 0, st>>>(N, K, w, ldw, sw, (uint8_t*)packed, status_word());
+  pack_w4_kernel<<<blocks, 256, 0, st>>>(N, K, w, ldw, sw, (uint8_t*)packed, scale_bf16 ? 1 : 0,
+                                         status_word());
   return launch_status();
 }
 
@@ -218,6 +224,40 @@ __device__ __forceinline__ float ld_stream_f32(const float* p) {
   return v;
 }
 
+// Scale of group g = lane + 32*i of row r (G groups per row) for the GEMV
+// lanes.  With bf16 scales the lane reads the 32-bit word holding the scales
+// of groups g and g^1; g has the lane's parity, so the half is picked with a
+// byte permute whose selector `sel` the caller fixes once per lane (0x1044:
+// low half, 0x3244: high half, moved to the top of an f32 pattern).
+template <bool SBF>
+__device__ __forceinline__ float ld_row_scale(const void* base, int64_t r, int G, int lane, int i,
+                                              uint32_t sel) {
+  if constexpr (SBF) {
+    const uint32_t* p = reinterpret_cast<const uint32_t*>(base) + r * (G >> 1) + (lane >> 1) + 16 * i;
+    uint32_t v, d;
+    asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
+    asm("prmt.b32 %0, %1, 0, %2;" : "=r"(d) : "r"(v), "r"(sel));
+    return __uint_as_float(d);
+  } else {
+    return ld_stream_f32(reinterpret_cast<const float*>(base) + r * G + lane + 32 * i);
+  }
+}
+
+// Group scale i of a packed W4 matrix, stored as f32 or (SBF) as bf16; a bf16
+// value widens to f32 exactly.  A bf16 scale is read as the aligned 32-bit
+// word holding it and its neighbour (the scale array starts 16-byte aligned).
+template <bool SBF>
+__device__ __forceinline__ float ld_scale(const void* base, int64_t i) {
+  if constexpr (SBF) {
+    const uint32_t* p = reinterpret_cast<const uint32_t*>(base) + (i >> 1);
+    uint32_t v;
+    asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
+    return __uint_as_float((i & 1) ? (v & 0xFFFF0000u) : (v << 16));
+  } else {
+    return ld_stream_f32(reinterpret_cast<const float*>(base) + i);
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Fused A8W4 GEMV (M = 1).
 //
@@ -231,10 +271,10 @@ __device__ __forceinline__ float ld_stream_f32(const float* p) {
 // per iteration keep eight 128-bit loads in flight per lane; their partial
 // sums are reduced together with five shuffles.
 // ---------------------------------------------------------------------------
-template <int GPL>
+template <int GPL, bool SBF>
 __global__ void __launch_bounds__(256) a8w4_gemv_kernel(
     int N, int K, const float* __restrict__ x, const uint8_t* __restrict__ wq,
-    const float* __restrict__ wscale, const float* __restrict__ bias, float clamp_lo,
+    const void* __restrict__ wscale, const float* __restrict__ bias, float clamp_lo,
     float clamp_hi, float* __restrict__ y, int8_t* __restrict__ q_out, float* __restrict__ scale_out,
     int32_t* __restrict__ zp_out) {
   extern __shared__ __align__(16) int8_t qa_s[];  // K bytes
@@ -255,8 +295,9 @@ __global__ void __launch_bounds__(256) a8w4_gemv_kernel(
       bytes -= c;
     }
     // scales: round the start down and the end down to 16 bytes (in bounds)
-    uintptr_t s0 = (uintptr_t)(wscale + (int64_t)n0 * G) & ~(uintptr_t)15;
-    uintptr_t s1 = (uintptr_t)(wscale + (int64_t)n1 * G) & ~(uintptr_t)15;
+    const int64_t sb = SBF ? 2 : 4;  // bytes per scale
+    uintptr_t s0 = ((uintptr_t)wscale + (uintptr_t)((int64_t)n0 * G * sb)) & ~(uintptr_t)15;
+    uintptr_t s1 = ((uintptr_t)wscale + (uintptr_t)((int64_t)n1 * G * sb)) & ~(uintptr_t)15;
     if (s1 > s0) bulk_prefetch_l2((const void*)s0, (uint32_t)(s1 - s0));
   }
 
@@ -318,10 +359,10 @@ __global__ void __launch_bounds__(256) a8w4_gemv_kernel(
         const int g = ch * 32 * GPL + lane + 32 * i;
         if (g < G) {
           w0[i] = ld_stream_u4(wq + (int64_t)r * rowbytes + 16 * g);
-          s0[i] = ld_stream_f32(wscale + (int64_t)r * G + g);
+          s0[i] = ld_scale<SBF>(wscale, (int64_t)r * G + g);
           if (has_b) {
             w1[i] = ld_stream_u4(wq + (int64_t)rb * rowbytes + 16 * g);
-            s1[i] = ld_stream_f32(wscale + (int64_t)rb * G + g);
+            s1[i] = ld_scale<SBF>(wscale, (int64_t)rb * G + g);
           }
         }
       }
@@ -410,10 +451,10 @@ __device__ __forceinline__ void prefetch_l2_interior(const void* p, int64_t byte
   }
 }
 
-template <int GPL, int W, int D>
+template <int GPL, int W, int D, bool SBF>
 __global__ void __launch_bounds__(W * 32, 1) a8w4_gemv_stream_kernel(
     int N, int K, int max_rows, const float* __restrict__ x, const uint8_t* __restrict__ wq,
-    const float* __restrict__ wscale, const float* __restrict__ bias, float clamp_lo,
+    const void* __restrict__ wscale, const float* __restrict__ bias, float clamp_lo,
     float clamp_hi, float* __restrict__ y, int8_t* __restrict__ q_out,
     float* __restrict__ scale_out, int32_t* __restrict__ zp_out, int* status) {
   extern __shared__ __align__(128) uint8_t sm[];
@@ -435,6 +476,7 @@ __global__ void __launch_bounds__(W * 32, 1) a8w4_gemv_stream_kernel(
   uint4 wbuf[D][GPL];
   float sbuf[D][GPL];
   // loads of this warp's row j into buffer u (nothing past the last row)
+  const uint32_t ssel = (lane & 1) ? 0x3244u : 0x1044u;  // bf16 half of the scale word
   auto load_row = [&](int u, int j) {
     if (j < nrows) {
       const int r = n0 + warp + W * j;
@@ -443,7 +485,7 @@ __global__ void __launch_bounds__(W * 32, 1) a8w4_gemv_stream_kernel(
         const int g = lane + 32 * i;
         if (g < G) {
           wbuf[u][i] = ld_stream_u4(wq + (int64_t)r * rowbytes + 16 * g);
-          sbuf[u][i] = ld_stream_f32(wscale + (int64_t)r * G + g);
+          sbuf[u][i] = ld_row_scale<SBF>(wscale, r, G, lane, i, ssel);
         }
       }
     }
@@ -463,7 +505,7 @@ __global__ void __launch_bounds__(W * 32, 1) a8w4_gemv_stream_kernel(
     const int g = lane + 32 * slot;
     if (g < G) {
       wsplit = ld_stream_u4(wq + (int64_t)r * rowbytes + 16 * g);
-      ssplit = ld_stream_f32(wscale + (int64_t)r * G + g);
+      ssplit = ld_row_scale<SBF>(wscale, r, G, lane, slot, ssel);
     }
   };
   if (warp / GPL < nleft) load_split(warp / GPL);
@@ -500,7 +542,9 @@ __global__ void __launch_bounds__(W * 32, 1) a8w4_gemv_stream_kernel(
     const int r_rest = n0 + W * min(D, nrows);  // rows beyond the ones already requested
     if (r_rest < n1) {
       prefetch_l2_interior(wq + (int64_t)r_rest * rowbytes, (int64_t)(n1 - r_rest) * rowbytes);
-      prefetch_l2_interior(wscale + (int64_t)r_rest * G, (int64_t)(n1 - r_rest) * G * 4);
+      constexpr int64_t sb = SBF ? 2 : 4;  // bytes per scale
+      prefetch_l2_interior((const uint8_t*)wscale + (int64_t)r_rest * G * sb,
+                           (int64_t)(n1 - r_rest) * G * sb);
     }
   }
   mn = warp_min(mn);
@@ -606,8 +650,8 @@ __global__ void __launch_bounds__(W * 32, 1) a8w4_gemv_stream_kernel(
   }
 }
 
-template <int GPL, int W, int D>
-static int launch_stream(int N, int K, const float* x, const uint8_t* wq, const float* ws,
+template <int GPL, int W, int D, bool SBF>
+static int launch_stream(int N, int K, const float* x, const uint8_t* wq, const void* ws,
                          const float* bias, float lo, float hi, float* y, int8_t* q_out,
                          float* scale_out, int32_t* zp_out, cudaStream_t st) {
   int grid = num_sms();
@@ -625,62 +669,72 @@ static int launch_stream(int N, int K, const float* x, const uint8_t* wq, const 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, a8w4_gemv_stream_kernel<GPL, W, D>, N, K, rows_per_cta,
+  cudaError_t e = cudaLaunchKernelEx(&cfg, a8w4_gemv_stream_kernel<GPL, W, D, SBF>, N, K, rows_per_cta,
                                      x, wq, ws, bias, lo, hi, y, q_out, scale_out, zp_out,
                                      status_word());
   return e == cudaSuccess ? QG_OK : QG_ERR_CUDA;
 }
 
-int launch_a8w4_gemv(int N, int K, const float* x, const void* packed, const float* bias,
-                     float lo, float hi, float* y, int8_t* q_out, float* scale_out,
-                     int32_t* zp_out, cudaStream_t st) {
+template <bool SBF>
+static int launch_a8w4_gemv_t(int N, int K, const float* x, const void* packed,
+                              const float* bias, float lo, float hi, float* y, int8_t* q_out,
+                              float* scale_out, int32_t* zp_out, cudaStream_t st) {
   const uint8_t* wq = (const uint8_t*)packed;
-  const float* ws = (const float*)(wq + (size_t)N * (K / 2));
+  const void* ws = wq + (size_t)N * (K / 2);
   const int G = K / 32;
   int grid = num_sms() * 2;
   if (grid > N) grid = N;
   if (K % 128 == 0 && K <= 8192 && ((uintptr_t)x & 15) == 0) {
     int rc;
-    if (G <= 32) rc = launch_stream<1, 16, 3>(N, K, x, wq, ws, bias, lo, hi, y, q_out, scale_out, zp_out, st);
-    else if (G <= 64) rc = launch_stream<2, 16, 3>(N, K, x, wq, ws, bias, lo, hi, y, q_out, scale_out, zp_out, st);
-    else if (G <= 128) rc = launch_stream<4, 16, 2>(N, K, x, wq, ws, bias, lo, hi, y, q_out, scale_out, zp_out, st);
-    else rc = launch_stream<8, 8, 3>(N, K, x, wq, ws, bias, lo, hi, y, q_out, scale_out, zp_out, st);
+    if (G <= 32) rc = launch_stream<1, 16, 3, SBF>(N, K, x, wq, ws, bias, lo, hi, y, q_out, scale_out, zp_out, st);
+    else if (G <= 64) rc = launch_stream<2, 16, 3, SBF>(N, K, x, wq, ws, bias, lo, hi, y, q_out, scale_out, zp_out, st);
+    else if (G <= 128) rc = launch_stream<4, 16, 2, SBF>(N, K, x, wq, ws, bias, lo, hi, y, q_out, scale_out, zp_out, st);
+    else rc = launch_stream<8, 8, 3, SBF>(N, K, x, wq, ws, bias, lo, hi, y, q_out, scale_out, zp_out, st);
     if (rc <= 0) return rc;
   }
   const size_t smem = (size_t)K;
   if (G <= 32) {
-    a8w4_gemv_kernel<1><<<grid, 256, smem, st>>>(N, K, x, wq, ws, bias, lo, hi, y, q_out,
-                                                 scale_out, zp_out);
+    a8w4_gemv_kernel<1, SBF><<<grid, 256, smem, st>>>(N, K, x, wq, ws, bias, lo, hi, y, q_out,
+                                                      scale_out, zp_out);
   } else if (G <= 64) {
-    a8w4_gemv_kernel<2><<<grid, 256, smem, st>>>(N, K, x, wq, ws, bias, lo, hi, y, q_out,
-                                                 scale_out, zp_out);
+    a8w4_gemv_kernel<2, SBF><<<grid, 256, smem, st>>>(N, K, x, wq, ws, bias, lo, hi, y, q_out,
+                                                      scale_out, zp_out);
   } else {
-    a8w4_gemv_kernel<4><<<grid, 256, smem, st>>>(N, K, x, wq, ws, bias, lo, hi, y, q_out,
-                                                 scale_out, zp_out);
+    a8w4_gemv_kernel<4, SBF><<<grid, 256, smem, st>>>(N, K, x, wq, ws, bias, lo, hi, y, q_out,
+                                                      scale_out, zp_out);
   }
   return launch_status();
 }
 
+int launch_a8w4_gemv(int N, int K, const float* x, const void* packed, const float* bias,
+                     float lo, float hi, float* y, int8_t* q_out, float* scale_out,
+                     int32_t* zp_out, bool scale_bf16, cudaStream_t st) {
+  return scale_bf16 ? launch_a8w4_gemv_t<true>(N, K, x, packed, bias, lo, hi, y, q_out,
+                                               scale_out, zp_out, st)
+                    : launch_a8w4_gemv_t<false>(N, K, x, packed, bias, lo, hi, y, q_out,
+                                                scale_out, zp_out, st);
+}
+
+template <bool SBF>
+static bool setup_a8w4_gemv_t() {
+  // up to 64 KiB of activations in shared memory for the plain kernel
+  const void* plain[] = {(const void*)a8w4_gemv_kernel<1, SBF>, (const void*)a8w4_gemv_kernel<2, SBF>,
+                         (const void*)a8w4_gemv_kernel<4, SBF>};
+  const void* stream[] = {(const void*)a8w4_gemv_stream_kernel<1, 16, 3, SBF>,
+                          (const void*)a8w4_gemv_stream_kernel<2, 16, 3, SBF>,
+                          (const void*)a8w4_gemv_stream_kernel<4, 16, 2, SBF>,
+                          (const void*)a8w4_gemv_stream_kernel<8, 8, 3, SBF>};
+  bool ok = true;
+  for (const void* f : plain)
+    ok &= cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, 65536) == cudaSuccess;
+  for (const void* f : stream)
+    ok &= cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmemMax) ==
+          cudaSuccess;
+  return ok;
+}
+
 int setup_a8w4_gemv() {
-  // allow up to 64 KiB of activations in shared memory
-  cudaError_t e1 = cudaFuncSetAttribute(a8w4_gemv_kernel<1>,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize, 65536);
-  cudaError_t e2 = cudaFuncSetAttribute(a8w4_gemv_kernel<2>,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize, 65536);
-  cudaError_t e3 = cudaFuncSetAttribute(a8w4_gemv_kernel<4>,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize, 65536);
-  cudaError_t e4 = cudaFuncSetAttribute(a8w4_gemv_stream_kernel<1, 16, 3>,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmemMax);
-  cudaError_t e5 = cudaFuncSetAttribute(a8w4_gemv_stream_kernel<2, 16, 3>,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmemMax);
-  cudaError_t e6 = cudaFuncSetAttribute(a8w4_gemv_stream_kernel<4, 16, 2>,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmemMax);
-  cudaError_t e7 = cudaFuncSetAttribute(a8w4_gemv_stream_kernel<8, 8, 3>,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmemMax);
-  return (e1 == cudaSuccess && e2 == cudaSuccess && e3 == cudaSuccess && e4 == cudaSuccess &&
-          e5 == cudaSuccess && e6 == cudaSuccess && e7 == cudaSuccess)
-             ? QG_OK
-             : QG_ERR_CUDA;
+  return (setup_a8w4_gemv_t<false>() && setup_a8w4_gemv_t<true>()) ? QG_OK : QG_ERR_CUDA;
 }
 
 // ---------------------------------------------------------------------------
@@ -692,10 +746,11 @@ int setup_a8w4_gemv() {
 // ---------------------------------------------------------------------------
 constexpr int kSimtRows = 8;
 
+template <bool SBF>
 __global__ void __launch_bounds__(256) a8w4_gemm_simt_kernel(
     int M, int N, int K, const int8_t* __restrict__ q, const float* __restrict__ sA,
     const int32_t* __restrict__ zA, const uint8_t* __restrict__ wq,
-    const float* __restrict__ wscale, const float* __restrict__ bias, float lo, float hi,
+    const void* __restrict__ wscale, const float* __restrict__ bias, float lo, float hi,
     float* __restrict__ y, int64_t ldy) {
   extern __shared__ __align__(16) int8_t qs[];  // kSimtRows * K
   const int G = K >> 5;
@@ -720,7 +775,7 @@ __global__ void __launch_bounds__(256) a8w4_gemm_simt_kernel(
     for (int r = 0; r < kSimtRows; ++r) acc[r] = 0.0f;
     for (int g = lane; g < G; g += 32) {
       const uint4 w = ld_stream_u4(wq + (int64_t)n * rowbytes + 16 * g);
-      const float s = ld_stream_f32(wscale + (int64_t)n * G + g);
+      const float s = ld_scale<SBF>(wscale, (int64_t)n * G + g);
 #pragma unroll
       for (int r = 0; r < kSimtRows; ++r) {
         if (r < rows) {
@@ -747,21 +802,28 @@ __global__ void __launch_bounds__(256) a8w4_gemm_simt_kernel(
 
 int launch_a8w4_gemm_simt(int M, int N, int K, const int8_t* q, const float* sA,
                           const int32_t* zA, const void* packed, const float* bias, float lo,
-                          float hi, float* y, int64_t ldy, cudaStream_t st) {
+                          float hi, float* y, int64_t ldy, bool scale_bf16, cudaStream_t st) {
   const uint8_t* wq = (const uint8_t*)packed;
-  const float* ws = (const float*)(wq + (size_t)N * (K / 2));
+  const void* ws = wq + (size_t)N * (K / 2);
   const int mblocks = (int)cdiv(M, kSimtRows);
   int nblocks = (int)max64(1, min64(cdiv((int64_t)num_sms() * 2, mblocks), cdiv(N, 8)));
   dim3 grid(nblocks, mblocks);
   const size_t smem = (size_t)kSimtRows * K;
-  a8w4_gemm_simt_kernel<<<grid, 256, smem, st>>>(M, N, K, q, sA, zA, wq, ws, bias, lo, hi, y, ldy);
+  if (scale_bf16)
+    a8w4_gemm_simt_kernel<true><<<grid, 256, smem, st>>>(M, N, K, q, sA, zA, wq, ws, bias, lo, hi,
+                                                         y, ldy);
+  else
+    a8w4_gemm_simt_kernel<false><<<grid, 256, smem, st>>>(M, N, K, q, sA, zA, wq, ws, bias, lo, hi,
+                                                          y, ldy);
   return launch_status();
 }
 
 int setup_a8w4_gemm_simt() {
-  cudaError_t e = cudaFuncSetAttribute(a8w4_gemm_simt_kernel,
+  cudaError_t e = cudaFuncSetAttribute(a8w4_gemm_simt_kernel<false>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-  return e == cudaSuccess ? QG_OK : QG_ERR_CUDA;
+  cudaError_t e2 = cudaFuncSetAttribute(a8w4_gemm_simt_kernel<true>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+  return (e == cudaSuccess && e2 == cudaSuccess) ? QG_OK : QG_ERR_CUDA;
 }
 
 }  // namespace qg

@@ -160,7 +160,8 @@ __device__ __forceinline__ float4 ld_dsmem_f4(uint32_t addr) {
 
 struct Args {
   int M, N, K, Kr, splits, n_tiles;
-  const float* wscale;  // packed group scales [N][K/32]
+  const void* wscale;   // packed group scales [N][K/32], f32 or bf16
+  int scale_bf16;
   const float* sA;
   const float* bias;
   float lo, hi;
@@ -322,7 +323,13 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int G = a.K / 32, g0 = k0 / 32;
       for (int i = etid; i < BN * Gr; i += EPI_THREADS) {
         const int n = i / Gr, g = i - n * Gr;
-        scl_t[g * BN + n] = (n0 + n < a.N) ? __ldg(a.wscale + (int64_t)(n0 + n) * G + g0 + g) : 0.0f;
+        const int64_t idx = (int64_t)(n0 + n) * G + g0 + g;
+        float v = 0.0f;
+        if (n0 + n < a.N)  // a bf16 scale widens to f32 exactly
+          v = a.scale_bf16
+                  ? __uint_as_float((uint32_t)__ldg(reinterpret_cast<const unsigned short*>(a.wscale) + idx) << 16)
+                  : __ldg(reinterpret_cast<const float*>(a.wscale) + idx);
+        scl_t[g * BN + n] = v;
       }
     }
     epi_sync(1);
@@ -565,7 +572,8 @@ int a8w4_tc_setup() {
 
 int launch_a8w4_tc(int M, int N, int K, const float* x, int64_t ldx, const void* packed,
                    const float* bias, float lo, float hi, float* y, int64_t ldy, int8_t* q_out,
-                   float* scale_out, int32_t* zp_out, void* ws, size_t ws_bytes, cudaStream_t st) {
+                   float* scale_out, int32_t* zp_out, void* ws, size_t ws_bytes, bool scale_bf16,
+                   cudaStream_t st) {
   const int splits = a8w4_tc_splits(M, N, K, num_sms());
   if (splits <= 0) return QG_ERR_UNSUPPORTED;
   if (!ws || ws_bytes < a8w4_tc_workspace_bytes(M, N, K, splits)) return QG_ERR_WORKSPACE;
@@ -584,7 +592,7 @@ int launch_a8w4_tc(int M, int N, int K, const float* x, int64_t ldx, const void*
   if (zp_out && cudaMemcpyAsync(zp_out, zA, (size_t)M * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
     return QG_ERR_CUDA;
   const uint8_t* wq = (const uint8_t*)packed;
-  const float* wsc = (const float*)(wq + (size_t)N * (K / 2));
+  const void* wsc = wq + (size_t)N * (K / 2);
   const int Kr = K / splits;
   CUtensorMap tmA, tmW;
   rc = make_tmap_generic(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, qc, (uint64_t)K, (uint64_t)M,
@@ -596,6 +604,7 @@ int launch_a8w4_tc(int M, int N, int K, const float* x, int64_t ldx, const void*
   Args a;
   a.M = M; a.N = N; a.K = K; a.Kr = Kr; a.splits = splits; a.n_tiles = (int)nt;
   a.wscale = wsc;
+  a.scale_bf16 = scale_bf16 ? 1 : 0;
   a.sA = sA; a.bias = bias; a.lo = lo; a.hi = hi; a.y = y; a.ldy = ldy;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(mt * nt * splits));

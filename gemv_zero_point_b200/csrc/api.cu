@@ -15,13 +15,13 @@ namespace qg {
 int launch_quantize_rows(int M, int K, const float* x, int64_t ldx, int8_t* q, int64_t ldq,
                          float* scale, int32_t* zp, cudaStream_t st);
 int launch_pack_w4(int N, int K, const int8_t* w, int64_t ldw, const float* sw, void* packed,
-                   cudaStream_t st);
+                   bool scale_bf16, cudaStream_t st);
 int launch_a8w4_gemv(int N, int K, const float* x, const void* packed, const float* bias,
                      float lo, float hi, float* y, int8_t* q_out, float* scale_out,
-                     int32_t* zp_out, cudaStream_t st);
+                     int32_t* zp_out, bool scale_bf16, cudaStream_t st);
 int launch_a8w4_gemm_simt(int M, int N, int K, const int8_t* q, const float* sA,
                           const int32_t* zA, const void* packed, const float* bias, float lo,
-                          float hi, float* y, int64_t ldy, cudaStream_t st);
+                          float hi, float* y, int64_t ldy, bool scale_bf16, cudaStream_t st);
 int setup_a8w4_gemv();
 int setup_a8w4_gemm_simt();
 int i8gemm_setup();
@@ -31,7 +31,8 @@ int a8w4_tc_splits(int M, int N, int K, int sms);
 size_t a8w4_tc_workspace_bytes(int M, int N, int K, int splits);
 int launch_a8w4_tc(int M, int N, int K, const float* x, int64_t ldx, const void* packed,
                    const float* bias, float lo, float hi, float* y, int64_t ldy, int8_t* q_out,
-                   float* scale_out, int32_t* zp_out, void* ws, size_t ws_bytes, cudaStream_t st);
+                   float* scale_out, int32_t* zp_out, void* ws, size_t ws_bytes, bool scale_bf16,
+                   cudaStream_t st);
 
 int i8gemm_pack_b(int K, int N, const int8_t* B, int64_t ldb, void* packed, cudaStream_t st);
 size_t i8gemm_pack_b_bytes(int K, int N);
@@ -319,15 +320,32 @@ extern "C" size_t pack_w4_g32_bytes(int N, int K) {
   return (size_t)N * (K / 2) + (size_t)N * (K / 32) * 4;
 }
 
-extern "C" int pack_w4_g32(int N, int K, const int8_t* w, int64_t ldw, const float* group_scales,
-                           void* packed, size_t packed_bytes, void* stream) {
+extern "C" size_t pack_w4_g32_bf16_bytes(int N, int K) {
+  if (N <= 0 || K <= 0 || K % 32) return 0;
+  return (size_t)N * (K / 2) + (size_t)N * (K / 32) * 2;
+}
+
+static int pack_w4(int N, int K, const int8_t* w, int64_t ldw, const float* group_scales,
+                   void* packed, size_t packed_bytes, bool scale_bf16, void* stream) {
   if (N <= 0 || K <= 0 || ldw < K || !w || !group_scales || !packed) return QG_ERR_INVALID_ARG;
   if (K % 32) return QG_ERR_UNSUPPORTED;
   if (!aligned(packed, 16) || !aligned(group_scales, 4)) return QG_ERR_MISALIGNED;
-  if (packed_bytes < pack_w4_g32_bytes(N, K)) return QG_ERR_WORKSPACE;
+  const size_t need = scale_bf16 ? pack_w4_g32_bf16_bytes(N, K) : pack_w4_g32_bytes(N, K);
+  if (packed_bytes < need) return QG_ERR_WORKSPACE;
   int rc = device_ready();
   if (rc != QG_OK) return rc;
-  return launch_pack_w4(N, K, w, ldw, group_scales, packed, (cudaStream_t)stream);
+  return launch_pack_w4(N, K, w, ldw, group_scales, packed, scale_bf16, (cudaStream_t)stream);
+}
+
+extern "C" int pack_w4_g32(int N, int K, const int8_t* w, int64_t ldw, const float* group_scales,
+                           void* packed, size_t packed_bytes, void* stream) {
+  return pack_w4(N, K, w, ldw, group_scales, packed, packed_bytes, false, stream);
+}
+
+extern "C" int pack_w4_g32_bf16(int N, int K, const int8_t* w, int64_t ldw,
+                                const float* group_scales, void* packed, size_t packed_bytes,
+                                void* stream) {
+  return pack_w4(N, K, w, ldw, group_scales, packed, packed_bytes, true, stream);
 }
 
 static const int kFusedGemvMaxK = 65536;   // activations held in shared memory
@@ -349,11 +367,10 @@ extern "C" size_t qgemm_a8w4_workspace_bytes(int M, int N, int K) {
   return a8w4_ws_layout(M, K, nullptr, nullptr);
 }
 
-extern "C" int qgemm_a8w4_f32(int M, int N, int K, const float* x, int64_t ldx,
-                              const void* packed_w, const float* bias, float clamp_min,
-                              float clamp_max, float* y, int64_t ldy, int8_t* q_out,
-                              float* scale_out, int32_t* zp_out, void* workspace,
-                              size_t workspace_bytes, void* stream) {
+static int a8w4_linear(int M, int N, int K, const float* x, int64_t ldx, const void* packed_w,
+                       const float* bias, float clamp_min, float clamp_max, float* y,
+                       int64_t ldy, int8_t* q_out, float* scale_out, int32_t* zp_out,
+                       void* workspace, size_t workspace_bytes, bool sbf, void* stream) {
   if (M < 0 || N <= 0 || K <= 0 || ldx < K || ldy < N) return QG_ERR_INVALID_ARG;
   if (K % 32) return QG_ERR_UNSUPPORTED;
   if (!(clamp_min <= clamp_max)) return QG_ERR_INVALID_ARG;  // also rejects NaN
@@ -368,12 +385,12 @@ extern "C" int qgemm_a8w4_f32(int M, int N, int K, const float* x, int64_t ldx,
   cudaStream_t st = (cudaStream_t)stream;
   if (M == 1 && K <= kFusedGemvMaxK)
     return launch_a8w4_gemv(N, K, x, packed_w, bias, clamp_min, clamp_max, y, q_out, scale_out,
-                            zp_out, st);
+                            zp_out, sbf, st);
   if (a8w4_tc_supported(M, N, K)) {
     if (!workspace) return QG_ERR_WORKSPACE;
     if (!aligned(workspace, 256)) return QG_ERR_MISALIGNED;
     return launch_a8w4_tc(M, N, K, x, ldx, packed_w, bias, clamp_min, clamp_max, y, ldy, q_out,
-                          scale_out, zp_out, workspace, workspace_bytes, st);
+                          scale_out, zp_out, workspace, workspace_bytes, sbf, st);
   }
   if (K > kSimtMaxK) return QG_ERR_UNSUPPORTED;
   size_t off_s = 0, off_z = 0;
@@ -393,5 +410,23 @@ extern "C" int qgemm_a8w4_f32(int M, int N, int K, const float* x, int64_t ldx,
   if (zp_out && cudaMemcpyAsync(zp_out, zA, (size_t)M * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
     return QG_ERR_CUDA;
   return launch_a8w4_gemm_simt(M, N, K, q, sA, zA, packed_w, bias, clamp_min, clamp_max, y, ldy,
-                               st);
+                               sbf, st);
+}
+
+extern "C" int qgemm_a8w4_f32(int M, int N, int K, const float* x, int64_t ldx,
+                              const void* packed_w, const float* bias, float clamp_min,
+                              float clamp_max, float* y, int64_t ldy, int8_t* q_out,
+                              float* scale_out, int32_t* zp_out, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  return a8w4_linear(M, N, K, x, ldx, packed_w, bias, clamp_min, clamp_max, y, ldy, q_out,
+                     scale_out, zp_out, workspace, workspace_bytes, false, stream);
+}
+
+extern "C" int qgemm_a8w4_f32_bf16s(int M, int N, int K, const float* x, int64_t ldx,
+                                    const void* packed_w, const float* bias, float clamp_min,
+                                    float clamp_max, float* y, int64_t ldy, int8_t* q_out,
+                                    float* scale_out, int32_t* zp_out, void* workspace,
+                                    size_t workspace_bytes, void* stream) {
+  return a8w4_linear(M, N, K, x, ldx, packed_w, bias, clamp_min, clamp_max, y, ldy, q_out,
+                     scale_out, zp_out, workspace, workspace_bytes, true, stream);
 }

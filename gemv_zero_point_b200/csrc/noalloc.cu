@@ -24,10 +24,10 @@ int launch_quantize_rows(int M, int K, const float* x, int64_t ldx, int8_t* q, i
                          float* scale, int32_t* zp, cudaStream_t st);
 int launch_a8w4_gemv(int N, int K, const float* x, const void* packed, const float* bias,
                      float lo, float hi, float* y, int8_t* q_out, float* scale_out,
-                     int32_t* zp_out, cudaStream_t st);
+                     int32_t* zp_out, bool scale_bf16, cudaStream_t st);
 int launch_a8w4_gemm_simt(int M, int N, int K, const int8_t* q, const float* sA,
                           const int32_t* zA, const void* packed, const float* bias, float lo,
-                          float hi, float* y, int64_t ldy, cudaStream_t st);
+                          float hi, float* y, int64_t ldy, bool scale_bf16, cudaStream_t st);
 int device_setup_status();
 
 namespace {
@@ -90,7 +90,7 @@ extern "C" int qgemm_a8w4_f32_noalloc(int M, int N, int K, const float* x, int64
   cudaStream_t st = (cudaStream_t)stream;
   if (M == 1 && K <= kFusedGemvMaxK)  // the fused GEMV keeps its scratch in shared memory
     return launch_a8w4_gemv(N, K, x, packed_w, bias, clamp_min, clamp_max, y, nullptr, nullptr,
-                            nullptr, st);
+                            nullptr, false, st);
   if (K > kSimtMaxK) return QG_ERR_UNSUPPORTED;
   if (M > kMaxRows || (size_t)M * (size_t)K > kMaxCodes) return QG_ERR_WORKSPACE;
   uint8_t* s = nullptr;
@@ -104,5 +104,5 @@ extern "C" int qgemm_a8w4_f32_noalloc(int M, int N, int K, const float* x, int64
   rc = launch_quantize_rows(M, K, x, ldx, q, K, sA, zA, st);
   if (rc != QG_OK) return rc;
   return launch_a8w4_gemm_simt(M, N, K, q, sA, zA, packed_w, bias, clamp_min, clamp_max, y, ldy,
-                               st);
+                               false, st);
 }

@@ -236,6 +236,30 @@ int qgemm_a8w4_f32(int M, int N, int K, const float* x, int64_t ldx,
                    void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * A8W4 with bf16 group scales.  [KAI] review of the packing call: the Kleidi
+ * packing is passed a bf16 type for the group scales, kept as bf16 to save
+ * space (scale bytes drop from 1/4 to 1/8 of the nibble bytes).
+ *   pack_w4_g32_bf16: as pack_w4_g32, except that each f32 group scale is
+ *   rounded to bf16 (round to nearest, ties to even) and stored in 2 bytes:
+ *   [N][K/2] nibble bytes, then [N][K/32] bf16 scales; size from
+ *   pack_w4_g32_bf16_bytes (0 when K % 32 != 0).  Same argument checks and
+ *   status codes as pack_w4_g32.
+ *   qgemm_a8w4_f32_bf16s: qgemm_a8w4_f32 on weights packed that way; the
+ *   formula above holds with sw[n,g] the stored bf16 value (widened to f32
+ *   exactly).  Arguments, workspace (qgemm_a8w4_workspace_bytes), layouts,
+ *   the stream ordering note and status codes are those of qgemm_a8w4_f32.
+ * ------------------------------------------------------------------------ */
+size_t pack_w4_g32_bf16_bytes(int N, int K);
+int pack_w4_g32_bf16(int N, int K, const int8_t* w, int64_t ldw, const float* group_scales,
+                     void* packed, size_t packed_bytes, void* stream);
+int qgemm_a8w4_f32_bf16s(int M, int N, int K, const float* x, int64_t ldx,
+                         const void* packed_w, const float* bias,
+                         float clamp_min, float clamp_max,
+                         float* y, int64_t ldy,
+                         int8_t* q_out, float* scale_out, int32_t* zp_out,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * qgemm_a8w4_f32 without a workspace.  The pages have no counterpart: this
  * entry point exists for callers that cannot allocate device memory for
  * scratch — a plugin inside a host framework that owns the allocator and

@@ -17,6 +17,7 @@ NULL = None
 def test_exports_every_declared_symbol():
     names = qg.exported_symbols()
     for expected in ["quantize_rows_a8", "pack_w4_g32", "qgemm_a8w4_f32", "qgemm_s8s8_requant",
+                     "pack_w4_g32_bf16", "qgemm_a8w4_f32_bf16s",
                      "qconv2d_s8_im2col", "qgemm_pack_b_s8", "qgemm_s8s8_requant_packed",
                      "qg_requant_params", "qg_status_string", "qg_device_status"]:
         assert expected in names
@@ -52,6 +53,8 @@ def test_requant_params_match_oracle_bit_exact():
 def test_workspace_queries():
     assert qg.pack_w4_g32_bytes(14336, 4096) == 14336 * 2048 + 14336 * 128 * 4
     assert qg.pack_w4_g32_bytes(10, 33) == 0          # K % 32 != 0
+    assert lib.pack_w4_g32_bf16_bytes(14336, 4096) == 14336 * 2048 + 14336 * 128 * 2
+    assert lib.pack_w4_g32_bf16_bytes(10, 33) == 0
     assert qg.qgemm_a8w4_workspace_bytes(1, 14336, 4096) == 0  # fused GEMV needs none
     assert qg.qgemm_a8w4_workspace_bytes(128, 4096, 4096) >= 128 * 4096 + 2 * 128 * 4
     assert qg.qgemm_pack_b_s8_bytes(129, 70) >= 256 * 256 + 256 * 4
@@ -122,3 +125,15 @@ def test_conv_validation():
     assert c(*args, FAKE, FAKE, FAKE, ctypes.byref(rqb), NULL, FAKE, 1 << 30, NULL) == -4
     big = [1, 8, 8, 4000, 4, 3, 3, 1, 1, 1, 1]         # K = 36000 breaks the bound
     assert c(*big, FAKE, FAKE, FAKE, ctypes.byref(rq), NULL, FAKE, 1 << 30, NULL) == -3
+
+
+def test_bf16_scale_entry_points_validate_like_f32_ones():
+    p = lib.pack_w4_g32_bf16
+    assert p(4, 48, FAKE, 48, FAKE, FAKE, 1 << 20, NULL) == -4      # K % 32
+    assert p(4, 64, FAKE, 63, FAKE, FAKE, 1 << 20, NULL) == -1      # ldw < K
+    assert p(4, 64, FAKE, 64, FAKE, ctypes.c_void_p(0x10008), 1 << 20, NULL) == -2
+    assert p(4, 64, FAKE, 64, FAKE, FAKE, 4 * 32 + 4 * 2 * 2 - 1, NULL) == -7   # one byte short
+    f = lib.qgemm_a8w4_f32_bf16s
+    assert f(1, 8, 48, FAKE, 48, FAKE, NULL, -1.0, 1.0, FAKE, 8, NULL, NULL, NULL, NULL, 0, NULL) == -4
+    assert f(1, 8, 64, FAKE, 64, FAKE, NULL, 1.0, -1.0, FAKE, 8, NULL, NULL, NULL, NULL, 0, NULL) == -1
+    assert f(0, 8, 64, FAKE, 64, FAKE, NULL, -1.0, 1.0, FAKE, 8, NULL, NULL, NULL, NULL, 0, NULL) == 0

@@ -97,16 +97,17 @@ def test_pack_w4_out_of_range_recorded(lib):
 # ---------------------------------------------------------------------------
 # A8W4 linear
 # ---------------------------------------------------------------------------
-def _run_a8w4(lib, w, ldy_pad=0, with_outputs=True):
+def _run_a8w4(lib, w, ldy_pad=0, with_outputs=True, bf16=False):
     M, N, K = w["M"], w["N"], w["K"]
-    packed = lib.pack_w4_g32(_dev(w["qw"]), _dev(w["sw"]))
+    packed = lib.pack_w4_g32(_dev(w["qw"]), _dev(w["sw"]), bf16_scales=bf16)
     x = _dev(w["x"])[:, :K]
     y = torch.full((M, N + ldy_pad), 7.0, dtype=torch.float32, device="cuda")
     q = torch.empty((M, K), dtype=torch.int8, device="cuda") if with_outputs else None
     s = torch.empty(M, dtype=torch.float32, device="cuda") if with_outputs else None
     z = torch.empty(M, dtype=torch.int32, device="cuda") if with_outputs else None
     bias = None if w["bias"] is None else _dev(w["bias"])
-    lib.qgemm_a8w4_f32(x, packed, N, bias, w["clamp_min"], w["clamp_max"], y[:, :N], q, s, z)
+    lib.qgemm_a8w4_f32(x, packed, N, bias, w["clamp_min"], w["clamp_max"], y[:, :N], q, s, z,
+                       bf16_scales=bf16)
     torch.cuda.synchronize()
     y_np = y.cpu().numpy()
     if ldy_pad:
@@ -117,10 +118,11 @@ def _run_a8w4(lib, w, ldy_pad=0, with_outputs=True):
     return out
 
 
-def _check_a8w4(lib, w, **kw):
-    y, q, s, z = _run_a8w4(lib, w, **kw)
-    y_ref, q_ref, s_ref, z_ref = oracle.qgemm_a8w4_f32(w["x"][:, :w["K"]], w["qw"], w["sw"],
-                                                       w["bias"], w["clamp_min"], w["clamp_max"])
+def _check_a8w4(lib, w, bf16=False, **kw):
+    y, q, s, z = _run_a8w4(lib, w, bf16=bf16, **kw)
+    ref = oracle.qgemm_a8w4_f32_bf16s if bf16 else oracle.qgemm_a8w4_f32
+    y_ref, q_ref, s_ref, z_ref = ref(w["x"][:, :w["K"]], w["qw"], w["sw"], w["bias"],
+                                     w["clamp_min"], w["clamp_max"])
     np.testing.assert_array_equal(q, q_ref)
     np.testing.assert_array_equal(s.view(np.int32), s_ref.view(np.int32))
     np.testing.assert_array_equal(z, z_ref)
@@ -184,3 +186,35 @@ def test_gemv_chain_on_one_stream(lib):
         y_np = y.cpu().numpy()
         assert_a8w4_close(y_np, y_ref)
         xin = y_np
+
+
+# ---------------------------------------------------------------------------
+# A8W4 with bf16 group scales (pack_w4_g32_bf16 / qgemm_a8w4_f32_bf16s)
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("N,K", [(7, 96), (300, 1024), (14336, 4096)])
+def test_pack_w4_bf16_bit_exact(lib, N, K):
+    w = workloads.a8w4(1, N, K, seed=N + K + 1)
+    packed = lib.pack_w4_g32_bf16(_dev(w["qw"]), _dev(w["sw"]))
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(packed.cpu().numpy(), oracle.pack_w4_g32_bf16(w["qw"], w["sw"]))
+
+
+def test_gemv_bf16_scales_full_size_cfg2(lib):
+    _check_a8w4(lib, workloads.cfg2_gemv(), bf16=True)
+
+
+@pytest.mark.parametrize("M,N,K", [
+    (1, 300, 1024),      # streaming GEMV
+    (1, 1000, 2080),     # plain GEMV (K % 128 != 0)
+    (1, 17, 12288),      # plain GEMV (K > 8192)
+    (9, 300, 1024),      # tensor cores
+    (129, 520, 384),     # tensor cores, ragged M
+    (5, 96, 96),         # CUDA cores (K % 128 != 0)
+])
+def test_a8w4_bf16_scales_shapes(lib, M, N, K):
+    w = workloads.a8w4(M, N, K, seed=M * 13 + N + K, clamp=(-np.inf, np.inf), ldx=K + 1)
+    _check_a8w4(lib, w, bf16=True, ldy_pad=1)
+
+
+def test_a8w4_bf16_scales_full_size_cfg3(lib):
+    _check_a8w4(lib, workloads.cfg3_gemm(), bf16=True)
