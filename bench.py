@@ -21,8 +21,10 @@ it: 2 GEMM sets (A + packed B = 135 MB each) and 8 GEMV weight sets (36.8 MB
 each, 295 MB in all).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
-                  [--workload headline|cfg0|cfg1|cfg2|cfg2b|cfg3|cfg4] [--no-cpu-baseline]
-(cfg2b: the A8W4 GEMV with bf16 group scales.)
+                  [--workload headline|<one workload name below>] [--no-cpu-baseline]
+Workloads: int8_gemm_130x70x129, int8_conv_56x56x64_3x3, a8w4_gemv_1x14336x4096,
+a8w4_gemv_bf16s_1x14336x4096 (bf16 group scales), a8w4_gemm_128x4096x4096,
+int8_gemm_8192x8192x8200.
 Under torchrun each rank runs the same work on its own GPU (replicas: the
 path has no exchange step), and value sums all ranks' work.
 """
@@ -365,20 +367,20 @@ class ConvCase:
 def build_cases(workload, qg, torch):
     import workloads as W
     if workload == "headline":
-        return [("int8_gemm_8192x8192x8200", GemmCase(qg, torch, W.cfg4_gemm_large(), 2), "tensor"),
-                ("a8w4_gemv_1x14336x4096", A8W4Case(qg, torch, W.cfg2_gemv(), 8), "hbm")]
-    if workload == "cfg0":
-        return [("int8_gemm_130x70x129", GemmCase(qg, torch, W.cfg0_gemm_small(), 1), "latency")]
-    if workload == "cfg1":
-        return [("int8_conv_56x56x64_3x3", ConvCase(qg, torch, W.cfg1_conv(), 1), "latency")]
-    if workload == "cfg2":
-        return [("a8w4_gemv_1x14336x4096", A8W4Case(qg, torch, W.cfg2_gemv(), 8), "hbm")]
-    if workload == "cfg3":
-        return [("a8w4_gemm_128x4096x4096", A8W4Case(qg, torch, W.cfg3_gemm(), 16), "hbm")]
-    if workload == "cfg2b":   # the GEMV with bf16 group scales (9 sets: 298 MB > L2)
-        return [("a8w4_gemv_bf16s_1x14336x4096", A8W4Case(qg, torch, W.cfg2_gemv(), 9, True), "hbm")]
-    if workload == "cfg4":
-        return [("int8_gemm_8192x8192x8200", GemmCase(qg, torch, W.cfg4_gemm_large(), 2), "tensor")]
+        return [("int8_gemm_8192x8192x8200", GemmCase(qg, torch, W.int8_gemm_8192x8192x8200(), 2), "tensor"),
+                ("a8w4_gemv_1x14336x4096", A8W4Case(qg, torch, W.a8w4_gemv_1x14336x4096(), 8), "hbm")]
+    if workload == "int8_gemm_130x70x129":
+        return [("int8_gemm_130x70x129", GemmCase(qg, torch, W.int8_gemm_130x70x129(), 1), "latency")]
+    if workload == "int8_conv_56x56x64_3x3":
+        return [("int8_conv_56x56x64_3x3", ConvCase(qg, torch, W.int8_conv_56x56x64_3x3(), 1), "latency")]
+    if workload == "a8w4_gemv_1x14336x4096":
+        return [("a8w4_gemv_1x14336x4096", A8W4Case(qg, torch, W.a8w4_gemv_1x14336x4096(), 8), "hbm")]
+    if workload == "a8w4_gemm_128x4096x4096":
+        return [("a8w4_gemm_128x4096x4096", A8W4Case(qg, torch, W.a8w4_gemm_128x4096x4096(), 16), "hbm")]
+    if workload == "a8w4_gemv_bf16s_1x14336x4096":   # the GEMV with bf16 group scales (9 sets: 298 MB > L2)
+        return [("a8w4_gemv_bf16s_1x14336x4096", A8W4Case(qg, torch, W.a8w4_gemv_1x14336x4096(), 9, True), "hbm")]
+    if workload == "int8_gemm_8192x8192x8200":
+        return [("int8_gemm_8192x8192x8200", GemmCase(qg, torch, W.int8_gemm_8192x8192x8200(), 2), "tensor")]
     raise SystemExit(f"unknown workload {workload}")
 
 
@@ -430,8 +432,8 @@ def oracle_sample(workload, budget_s=12.0, rows_gemm=None, small=False):
     import oracle
     import workloads as W
     ops, spent, parts = 0.0, 0.0, []
-    if workload in ("headline", "cfg4"):
-        w = W.cfg4_gemm_large()
+    if workload in ("headline", "int8_gemm_8192x8192x8200"):
+        w = W.int8_gemm_8192x8192x8200()
         m0 = np.array([oracle.requant_params(float(r))[0] for r in w["ratio"]])
         sh = np.array([oracle.requant_params(float(r))[1] for r in w["ratio"]])
         cols = 512 if small else w["N"]
@@ -443,25 +445,25 @@ def oracle_sample(workload, budget_s=12.0, rows_gemm=None, small=False):
         dt = time.perf_counter() - t
         ops += gemm_ops(rows, cols, w["K"]); spent += dt
         parts.append(f"int8 GEMM {rows} row(s) x {cols} cols of 8192x8192x8200")
-    if workload in ("headline", "cfg2", "cfg2b"):
-        w = W.cfg2_gemv()
+    if workload in ("headline", "a8w4_gemv_1x14336x4096", "a8w4_gemv_bf16s_1x14336x4096"):
+        w = W.a8w4_gemv_1x14336x4096()
         n = 512 if small else w["N"]
         t = time.perf_counter()
-        fn = oracle.qgemm_a8w4_f32_bf16s if workload == "cfg2b" else oracle.qgemm_a8w4_f32
+        fn = oracle.qgemm_a8w4_f32_bf16s if workload == "a8w4_gemv_bf16s_1x14336x4096" else oracle.qgemm_a8w4_f32
         fn(w["x"], w["qw"][:n], w["sw"][:n], w["bias"][:n], -6.0, 6.0)
         dt = time.perf_counter() - t
         ops += a8w4_ops(1, n, w["K"]); spent += dt
-        parts.append(f"A8W4 GEMV{' (bf16 scales)' if workload == 'cfg2b' else ''} {n} of 14336 rows")
-    if workload == "cfg3":
-        w = W.cfg3_gemm()
+        parts.append(f"A8W4 GEMV{' (bf16 scales)' if workload == 'a8w4_gemv_bf16s_1x14336x4096' else ''} {n} of 14336 rows")
+    if workload == "a8w4_gemm_128x4096x4096":
+        w = W.a8w4_gemm_128x4096x4096()
         rows = 1 if small else 4
         t = time.perf_counter()
         oracle.qgemm_a8w4_f32(w["x"][:rows], w["qw"], w["sw"], w["bias"], -6.0, 6.0)
         dt = time.perf_counter() - t
         ops += a8w4_ops(rows, w["N"], w["K"]); spent += dt
         parts.append(f"A8W4 GEMM {rows} of 128 rows")
-    if workload == "cfg0":
-        w = W.cfg0_gemm_small()
+    if workload == "int8_gemm_130x70x129":
+        w = W.int8_gemm_130x70x129()
         m0, sh = oracle.requant_params(float(w["ratio"][0]))
         t = time.perf_counter()
         oracle.qgemm_s8s8_requant(w["A"], w["B"], w["za"], w["zb"], w["bias"], m0, sh,
@@ -469,8 +471,8 @@ def oracle_sample(workload, budget_s=12.0, rows_gemm=None, small=False):
         dt = time.perf_counter() - t
         ops += gemm_ops(130, 70, 129); spent += dt
         parts.append("int8 GEMM 130x70x129 (whole)")
-    if workload == "cfg1":
-        w = W.cfg1_conv()
+    if workload == "int8_conv_56x56x64_3x3":
+        w = W.int8_conv_56x56x64_3x3()
         pr = [oracle.requant_params(float(r)) for r in w["ratio"]]
         m0 = np.array([p[0] for p in pr]); sh = np.array([p[1] for p in pr])
         t = time.perf_counter()
@@ -517,7 +519,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="headline",
-                    choices=["headline", "cfg0", "cfg1", "cfg2", "cfg2b", "cfg3", "cfg4"])
+                    choices=["headline", "int8_gemm_130x70x129", "int8_conv_56x56x64_3x3", "a8w4_gemv_1x14336x4096", "a8w4_gemv_bf16s_1x14336x4096", "a8w4_gemm_128x4096x4096", "int8_gemm_8192x8192x8200"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=10)
     args = ap.parse_args()

@@ -130,8 +130,8 @@ def _check_a8w4(lib, w, bf16=False, **kw):
     return y, y_ref
 
 
-def test_gemv_full_size_cfg2(lib):
-    w = workloads.cfg2_gemv()
+def test_gemv_full_size_1x14336x4096(lib):
+    w = workloads.a8w4_gemv_1x14336x4096()
     y, y_ref = _check_a8w4(lib, w)
     # the clamp binds on a large share of outputs at this scale; both sides agree where it does
     assert ((np.abs(y_ref) == 6.0) == (np.abs(y) == 6.0)).mean() > 0.999
@@ -155,8 +155,8 @@ def test_a8w4_gemm_shapes(lib, M, N, K):
     _check_a8w4(lib, w, ldy_pad=1)
 
 
-def test_a8w4_gemm_full_size_cfg3(lib):
-    _check_a8w4(lib, workloads.cfg3_gemm())
+def test_a8w4_gemm_full_size_128x4096x4096(lib):
+    _check_a8w4(lib, workloads.a8w4_gemm_128x4096x4096())
 
 
 def test_gemv_without_optional_outputs_matches(lib):
@@ -199,8 +199,8 @@ def test_pack_w4_bf16_bit_exact(lib, N, K):
     np.testing.assert_array_equal(packed.cpu().numpy(), oracle.pack_w4_g32_bf16(w["qw"], w["sw"]))
 
 
-def test_gemv_bf16_scales_full_size_cfg2(lib):
-    _check_a8w4(lib, workloads.cfg2_gemv(), bf16=True)
+def test_gemv_bf16_scales_full_size_1x14336x4096(lib):
+    _check_a8w4(lib, workloads.a8w4_gemv_1x14336x4096(), bf16=True)
 
 
 @pytest.mark.parametrize("M,N,K", [
@@ -216,5 +216,5 @@ def test_a8w4_bf16_scales_shapes(lib, M, N, K):
     _check_a8w4(lib, w, bf16=True, ldy_pad=1)
 
 
-def test_a8w4_bf16_scales_full_size_cfg3(lib):
-    _check_a8w4(lib, workloads.cfg3_gemm(), bf16=True)
+def test_a8w4_bf16_scales_full_size_128x4096x4096(lib):
+    _check_a8w4(lib, workloads.a8w4_gemm_128x4096x4096(), bf16=True)

@@ -75,15 +75,15 @@ def check_gemm(lib, w, rows=None, **kw):
     return C, C_ref
 
 
-def test_gemm_cfg0_bit_exact(lib):
-    w = workloads.cfg0_gemm_small()
+def test_gemm_130x70x129_bit_exact(lib):
+    w = workloads.int8_gemm_130x70x129()
     C, C_ref = check_gemm(lib, w)
     # the outputs are not trivially saturated
     assert 0.05 < np.mean(np.abs(C_ref.astype(int)) < 127)
 
 
-def test_gemm_cfg0_packed_bit_exact(lib):
-    check_gemm(lib, workloads.cfg0_gemm_small(), packed=True, ldc_pad=3)
+def test_gemm_130x70x129_packed_bit_exact(lib):
+    check_gemm(lib, workloads.int8_gemm_130x70x129(), packed=True, ldc_pad=3)
 
 
 SHAPES = [(1, 1, 1), (2, 16, 31), (127, 70, 129), (128, 256, 128), (129, 257, 256),
@@ -139,8 +139,8 @@ def test_gemm_deterministic(lib):
     np.testing.assert_array_equal(a1, a2)
 
 
-def test_gemm_cfg4_full_size_sampled_rows(lib):
-    w = workloads.cfg4_gemm_large()
+def test_gemm_8192x8192x8200_sampled_rows(lib):
+    w = workloads.int8_gemm_8192x8192x8200()
     rows = np.array([0, 1, 127, 128, 129, 2047, 4096, 5000, 8063, 8064, 8190, 8191])
     C, C_ref = check_gemm(lib, w, packed=True, rows=rows)
     # every column of the sampled rows is checked; outputs are not all saturated
@@ -169,8 +169,8 @@ def run_conv(lib, w, with_acc=True):
     return y_ref
 
 
-def test_conv_cfg1_bit_exact(lib):
-    y_ref = run_conv(lib, workloads.cfg1_conv())
+def test_conv_56x56x64_bit_exact(lib):
+    y_ref = run_conv(lib, workloads.int8_conv_56x56x64_3x3())
     assert (y_ref == -10).mean() > 0.05      # the ReLU floor at the out zero-point binds
 
 

@@ -57,7 +57,7 @@ def test_reference_arm_prints_on_rank0_only():
                    MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), CUDA_VISIBLE_DEVICES="")
         procs.append(subprocess.Popen(
             [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2",
-             "--steps", "1", "--warmup", "3", "--workload", "cfg0"],
+             "--steps", "1", "--warmup", "3", "--workload", "int8_gemm_130x70x129"],
             env=env, stdout=subprocess.PIPE, stderr=subprocess.PIPE, text=True))
     outs = [p.communicate(timeout=300) for p in procs]
     for p, (o, e) in zip(procs, outs):

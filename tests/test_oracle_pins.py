@@ -29,7 +29,7 @@ def _golden(name):
 # ---------------------------------------------------------------------------
 def test_p1_tiling_counts_match_page():
     g = _golden("qg_tiling_130x70x129.json")
-    w = workloads.cfg0_gemm_small()
+    w = workloads.int8_gemm_130x70x129()
     assert (w["M"], w["N"], w["K"]) == (g["M"], g["N"], g["K"])
     A, B = w["A"][:, :w["K"]], w["B"][:, :w["N"]]
     acc_t, st = oracle.tiled_int8_gemm(A, B, w["za"], w["zb"], w["bias"],
@@ -89,7 +89,7 @@ def test_p2_bound_edge_and_rejection():
 # P3: padding stands for real zero (section 2)
 # ---------------------------------------------------------------------------
 def test_p3_zero_point_padding_invariance():
-    w = workloads.cfg0_gemm_small()
+    w = workloads.int8_gemm_130x70x129()
     A, B = w["A"][:, :129], w["B"][:, :70]
     za, zb = 11, -7        # non-zero on both sides so raw-zero padding is visible
     acc = oracle.int8_gemm_acc(A, B, za, zb, w["bias"])
@@ -157,7 +157,7 @@ def test_conv_brute_force_loops():
 # P4: accumulate across K, requantize once (section 4)
 # ---------------------------------------------------------------------------
 def test_p4_k_block_accumulation():
-    w = workloads.cfg0_gemm_small()
+    w = workloads.int8_gemm_130x70x129()
     A, B = w["A"][:, :129], w["B"][:, :70]
     acc = oracle.int8_gemm_acc(A, B, w["za"], w["zb"])
     parts = [oracle.int8_gemm_acc(A[:, k:k + 32], B[k:k + 32], w["za"], w["zb"])

@@ -76,12 +76,12 @@ def int8_gemm(M, N, K, seed, *, za=None, zb=None, za_range=(-20, 20),
                 out_zp=int(out_zp), clamp_min=int(clamp[0]), clamp_max=int(clamp[1]))
 
 
-def cfg0_gemm_small(seed=1001):
+def int8_gemm_130x70x129(seed=1001):
     """Affine INT8 GEMM M=130, N=70, K=129 (tails in all three dims)."""
     return int8_gemm(130, 70, 129, seed)
 
 
-def cfg4_gemm_large(seed=1005):
+def int8_gemm_8192x8192x8200(seed=1005):
     """INT8 GEMM M=N=8192, K=8200 (K tail 8 past 64 blocks of 128), za=7,
     symmetric B with per-column scales log-uniform [1e-3, 1e-1],
     sA/sO = 0.01 so per-column ratios lie in [1e-5, 1e-3]."""
@@ -108,7 +108,7 @@ def int8_conv(Nb, H, W, Cin, Cout, KH, KW, stride, pad, seed, *, za=-5,
                 clamp_max=INT8_MAX)
 
 
-def cfg1_conv(seed=1002):
+def int8_conv_56x56x64_3x3(seed=1002):
     """1x56x56x64 -> 64, 3x3, stride 1, pad 1, input zp -5 (also the pad
     value), per-Cout weight scales, fused ReLU (clamp floor = out zp)."""
     return int8_conv(1, 56, 56, 64, 64, 3, 3, (1, 1), (1, 1), seed)
@@ -132,20 +132,20 @@ def a8w4(M, N, K, seed, *, clamp=(-6.0, 6.0), with_bias=True, ldx=None):
                 clamp_min=float(clamp[0]), clamp_max=float(clamp[1]))
 
 
-def cfg2_gemv(seed=1003):
+def a8w4_gemv_1x14336x4096(seed=1003):
     """A8W4 GEMV M=1, N=14336, K=4096."""
     return a8w4(1, 14336, 4096, seed)
 
 
-def cfg3_gemm(seed=1004):
+def a8w4_gemm_128x4096x4096(seed=1004):
     """A8W4 GEMM M=128, N=4096, K=4096."""
     return a8w4(128, 4096, 4096, seed)
 
 
 WORKLOADS = {
-    "cfg0_int8_gemm_130x70x129": cfg0_gemm_small,
-    "cfg1_int8_conv_56x56x64_3x3": cfg1_conv,
-    "cfg2_a8w4_gemv_1x14336x4096": cfg2_gemv,
-    "cfg3_a8w4_gemm_128x4096x4096": cfg3_gemm,
-    "cfg4_int8_gemm_8192x8192x8200": cfg4_gemm_large,
+    "int8_gemm_130x70x129": int8_gemm_130x70x129,
+    "int8_conv_56x56x64_3x3": int8_conv_56x56x64_3x3,
+    "a8w4_gemv_1x14336x4096": a8w4_gemv_1x14336x4096,
+    "a8w4_gemm_128x4096x4096": a8w4_gemm_128x4096x4096,
+    "int8_gemm_8192x8192x8200": int8_gemm_8192x8192x8200,
 }
