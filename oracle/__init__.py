@@ -307,6 +307,21 @@ def quantize_rows_a8(x):
     return q, scale, zp
 
 
+def quantize_blocks_a8(x, block):
+    """Per-block dynamic quantization ([MNN] ConvInt8TiledExecutor: with the
+    dynamic-quant option 2 the input is quantized in as many K blocks as the
+    weights have quant blocks, each with its own scale and zero-point).
+    READING R13: block = the weight group size; every block of `block`
+    consecutive k of a row is quantized by the per-row rule above (R5).
+    Returns q int8 [M][K], scale float32 [M][K/block], zp int32 [M][K/block].
+    """
+    x = np.asarray(x, dtype=np.float32)
+    M, K = x.shape
+    assert K % block == 0
+    q, s, z = quantize_rows_a8(x.reshape(M * (K // block), block))
+    return q.reshape(M, K), s.reshape(M, K // block), z.reshape(M, K // block)
+
+
 def dequantize_rows(q, scale, zp):
     """real = scale * (q - zero_point)  ([QG] section 1), in float64."""
     return (np.asarray(scale, np.float64)[:, None]
@@ -433,3 +448,29 @@ def qgemm_a8w4_f32(x, qw, sw, bias, clamp_min, clamp_max):
 def qgemm_a8w4_f32_bf16s(x, qw, sw, bias, clamp_min, clamp_max):
     """O4 with every group scale replaced by its bf16 value (O5, R12)."""
     return qgemm_a8w4_f32(x, qw, bf16_scales(sw), bias, clamp_min, clamp_max)
+
+
+def qgemm_a8w4_f32_actblock(x, qw, sw, bias, clamp_min, clamp_max):
+    """O4 with the activations quantized per 32-wide K block (O6, R13):
+        y[m,n] = clamp(f32( sum_g sw[n,g]*sA[m,g]*I[m,n,g] + bias[n] ), lo, hi)
+        I[m,n,g] = sum_{k in group g} (qA[m,k]-za[m,g]) * qw[n,k]   (exact int)
+    with the combination over groups in float64.
+    Returns (y float32 [M,N], qA int8 [M,K], sA float32 [M,G], za int32 [M,G]).
+    """
+    qw = np.asarray(qw, dtype=np.int64)
+    N, K = qw.shape
+    G = K // GROUP
+    qA, sA, za = quantize_blocks_a8(x, GROUP)
+    M = qA.shape[0]
+    swd = np.asarray(sw, dtype=np.float64)
+    wg = qw.reshape(N, G, GROUP)
+    y = np.empty((M, N), dtype=np.float32)
+    lo, hi = np.float32(clamp_min), np.float32(clamp_max)
+    for m in range(M):
+        a = qA[m].astype(np.int64).reshape(G, GROUP) - za[m].astype(np.int64)[:, None]
+        I = np.einsum("gj,ngj->ng", a, wg)                       # exact
+        comb = (swd * sA[m].astype(np.float64)[None, :] * I.astype(np.float64)).sum(axis=1)
+        if bias is not None:
+            comb = comb + np.asarray(bias, np.float64)
+        y[m] = np.minimum(np.maximum(comb.astype(np.float32), lo), hi)
+    return y, qA, sA, za

@@ -407,3 +407,61 @@ def test_p9_bf16_linear_equals_f32_linear_on_representable_scales():
     y16g = oracle.qgemm_a8w4_f32_bf16s(w["x"], w["qw"], w["sw"], w["bias"], -6.0, 6.0)[0]
     y32r = oracle.qgemm_a8w4_f32(w["x"], w["qw"], oracle.bf16_scales(w["sw"]), w["bias"], -6.0, 6.0)[0]
     np.testing.assert_array_equal(y16g, y32r)
+
+
+# ---------------------------------------------------------------------------
+# P10: per-block activation quantization (reading R13: 32-wide K blocks, the
+# per-row rule applied to each block)
+# ---------------------------------------------------------------------------
+def test_p10_one_block_per_row_is_the_per_row_rule():
+    x = np.random.default_rng(3).standard_normal((4, 256)).astype(np.float32)
+    qb, sb, zb = oracle.quantize_blocks_a8(x, 256)
+    qr, sr, zr = oracle.quantize_rows_a8(x)
+    np.testing.assert_array_equal(qb, qr)
+    np.testing.assert_array_equal(sb[:, 0], sr)
+    np.testing.assert_array_equal(zb[:, 0], zr)
+
+
+def test_p10_block_specials_and_reconstruction():
+    rng = np.random.default_rng(4)
+    x = rng.standard_normal((2, 128)).astype(np.float32) * np.repeat(
+        np.float32(10.0) ** rng.integers(-3, 3, (2, 4)), 32, axis=1)
+    x[0, 32:64] = 0.0                           # an all-zero block
+    x[1, 64:96] = 2.5                           # a constant positive block
+    q, s, z = oracle.quantize_blocks_a8(x, 32)
+    assert s[0, 1] == 1.0 and z[0, 1] == -128 and (q[0, 32:64] == -128).all()
+    # constant 2.5: range [0, 2.5], scale 2.5/255, zp -128, codes 127
+    assert s[1, 2] == np.float32(np.float32(2.5) / np.float32(255.0)) and z[1, 2] == -128
+    assert (q[1, 64:96] == 127).all()
+    # every value is reconstructed within half a step of its own block's scale
+    rec = (s.repeat(32, axis=1).astype(np.float64)
+           * (q.astype(np.float64) - z.repeat(32, axis=1)))
+    assert (np.abs(rec - x) <= 0.5 * s.repeat(32, axis=1) * (1 + 1e-5) + 1e-30).all()
+
+
+def test_p10_blockwise_linear_equals_rowwise_when_blocks_share_the_range():
+    # every block holds the row's min and max: block scales = row scale
+    w = workloads.a8w4(2, 24, 128, seed=6)
+    x = np.asarray(w["x"][:, :128], np.float32).copy()
+    for m in range(2):
+        lo, hi = x[m].min(), x[m].max()
+        for g in range(4):
+            x[m, 32 * g], x[m, 32 * g + 1] = lo, hi
+    yb, qb, sb, zb = oracle.qgemm_a8w4_f32_actblock(x, w["qw"], w["sw"], w["bias"], -6.0, 6.0)
+    yr, qr, sr, zr = oracle.qgemm_a8w4_f32(x, w["qw"], w["sw"], w["bias"], -6.0, 6.0)
+    np.testing.assert_array_equal(sb, np.repeat(sr[:, None], 4, axis=1))
+    np.testing.assert_array_equal(qb, qr)
+    np.testing.assert_array_equal(yb, yr)
+
+
+def test_p10_blockwise_brute_force_loops():
+    w = workloads.a8w4(1, 3, 64, seed=8)
+    x = np.asarray(w["x"][:, :64], np.float32)
+    y, q, s, z = oracle.qgemm_a8w4_f32_actblock(x, w["qw"], w["sw"], w["bias"], -1e30, 1e30)
+    for n in range(3):
+        tot = 0.0
+        for g in range(2):
+            I = sum((int(q[0, k]) - int(z[0, g])) * int(w["qw"][n, k]) for k in range(32 * g, 32 * g + 32))
+            tot += float(w["sw"][n, g]) * float(s[0, g]) * I
+        tot += float(w["bias"][n])
+        assert y[0, n] == np.float32(tot)
