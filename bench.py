@@ -23,7 +23,8 @@ each, 295 MB in all).
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
                   [--workload headline|<one workload name below>] [--no-cpu-baseline]
 Workloads: int8_gemm_130x70x129, int8_conv_56x56x64_3x3, a8w4_gemv_1x14336x4096,
-a8w4_gemv_bf16s_1x14336x4096 (bf16 group scales), a8w4_gemm_128x4096x4096,
+a8w4_gemv_bf16s_1x14336x4096 (bf16 group scales), a8w4_gemv_actblock_1x14336x4096
+(activations quantized per 32-wide K block), a8w4_gemm_128x4096x4096,
 int8_gemm_8192x8192x8200.
 Under torchrun each rank runs the same work on its own GPU (replicas: the
 path has no exchange step), and value sums all ranks' work.
@@ -264,10 +265,11 @@ class GemmCase:
 
 
 class A8W4Case:
-    def __init__(self, qg, torch, w, sets, bf16_scales=False):
+    def __init__(self, qg, torch, w, sets, bf16_scales=False, actblock=False):
         self.M, self.N, self.K = w["M"], w["N"], w["K"]
         self.qg, self.torch = qg, torch
         self.bf16 = bf16_scales
+        self.actblock = actblock  # activations quantized per 32-wide K block (M = 1)
         qw = dev(w["qw"], torch)
         sw = dev(w["sw"], torch)
         self.packed = []
@@ -288,6 +290,10 @@ class A8W4Case:
         self.d2h_host = torch.empty((self.M, self.N), dtype=torch.float32).pin_memory()
 
     def run(self, i, stream=None):
+        if self.actblock:
+            self.qg.qgemm_a8w4_f32_actblock(self.x, self.packed[i % len(self.packed)], self.N,
+                                            self.bias, self.lo, self.hi, self.y, stream=stream)
+            return
         self.qg.qgemm_a8w4_f32(self.x, self.packed[i % len(self.packed)], self.N, self.bias,
                                self.lo, self.hi, self.y, workspace=self.ws, stream=stream,
                                bf16_scales=self.bf16)
@@ -297,8 +303,12 @@ class A8W4Case:
 
     def run_e2e(self, i):
         self.e2e_x.copy_(self.h2d_host, non_blocking=True)
-        self.qg.qgemm_a8w4_f32(self.e2e_x, self.packed[0], self.N, self.bias, self.lo, self.hi,
-                               self.y, workspace=self.ws, bf16_scales=self.bf16)
+        if self.actblock:
+            self.qg.qgemm_a8w4_f32_actblock(self.e2e_x, self.packed[0], self.N, self.bias,
+                                            self.lo, self.hi, self.y)
+        else:
+            self.qg.qgemm_a8w4_f32(self.e2e_x, self.packed[0], self.N, self.bias, self.lo,
+                                   self.hi, self.y, workspace=self.ws, bf16_scales=self.bf16)
         self.d2h_host.copy_(self.y, non_blocking=True)
 
     def ops(self):
@@ -377,6 +387,9 @@ def build_cases(workload, qg, torch):
         return [("a8w4_gemv_1x14336x4096", A8W4Case(qg, torch, W.a8w4_gemv_1x14336x4096(), 8), "hbm")]
     if workload == "a8w4_gemm_128x4096x4096":
         return [("a8w4_gemm_128x4096x4096", A8W4Case(qg, torch, W.a8w4_gemm_128x4096x4096(), 16), "hbm")]
+    if workload == "a8w4_gemv_actblock_1x14336x4096":   # activations quantized per K block
+        return [("a8w4_gemv_actblock_1x14336x4096",
+                 A8W4Case(qg, torch, W.a8w4_gemv_1x14336x4096(), 8, actblock=True), "hbm")]
     if workload == "a8w4_gemv_bf16s_1x14336x4096":   # the GEMV with bf16 group scales (9 sets: 298 MB > L2)
         return [("a8w4_gemv_bf16s_1x14336x4096", A8W4Case(qg, torch, W.a8w4_gemv_1x14336x4096(), 9, True), "hbm")]
     if workload == "int8_gemm_8192x8192x8200":
@@ -395,6 +408,7 @@ KERNEL_SOURCES = {
     "a8w4_gemv_1x14336x4096": "a8w4.cu",
     "a8w4_gemm_128x4096x4096": "a8w4_tc.cu",
     "a8w4_gemv_bf16s_1x14336x4096": "a8w4.cu",
+    "a8w4_gemv_actblock_1x14336x4096": "a8w4.cu",
 }
 
 
@@ -445,15 +459,20 @@ def oracle_sample(workload, budget_s=12.0, rows_gemm=None, small=False):
         dt = time.perf_counter() - t
         ops += gemm_ops(rows, cols, w["K"]); spent += dt
         parts.append(f"int8 GEMM {rows} row(s) x {cols} cols of 8192x8192x8200")
-    if workload in ("headline", "a8w4_gemv_1x14336x4096", "a8w4_gemv_bf16s_1x14336x4096"):
+    if workload in ("headline", "a8w4_gemv_1x14336x4096", "a8w4_gemv_bf16s_1x14336x4096",
+                    "a8w4_gemv_actblock_1x14336x4096"):
         w = W.a8w4_gemv_1x14336x4096()
         n = 512 if small else w["N"]
         t = time.perf_counter()
-        fn = oracle.qgemm_a8w4_f32_bf16s if workload == "a8w4_gemv_bf16s_1x14336x4096" else oracle.qgemm_a8w4_f32
+        fn = {"a8w4_gemv_bf16s_1x14336x4096": oracle.qgemm_a8w4_f32_bf16s,
+              "a8w4_gemv_actblock_1x14336x4096": oracle.qgemm_a8w4_f32_actblock}.get(
+                  workload, oracle.qgemm_a8w4_f32)
         fn(w["x"], w["qw"][:n], w["sw"][:n], w["bias"][:n], -6.0, 6.0)
         dt = time.perf_counter() - t
         ops += a8w4_ops(1, n, w["K"]); spent += dt
-        parts.append(f"A8W4 GEMV{' (bf16 scales)' if workload == 'a8w4_gemv_bf16s_1x14336x4096' else ''} {n} of 14336 rows")
+        tag = {"a8w4_gemv_bf16s_1x14336x4096": " (bf16 scales)",
+               "a8w4_gemv_actblock_1x14336x4096": " (per-block activations)"}.get(workload, "")
+        parts.append(f"A8W4 GEMV{tag} {n} of 14336 rows")
     if workload == "a8w4_gemm_128x4096x4096":
         w = W.a8w4_gemm_128x4096x4096()
         rows = 1 if small else 4
@@ -519,7 +538,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="headline",
-                    choices=["headline", "int8_gemm_130x70x129", "int8_conv_56x56x64_3x3", "a8w4_gemv_1x14336x4096", "a8w4_gemv_bf16s_1x14336x4096", "a8w4_gemm_128x4096x4096", "int8_gemm_8192x8192x8200"])
+                    choices=["headline", "int8_gemm_130x70x129", "int8_conv_56x56x64_3x3", "a8w4_gemv_1x14336x4096", "a8w4_gemv_bf16s_1x14336x4096", "a8w4_gemv_actblock_1x14336x4096", "a8w4_gemm_128x4096x4096", "int8_gemm_8192x8192x8200"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=10)
     args = ap.parse_args()

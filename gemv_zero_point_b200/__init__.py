@@ -88,6 +88,8 @@ _sig("pack_w4_g32", _i32, [_i32, _i32, _vp, _i64, _vp, _vp, _sz, _vp])
 _sig("qgemm_a8w4_workspace_bytes", _sz, [_i32, _i32, _i32])
 _sig("qgemm_a8w4_f32", _i32, [_i32, _i32, _i32, _vp, _i64, _vp, _vp, _f32, _f32, _vp, _i64,
                               _vp, _vp, _vp, _vp, _sz, _vp])
+_sig("qgemm_a8w4_f32_actblock", _i32, [_i32, _i32, _i32, _vp, _i64, _vp, _vp, _f32, _f32, _vp,
+                                       _i64, _vp, _vp, _vp, _vp])
 _sig("pack_w4_g32_bf16_bytes", _sz, [_i32, _i32])
 _sig("pack_w4_g32_bf16", _i32, [_i32, _i32, _vp, _i64, _vp, _vp, _sz, _vp])
 _sig("qgemm_a8w4_f32_bf16s", _i32, [_i32, _i32, _i32, _vp, _i64, _vp, _vp, _f32, _f32, _vp,
@@ -206,6 +208,17 @@ def qgemm_a8w4_f32(x, packed_w, N, bias, clamp_min, clamp_max, y, q_out=None, sc
               float(clamp_min), float(clamp_max), _p(y), _ld(y), _p(q_out),
               _p(scale_out), _p(zp_out), _p(workspace),
               0 if workspace is None else workspace.numel(), _stream(stream)), fn.__name__)
+
+
+def qgemm_a8w4_f32_actblock(x, packed_w, N, bias, clamp_min, clamp_max, y, q_out=None,
+                            scale_out=None, zp_out=None, stream=None):
+    """A8W4 GEMV (M = 1) with the activations quantized per 32-wide K block;
+    scale_out / zp_out, when given, receive K/32 values."""
+    M, K = x.shape
+    _check(lib.qgemm_a8w4_f32_actblock(M, N, K, _p(x), _ld(x), _p(packed_w), _p(bias),
+                                       float(clamp_min), float(clamp_max), _p(y), _ld(y),
+                                       _p(q_out), _p(scale_out), _p(zp_out), _stream(stream)),
+           "qgemm_a8w4_f32_actblock")
 
 
 def qgemm_a8w4_f32_bf16s(x, packed_w, N, bias, clamp_min, clamp_max, y, **kw):

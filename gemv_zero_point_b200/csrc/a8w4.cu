@@ -451,7 +451,7 @@ __device__ __forceinline__ void prefetch_l2_interior(const void* p, int64_t byte
   }
 }
 
-template <int GPL, int W, int D, bool SBF>
+template <int GPL, int W, int D, bool SBF, bool ABLK>
 __global__ void __launch_bounds__(W * 32, 1) a8w4_gemv_stream_kernel(
     int N, int K, int max_rows, const float* __restrict__ x, const uint8_t* __restrict__ wq,
     const void* __restrict__ wscale, const float* __restrict__ bias, float clamp_lo,
@@ -460,6 +460,10 @@ __global__ void __launch_bounds__(W * 32, 1) a8w4_gemv_stream_kernel(
   extern __shared__ __align__(128) uint8_t sm[];
   __shared__ float red[2 * W];
   __shared__ float part_s[W * GPL];        // partial sums of the split rows
+  // ABLK (activations quantized per 32-wide K block): scale and zero-point of
+  // each block
+  __shared__ float blk_scale_s[ABLK ? GPL * 32 : 1];
+  __shared__ int blk_zp_s[ABLK ? GPL * 32 : 1];
   const int G = K >> 5;
   const int rowbytes = K >> 1;
   int8_t* qa_s = reinterpret_cast<int8_t*>(sm);      // [K] quantized x
@@ -547,39 +551,86 @@ __global__ void __launch_bounds__(W * 32, 1) a8w4_gemv_stream_kernel(
                            (int64_t)(n1 - r_rest) * G * sb);
     }
   }
-  mn = warp_min(mn);
-  mx = warp_max(mx);
-  if (lane == 0) {
-    red[warp] = mn;
-    red[W + warp] = mx;
-  }
-  gemv_bar<W>();
-  // every warp combines the W per-warp results (lanes past W repeat warp 0's)
-  mn = warp_min(red[lane < W ? lane : 0]);
-  mx = warp_max(red[W + (lane < W ? lane : 0)]);
-  const RowQuant rq = row_quant_params(mn, mx);
+  RowQuant rq;
+  if constexpr (!ABLK) {
+    mn = warp_min(mn);
+    mx = warp_max(mx);
+    if (lane == 0) {
+      red[warp] = mn;
+      red[W + warp] = mx;
+    }
+    gemv_bar<W>();
+    // every warp combines the W per-warp results (lanes past W repeat warp 0's)
+    mn = warp_min(red[lane < W ? lane : 0]);
+    mx = warp_max(red[W + (lane < W ? lane : 0)]);
+    rq = row_quant_params(mn, mx);
 #pragma unroll
-  for (int j = 0; j < XV; ++j) {
-    const int c = threadIdx.x + j * W * 32;
-    if (4 * c < K) {
-      const uint32_t b0 = (uint32_t)quant_one(xv[j].x, rq) & 0xFFu;
-      const uint32_t b1 = (uint32_t)quant_one(xv[j].y, rq) & 0xFFu;
-      const uint32_t b2 = (uint32_t)quant_one(xv[j].z, rq) & 0xFFu;
-      const uint32_t b3 = (uint32_t)quant_one(xv[j].w, rq) & 0xFFu;
-      reinterpret_cast<uint32_t*>(qa_s)[c] = b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
-      if (blockIdx.x == 0 && q_out) {
-        int8_t* qo = q_out + 4 * c;
-        qo[0] = (int8_t)b0; qo[1] = (int8_t)b1; qo[2] = (int8_t)b2; qo[3] = (int8_t)b3;
+    for (int j = 0; j < XV; ++j) {
+      const int c = threadIdx.x + j * W * 32;
+      if (4 * c < K) {
+        const uint32_t b0 = (uint32_t)quant_one(xv[j].x, rq) & 0xFFu;
+        const uint32_t b1 = (uint32_t)quant_one(xv[j].y, rq) & 0xFFu;
+        const uint32_t b2 = (uint32_t)quant_one(xv[j].z, rq) & 0xFFu;
+        const uint32_t b3 = (uint32_t)quant_one(xv[j].w, rq) & 0xFFu;
+        reinterpret_cast<uint32_t*>(qa_s)[c] = b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
+        if (blockIdx.x == 0 && q_out) {
+          int8_t* qo = q_out + 4 * c;
+          qo[0] = (int8_t)b0; qo[1] = (int8_t)b1; qo[2] = (int8_t)b2; qo[3] = (int8_t)b3;
+        }
       }
     }
-  }
-  if (blockIdx.x == 0 && threadIdx.x == 0) {
-    if (scale_out) scale_out[0] = rq.scale;
-    if (zp_out) zp_out[0] = rq.zp;
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+      if (scale_out) scale_out[0] = rq.scale;
+      if (zp_out) zp_out[0] = rq.zp;
+    }
+  } else {
+    // One 32-wide block = 8 consecutive float4 chunks, held by 8 consecutive
+    // lanes (K % 128 == 0: a warp's 32 chunks are all in range or all out).
+    // The per-row rule applies to each block: range including 0, f32 scale.
+#pragma unroll
+    for (int j = 0; j < XV; ++j) {
+      const int c = threadIdx.x + j * W * 32;
+      float bmn = fminf(0.0f, fminf(fminf(xv[j].x, xv[j].y), fminf(xv[j].z, xv[j].w)));
+      float bmx = fmaxf(0.0f, fmaxf(fmaxf(xv[j].x, xv[j].y), fmaxf(xv[j].z, xv[j].w)));
+#pragma unroll
+      for (int o = 1; o < 8; o <<= 1) {
+        bmn = fminf(bmn, __shfl_xor_sync(0xffffffffu, bmn, o));
+        bmx = fmaxf(bmx, __shfl_xor_sync(0xffffffffu, bmx, o));
+      }
+      if (4 * c < K) {
+        const RowQuant bq = row_quant_params(bmn, bmx);
+        const uint32_t b0 = (uint32_t)quant_one(xv[j].x, bq) & 0xFFu;
+        const uint32_t b1 = (uint32_t)quant_one(xv[j].y, bq) & 0xFFu;
+        const uint32_t b2 = (uint32_t)quant_one(xv[j].z, bq) & 0xFFu;
+        const uint32_t b3 = (uint32_t)quant_one(xv[j].w, bq) & 0xFFu;
+        reinterpret_cast<uint32_t*>(qa_s)[c] = b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
+        if (blockIdx.x == 0 && q_out) {
+          int8_t* qo = q_out + 4 * c;
+          qo[0] = (int8_t)b0; qo[1] = (int8_t)b1; qo[2] = (int8_t)b2; qo[3] = (int8_t)b3;
+        }
+        if ((lane & 7) == 0) {
+          blk_scale_s[c >> 3] = bq.scale;
+          blk_zp_s[c >> 3] = bq.zp;
+          if (blockIdx.x == 0 && scale_out) scale_out[c >> 3] = bq.scale;
+          if (blockIdx.x == 0 && zp_out) zp_out[c >> 3] = bq.zp;
+        }
+      }
+    }
+    rq.scale = 1.0f;  // the activation scales enter per group below
+    rq.inv = 1.0f;
+    rq.zp = 0;
   }
   gemv_bar<W>();
 
-  const int za = rq.zp;
+  // zero-point and scale of the activations of each of this lane's groups
+  int zag[GPL];
+  float sag[GPL];
+#pragma unroll
+  for (int i = 0; i < GPL; ++i) {
+    const int g = lane + 32 * i;
+    zag[i] = ABLK ? (g < G ? blk_zp_s[g] : 0) : rq.zp;
+    sag[i] = ABLK ? (g < G ? blk_scale_s[g] : 0.0f) : 1.0f;
+  }
   int a[GPL][8];
   int cseed[GPL];
 #pragma unroll
@@ -590,7 +641,7 @@ __global__ void __launch_bounds__(W * 32, 1) a8w4_gemv_stream_kernel(
       const int4 v0 = src[0], v1 = src[1];
       a[i][0] = v0.x; a[i][1] = v0.y; a[i][2] = v0.z; a[i][3] = v0.w;
       a[i][4] = v1.x; a[i][5] = v1.y; a[i][6] = v1.z; a[i][7] = v1.w;
-      cseed[i] = act_seed(a[i], za);
+      cseed[i] = act_seed(a[i], zag[i]);
     } else {
 #pragma unroll
       for (int j = 0; j < 8; ++j) a[i][j] = 0;
@@ -608,14 +659,17 @@ __global__ void __launch_bounds__(W * 32, 1) a8w4_gemv_stream_kernel(
 #pragma unroll
         for (int i = 0; i < GPL; ++i) {
           const int g = lane + 32 * i;
-          if (g < G) acc = fmaf(sbuf[u][i], (float)group_dot(wbuf[u][i], a[i], cseed[i], za), acc);
+          if (g < G) {
+            const float sc = ABLK ? __fmul_rn(sbuf[u][i], sag[i]) : sbuf[u][i];
+            acc = fmaf(sc, (float)group_dot(wbuf[u][i], a[i], cseed[i], zag[i]), acc);
+          }
         }
         load_row(u, j + D);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
         if (lane == 0) {
           const int r = n0 + warp + W * j;
-          float v = __fmul_rn(rq.scale, acc);
+          float v = ABLK ? acc : __fmul_rn(rq.scale, acc);
           if (bias) v = __fadd_rn(v, bias_s[r - n0]);
           y[r] = fminf(fmaxf(v, clamp_lo), clamp_hi);
         }
@@ -631,7 +685,9 @@ __global__ void __launch_bounds__(W * 32, 1) a8w4_gemv_stream_kernel(
       const int g = lane + 32 * slot;
 #pragma unroll
       for (int i = 0; i < GPL; ++i)  // static register indexing of a[slot]
-        if (i == slot && g < G) part = __fmul_rn(ssplit, (float)group_dot(wsplit, a[i], cseed[i], za));
+        if (i == slot && g < G)
+          part = __fmul_rn(ABLK ? __fmul_rn(ssplit, sag[i]) : ssplit,
+                           (float)group_dot(wsplit, a[i], cseed[i], zag[i]));
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
       if (lane == 0) part_s[k * GPL + slot] = part;
@@ -643,14 +699,14 @@ __global__ void __launch_bounds__(W * 32, 1) a8w4_gemv_stream_kernel(
 #pragma unroll
       for (int i = 1; i < GPL; ++i) acc += part_s[k * GPL + i];
       const int r = n0 + W * nrows + k;
-      float v = __fmul_rn(rq.scale, acc);
+      float v = ABLK ? acc : __fmul_rn(rq.scale, acc);
       if (bias) v = __fadd_rn(v, bias_s[r - n0]);
       y[r] = fminf(fmaxf(v, clamp_lo), clamp_hi);
     }
   }
 }
 
-template <int GPL, int W, int D, bool SBF>
+template <int GPL, int W, int D, bool SBF, bool ABLK = false>
 static int launch_stream(int N, int K, const float* x, const uint8_t* wq, const void* ws,
                          const float* bias, float lo, float hi, float* y, int8_t* q_out,
                          float* scale_out, int32_t* zp_out, cudaStream_t st) {
@@ -669,7 +725,7 @@ static int launch_stream(int N, int K, const float* x, const uint8_t* wq, const 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, a8w4_gemv_stream_kernel<GPL, W, D, SBF>, N, K, rows_per_cta,
+  cudaError_t e = cudaLaunchKernelEx(&cfg, a8w4_gemv_stream_kernel<GPL, W, D, SBF, ABLK>, N, K, rows_per_cta,
                                      x, wq, ws, bias, lo, hi, y, q_out, scale_out, zp_out,
                                      status_word());
   return e == cudaSuccess ? QG_OK : QG_ERR_CUDA;
@@ -715,15 +771,33 @@ int launch_a8w4_gemv(int N, int K, const float* x, const void* packed, const flo
                                                 scale_out, zp_out, st);
 }
 
+// A8W4 GEMV with the activations quantized per 32-wide K block (f32 group
+// scales): the streaming kernel only (K % 128 == 0, K <= 8192, x 16-byte
+// aligned), else QG_ERR_UNSUPPORTED.
+int launch_a8w4_gemv_actblock(int N, int K, const float* x, const void* packed, const float* bias,
+                              float lo, float hi, float* y, int8_t* q_out, float* scale_out,
+                              int32_t* zp_out, cudaStream_t st) {
+  if (K % 128 != 0 || K > 8192 || ((uintptr_t)x & 15) != 0) return QG_ERR_UNSUPPORTED;
+  const uint8_t* wq = (const uint8_t*)packed;
+  const void* ws = wq + (size_t)N * (K / 2);
+  const int G = K / 32;
+  int rc;
+  if (G <= 32) rc = launch_stream<1, 16, 3, false, true>(N, K, x, wq, ws, bias, lo, hi, y, q_out, scale_out, zp_out, st);
+  else if (G <= 64) rc = launch_stream<2, 16, 3, false, true>(N, K, x, wq, ws, bias, lo, hi, y, q_out, scale_out, zp_out, st);
+  else if (G <= 128) rc = launch_stream<4, 16, 2, false, true>(N, K, x, wq, ws, bias, lo, hi, y, q_out, scale_out, zp_out, st);
+  else rc = launch_stream<8, 8, 3, false, true>(N, K, x, wq, ws, bias, lo, hi, y, q_out, scale_out, zp_out, st);
+  return rc > 0 ? QG_ERR_UNSUPPORTED : rc;
+}
+
 template <bool SBF>
 static bool setup_a8w4_gemv_t() {
   // up to 64 KiB of activations in shared memory for the plain kernel
   const void* plain[] = {(const void*)a8w4_gemv_kernel<1, SBF>, (const void*)a8w4_gemv_kernel<2, SBF>,
                          (const void*)a8w4_gemv_kernel<4, SBF>};
-  const void* stream[] = {(const void*)a8w4_gemv_stream_kernel<1, 16, 3, SBF>,
-                          (const void*)a8w4_gemv_stream_kernel<2, 16, 3, SBF>,
-                          (const void*)a8w4_gemv_stream_kernel<4, 16, 2, SBF>,
-                          (const void*)a8w4_gemv_stream_kernel<8, 8, 3, SBF>};
+  const void* stream[] = {(const void*)a8w4_gemv_stream_kernel<1, 16, 3, SBF, false>,
+                          (const void*)a8w4_gemv_stream_kernel<2, 16, 3, SBF, false>,
+                          (const void*)a8w4_gemv_stream_kernel<4, 16, 2, SBF, false>,
+                          (const void*)a8w4_gemv_stream_kernel<8, 8, 3, SBF, false>};
   bool ok = true;
   for (const void* f : plain)
     ok &= cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, 65536) == cudaSuccess;
@@ -734,7 +808,15 @@ static bool setup_a8w4_gemv_t() {
 }
 
 int setup_a8w4_gemv() {
-  return (setup_a8w4_gemv_t<false>() && setup_a8w4_gemv_t<true>()) ? QG_OK : QG_ERR_CUDA;
+  bool ok = setup_a8w4_gemv_t<false>() && setup_a8w4_gemv_t<true>();
+  const void* blk[] = {(const void*)a8w4_gemv_stream_kernel<1, 16, 3, false, true>,
+                       (const void*)a8w4_gemv_stream_kernel<2, 16, 3, false, true>,
+                       (const void*)a8w4_gemv_stream_kernel<4, 16, 2, false, true>,
+                       (const void*)a8w4_gemv_stream_kernel<8, 8, 3, false, true>};
+  for (const void* f : blk)
+    ok &= cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmemMax) ==
+          cudaSuccess;
+  return ok ? QG_OK : QG_ERR_CUDA;
 }
 
 // ---------------------------------------------------------------------------

@@ -22,6 +22,9 @@ int launch_a8w4_gemv(int N, int K, const float* x, const void* packed, const flo
 int launch_a8w4_gemm_simt(int M, int N, int K, const int8_t* q, const float* sA,
                           const int32_t* zA, const void* packed, const float* bias, float lo,
                           float hi, float* y, int64_t ldy, bool scale_bf16, cudaStream_t st);
+int launch_a8w4_gemv_actblock(int N, int K, const float* x, const void* packed, const float* bias,
+                              float lo, float hi, float* y, int8_t* q_out, float* scale_out,
+                              int32_t* zp_out, cudaStream_t st);
 int setup_a8w4_gemv();
 int setup_a8w4_gemm_simt();
 int i8gemm_setup();
@@ -429,4 +432,25 @@ extern "C" int qgemm_a8w4_f32_bf16s(int M, int N, int K, const float* x, int64_t
                                     size_t workspace_bytes, void* stream) {
   return a8w4_linear(M, N, K, x, ldx, packed_w, bias, clamp_min, clamp_max, y, ldy, q_out,
                      scale_out, zp_out, workspace, workspace_bytes, true, stream);
+}
+
+extern "C" int qgemm_a8w4_f32_actblock(int M, int N, int K, const float* x, int64_t ldx,
+                                       const void* packed_w, const float* bias,
+                                       float clamp_min, float clamp_max, float* y,
+                                       int64_t ldy, int8_t* q_out, float* scale_out,
+                                       int32_t* zp_out, void* stream) {
+  if (M < 0 || N <= 0 || K <= 0 || ldx < K || ldy < N) return QG_ERR_INVALID_ARG;
+  if (K % 32) return QG_ERR_UNSUPPORTED;
+  if (!(clamp_min <= clamp_max)) return QG_ERR_INVALID_ARG;  // also rejects NaN
+  if (M == 0) return QG_OK;
+  if (M != 1) return QG_ERR_UNSUPPORTED;
+  if (!x || !packed_w || !y) return QG_ERR_INVALID_ARG;
+  if (!aligned(packed_w, 16)) return QG_ERR_MISALIGNED;
+  if (!aligned(x, 4) || !aligned(y, 4) || (bias && !aligned(bias, 4))) return QG_ERR_MISALIGNED;
+  if ((scale_out && !aligned(scale_out, 4)) || (zp_out && !aligned(zp_out, 4)))
+    return QG_ERR_MISALIGNED;
+  int rc = device_ready();
+  if (rc != QG_OK) return rc;
+  return launch_a8w4_gemv_actblock(N, K, x, packed_w, bias, clamp_min, clamp_max, y, q_out,
+                                   scale_out, zp_out, (cudaStream_t)stream);
 }

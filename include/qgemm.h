@@ -260,6 +260,29 @@ int qgemm_a8w4_f32_bf16s(int M, int N, int K, const float* x, int64_t ldx,
                          void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * A8W4 GEMV with the activations quantized per K block.  [MNN]
+ * ConvInt8TiledExecutor, dynamic-quant option 2: the input is quantized in as
+ * many K blocks as the weights have quant blocks, each block with its own
+ * scale and zero-point.  Here a block is one 32-wide weight group:
+ *   y[n] = clamp(sum_g sw[n,g] * sA[g] * I[n,g] + bias[n])
+ *   I[n,g] = sum_{k in g} (qA[k] - zA[g]) * w[n,k]      (exact integer)
+ * with sA[g], zA[g] from the per-row rule of quantize_rows_a8 applied to the
+ * 32 values of block g, and the group combination in float32.
+ *   M must be 1 (else QG_ERR_UNSUPPORTED); K % 128 == 0, K <= 8192 and x
+ *   16-byte aligned (else QG_ERR_UNSUPPORTED); packed_w from pack_w4_g32
+ *   (f32 group scales).  q_out [K] int8, scale_out [K/32] f32 and
+ *   zp_out [K/32] int32 are optional.  No workspace.  The same stream note
+ *   as qgemm_a8w4_f32 (M == 1) applies: packed_w may be read before the
+ *   previous M == 1 call on the stream has completed.
+ * ------------------------------------------------------------------------ */
+int qgemm_a8w4_f32_actblock(int M, int N, int K, const float* x, int64_t ldx,
+                            const void* packed_w, const float* bias,
+                            float clamp_min, float clamp_max,
+                            float* y, int64_t ldy,
+                            int8_t* q_out, float* scale_out, int32_t* zp_out,
+                            void* stream);
+
+/* ------------------------------------------------------------------------
  * qgemm_a8w4_f32 without a workspace.  The pages have no counterpart: this
  * entry point exists for callers that cannot allocate device memory for
  * scratch — a plugin inside a host framework that owns the allocator and

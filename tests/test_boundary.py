@@ -17,7 +17,7 @@ NULL = None
 def test_exports_every_declared_symbol():
     names = qg.exported_symbols()
     for expected in ["quantize_rows_a8", "pack_w4_g32", "qgemm_a8w4_f32", "qgemm_s8s8_requant",
-                     "pack_w4_g32_bf16", "qgemm_a8w4_f32_bf16s",
+                     "pack_w4_g32_bf16", "qgemm_a8w4_f32_bf16s", "qgemm_a8w4_f32_actblock",
                      "qconv2d_s8_im2col", "qgemm_pack_b_s8", "qgemm_s8s8_requant_packed",
                      "qg_requant_params", "qg_status_string", "qg_device_status"]:
         assert expected in names
@@ -137,3 +137,12 @@ def test_bf16_scale_entry_points_validate_like_f32_ones():
     assert f(1, 8, 48, FAKE, 48, FAKE, NULL, -1.0, 1.0, FAKE, 8, NULL, NULL, NULL, NULL, 0, NULL) == -4
     assert f(1, 8, 64, FAKE, 64, FAKE, NULL, 1.0, -1.0, FAKE, 8, NULL, NULL, NULL, NULL, 0, NULL) == -1
     assert f(0, 8, 64, FAKE, 64, FAKE, NULL, -1.0, 1.0, FAKE, 8, NULL, NULL, NULL, NULL, 0, NULL) == 0
+
+
+def test_actblock_gemv_validation():
+    f = lib.qgemm_a8w4_f32_actblock
+    assert f(2, 8, 128, FAKE, 128, FAKE, NULL, -1.0, 1.0, FAKE, 8, NULL, NULL, NULL, NULL) == -4  # M != 1
+    assert f(1, 8, 48, FAKE, 48, FAKE, NULL, -1.0, 1.0, FAKE, 8, NULL, NULL, NULL, NULL) == -4    # K % 32
+    assert f(1, 8, 128, FAKE, 128, FAKE, NULL, 1.0, -1.0, FAKE, 8, NULL, NULL, NULL, NULL) == -1  # lo > hi
+    assert f(1, 8, 128, FAKE, 127, FAKE, NULL, -1.0, 1.0, FAKE, 8, NULL, NULL, NULL, NULL) == -1  # ldx < K
+    assert f(0, 8, 128, FAKE, 128, FAKE, NULL, -1.0, 1.0, FAKE, 8, NULL, NULL, NULL, NULL) == 0   # empty

@@ -218,3 +218,54 @@ def test_a8w4_bf16_scales_shapes(lib, M, N, K):
 
 def test_a8w4_bf16_scales_full_size_128x4096x4096(lib):
     _check_a8w4(lib, workloads.a8w4_gemm_128x4096x4096(), bf16=True)
+
+
+# ---------------------------------------------------------------------------
+# A8W4 GEMV with the activations quantized per 32-wide K block
+# ---------------------------------------------------------------------------
+def _check_actblock(lib, w):
+    N, K = w["N"], w["K"]
+    packed = lib.pack_w4_g32(_dev(w["qw"]), _dev(w["sw"]))
+    x = _dev(w["x"])[:, :K]
+    y = torch.full((1, N + 1), 7.0, dtype=torch.float32, device="cuda")
+    q = torch.empty((1, K), dtype=torch.int8, device="cuda")
+    s = torch.empty(K // 32, dtype=torch.float32, device="cuda")
+    z = torch.empty(K // 32, dtype=torch.int32, device="cuda")
+    bias = None if w["bias"] is None else _dev(w["bias"])
+    lib.qgemm_a8w4_f32_actblock(x, packed, N, bias, w["clamp_min"], w["clamp_max"], y[:, :N],
+                                q, s, z)
+    torch.cuda.synchronize()
+    y_ref, q_ref, s_ref, z_ref = oracle.qgemm_a8w4_f32_actblock(
+        w["x"][:, :K], w["qw"], w["sw"], w["bias"], w["clamp_min"], w["clamp_max"])
+    np.testing.assert_array_equal(q.cpu().numpy(), q_ref)
+    np.testing.assert_array_equal(s.cpu().numpy().view(np.int32), s_ref[0].view(np.int32))
+    np.testing.assert_array_equal(z.cpu().numpy(), z_ref[0])
+    y_np = y.cpu().numpy()
+    assert (y_np[:, N:] == 7.0).all()
+    assert_a8w4_close(y_np[:, :N], y_ref)
+
+
+def test_gemv_actblock_full_size_1x14336x4096(lib):
+    _check_actblock(lib, workloads.a8w4_gemv_1x14336x4096())
+
+
+@pytest.mark.parametrize("N,K", [(1, 128), (300, 1024), (1000, 2048), (33, 8192), (5000, 4096)])
+def test_gemv_actblock_shapes(lib, N, K):
+    w = workloads.a8w4(1, N, K, seed=N * 3 + K, clamp=(-np.inf, np.inf), ldx=K + 3)
+    # blocks of very different magnitudes and a zero block
+    scale = np.float32(10.0) ** np.random.default_rng(N).integers(-3, 3, K // 32)
+    w["x"][:, :K] *= np.repeat(scale, 32)[None, :]
+    w["x"][:, 32:64] = 0.0
+    _check_actblock(lib, w)
+
+
+def test_gemv_actblock_rejects_what_it_does_not_cover(lib):
+    w = workloads.a8w4(2, 64, 256, seed=1)
+    packed = lib.pack_w4_g32(_dev(w["qw"]), _dev(w["sw"]))
+    y = torch.empty((2, 64), dtype=torch.float32, device="cuda")
+    with pytest.raises(lib.QGError):                       # M != 1
+        lib.qgemm_a8w4_f32_actblock(_dev(w["x"])[:, :256], packed, 64, None, -1.0, 1.0, y)
+    w = workloads.a8w4(1, 64, 96, seed=2)
+    packed = lib.pack_w4_g32(_dev(w["qw"]), _dev(w["sw"]))
+    with pytest.raises(lib.QGError):                       # K % 128 != 0
+        lib.qgemm_a8w4_f32_actblock(_dev(w["x"])[:, :96], packed, 64, None, -1.0, 1.0, y[:1])
