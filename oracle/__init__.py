@@ -474,3 +474,49 @@ def qgemm_a8w4_f32_actblock(x, qw, sw, bias, clamp_min, clamp_max):
             comb = comb + np.asarray(bias, np.float64)
         y[m] = np.minimum(np.maximum(comb.astype(np.float32), lo), hi)
     return y, qA, sA, za
+
+
+# ---------------------------------------------------------------------------
+# O7: asymmetric int4 weights ([MNN] ConvInt8TiledExecutor, asymmetric quant
+# info: each (output channel, block) carries a zero and an alpha, and the
+# weight is alpha * code + zero).  READING R14: w_real[n,k] = sw[n,g]*w[n,k]
+# + zw[n,g] with the int4 code w in [-8,7] as in the symmetric packing and a
+# float32 zero zw per (row, 32-wide group).
+# ---------------------------------------------------------------------------
+def pack_w4_g32_asym_bytes(N, K):
+    return N * (K // 2) + 2 * N * (K // GROUP) * 4
+
+
+def pack_w4_g32_asym(qw, sw, zw):
+    """pack_w4_g32's nibbles and f32 scales, then the f32 zeros zw[N][K/32]."""
+    packed = pack_w4_g32(qw, sw)
+    z_bytes = np.ascontiguousarray(np.asarray(zw, dtype=np.float32)).view(np.uint8).reshape(-1)
+    return np.concatenate([packed, z_bytes])
+
+
+def qgemm_a8w4_f32_asym(x, qw, sw, zw, bias, clamp_min, clamp_max):
+    """y[m,n] = clamp(f32( sum_g sA[m]*(sw[n,g]*I[m,n,g] + zw[n,g]*S[m,g]) + bias[n] ))
+    with I as in O4 and S[m,g] = sum_{k in g} (qA[m,k]-za[m]) (exact int):
+    the dequantized activations times (sw*w + zw), grouped.  The combination
+    is in float64.  Returns (y float32 [M,N], qA, sA, za) as O4."""
+    qA, sA, za = quantize_rows_a8(x)
+    qw = np.asarray(qw, dtype=np.int64)
+    N, K = qw.shape
+    G = K // GROUP
+    M = qA.shape[0]
+    swd = np.asarray(sw, dtype=np.float64)
+    zwd = np.asarray(zw, dtype=np.float64)
+    wg = qw.reshape(N, G, GROUP)
+    y = np.empty((M, N), dtype=np.float32)
+    lo, hi = np.float32(clamp_min), np.float32(clamp_max)
+    for m in range(M):
+        a = (qA[m].astype(np.int64) - int(za[m])).reshape(G, GROUP)
+        I = np.einsum("gj,ngj->ng", a, wg)                       # exact
+        S = a.sum(axis=1)                                        # exact
+        sa = np.float64(sA[m])
+        comb = (swd * sa * I.astype(np.float64) + zwd * sa * S.astype(np.float64)[None, :]).sum(axis=1)
+        if bias is not None:
+            comb = comb + np.asarray(bias, np.float64)
+        y[m] = np.minimum(np.maximum(comb.astype(np.float32), lo), hi)
+    return y, qA, sA, za
+

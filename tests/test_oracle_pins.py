@@ -465,3 +465,41 @@ def test_p10_blockwise_brute_force_loops():
             tot += float(w["sw"][n, g]) * float(s[0, g]) * I
         tot += float(w["bias"][n])
         assert y[0, n] == np.float32(tot)
+
+
+# ---------------------------------------------------------------------------
+# P11: asymmetric int4 weights (reading R14: w_real = sw*w + zw per group)
+# ---------------------------------------------------------------------------
+def _asym_case(M, N, K, seed):
+    w = workloads.a8w4(M, N, K, seed=seed)
+    zw = (w["sw"] * np.random.default_rng(seed).uniform(-8, 8, w["sw"].shape)).astype(np.float32)
+    return w, zw
+
+
+def test_p11_zero_zeros_reduce_to_the_symmetric_method():
+    w, _ = _asym_case(3, 20, 128, 21)
+    zw = np.zeros_like(w["sw"])
+    ya = oracle.qgemm_a8w4_f32_asym(w["x"], w["qw"], w["sw"], zw, w["bias"], -6.0, 6.0)[0]
+    ys = oracle.qgemm_a8w4_f32(w["x"], w["qw"], w["sw"], w["bias"], -6.0, 6.0)[0]
+    np.testing.assert_array_equal(ya, ys)
+
+
+def test_p11_equals_dense_float_product_of_dequantized_operands():
+    # a different computation: dequantize both operands, one float64 matmul
+    w, zw = _asym_case(4, 30, 256, 22)
+    K = 256
+    y = oracle.qgemm_a8w4_f32_asym(w["x"][:, :K], w["qw"], w["sw"], zw, w["bias"], -1e30, 1e30)[0]
+    qA, sA, za = oracle.quantize_rows_a8(w["x"][:, :K])
+    xa = oracle.dequantize_rows(qA, sA, za)                                   # [M][K]
+    wr = (np.repeat(w["sw"].astype(np.float64), 32, axis=1) * w["qw"].astype(np.float64)
+          + np.repeat(zw.astype(np.float64), 32, axis=1))                     # [N][K]
+    ref = xa @ wr.T + w["bias"].astype(np.float64)
+    np.testing.assert_allclose(y.astype(np.float64), ref, rtol=1e-6, atol=1e-6)
+
+
+def test_p11_pack_layout():
+    w, zw = _asym_case(1, 6, 64, 23)
+    p = oracle.pack_w4_g32_asym(w["qw"], w["sw"], zw)
+    assert p.size == oracle.pack_w4_g32_asym_bytes(6, 64) == 6 * 32 + 2 * 6 * 2 * 4
+    np.testing.assert_array_equal(p[:6 * 32 + 6 * 2 * 4], oracle.pack_w4_g32(w["qw"], w["sw"]))
+    np.testing.assert_array_equal(p[6 * 32 + 6 * 2 * 4:].view(np.float32).reshape(6, 2), zw)
