@@ -24,7 +24,8 @@ each, 295 MB in all).
                   [--workload headline|<one workload name below>] [--no-cpu-baseline]
 Workloads: int8_gemm_130x70x129, int8_conv_56x56x64_3x3, a8w4_gemv_1x14336x4096,
 a8w4_gemv_bf16s_1x14336x4096 (bf16 group scales), a8w4_gemv_actblock_1x14336x4096
-(activations quantized per 32-wide K block), a8w4_gemm_128x4096x4096,
+(activations quantized per 32-wide K block), a8w4_gemv_asym_1x14336x4096
+(asymmetric int4 weights), a8w4_gemm_128x4096x4096,
 int8_gemm_8192x8192x8200.
 Under torchrun each rank runs the same work on its own GPU (replicas: the
 path has no exchange step), and value sums all ranks' work.
@@ -265,18 +266,24 @@ class GemmCase:
 
 
 class A8W4Case:
-    def __init__(self, qg, torch, w, sets, bf16_scales=False, actblock=False):
+    def __init__(self, qg, torch, w, sets, bf16_scales=False, actblock=False, asym=False):
         self.M, self.N, self.K = w["M"], w["N"], w["K"]
         self.qg, self.torch = qg, torch
         self.bf16 = bf16_scales
         self.actblock = actblock  # activations quantized per 32-wide K block (M = 1)
+        self.asym = asym          # asymmetric int4 weights: an f32 zero per group (M = 1)
         qw = dev(w["qw"], torch)
         sw = dev(w["sw"], torch)
         self.packed = []
         for s in range(sets):
             # distinct weight sets: rotate the int4 codes along K (still in [-8,7])
             src = qw if s == 0 else torch.roll(qw, shifts=32 * s, dims=1)
-            self.packed.append(qg.pack_w4_g32(src, sw, bf16_scales=bf16_scales))
+            if asym:
+                zw = sw * torch.empty_like(sw).uniform_(-8.0, 8.0, generator=torch.Generator(
+                    device=sw.device).manual_seed(77 + s))
+                self.packed.append(qg.pack_w4_g32_asym(src, sw, zw))
+            else:
+                self.packed.append(qg.pack_w4_g32(src, sw, bf16_scales=bf16_scales))
         del qw
         self.x = dev(w["x"], torch)
         self.bias = None if w["bias"] is None else dev(w["bias"], torch)
@@ -290,6 +297,10 @@ class A8W4Case:
         self.d2h_host = torch.empty((self.M, self.N), dtype=torch.float32).pin_memory()
 
     def run(self, i, stream=None):
+        if self.asym:
+            self.qg.qgemm_a8w4_f32_asym(self.x, self.packed[i % len(self.packed)], self.N,
+                                        self.bias, self.lo, self.hi, self.y, stream=stream)
+            return
         if self.actblock:
             self.qg.qgemm_a8w4_f32_actblock(self.x, self.packed[i % len(self.packed)], self.N,
                                             self.bias, self.lo, self.hi, self.y, stream=stream)
@@ -303,7 +314,10 @@ class A8W4Case:
 
     def run_e2e(self, i):
         self.e2e_x.copy_(self.h2d_host, non_blocking=True)
-        if self.actblock:
+        if self.asym:
+            self.qg.qgemm_a8w4_f32_asym(self.e2e_x, self.packed[0], self.N, self.bias, self.lo,
+                                        self.hi, self.y)
+        elif self.actblock:
             self.qg.qgemm_a8w4_f32_actblock(self.e2e_x, self.packed[0], self.N, self.bias,
                                             self.lo, self.hi, self.y)
         else:
@@ -315,7 +329,8 @@ class A8W4Case:
         return a8w4_ops(self.M, self.N, self.K)
 
     def bytes(self):
-        return a8w4_bytes(self.M, self.N, self.K, 2 if self.bf16 else 4)
+        zeros = self.N * (self.K // 32) * 4 if self.asym else 0
+        return a8w4_bytes(self.M, self.N, self.K, 2 if self.bf16 else 4) + zeros
 
     def h2d(self):
         return self.h2d_host.numel() * 4
@@ -387,6 +402,9 @@ def build_cases(workload, qg, torch):
         return [("a8w4_gemv_1x14336x4096", A8W4Case(qg, torch, W.a8w4_gemv_1x14336x4096(), 8), "hbm")]
     if workload == "a8w4_gemm_128x4096x4096":
         return [("a8w4_gemm_128x4096x4096", A8W4Case(qg, torch, W.a8w4_gemm_128x4096x4096(), 16), "hbm")]
+    if workload == "a8w4_gemv_asym_1x14336x4096":   # asymmetric int4 weights (44 MB per set)
+        return [("a8w4_gemv_asym_1x14336x4096",
+                 A8W4Case(qg, torch, W.a8w4_gemv_1x14336x4096(), 7, asym=True), "hbm")]
     if workload == "a8w4_gemv_actblock_1x14336x4096":   # activations quantized per K block
         return [("a8w4_gemv_actblock_1x14336x4096",
                  A8W4Case(qg, torch, W.a8w4_gemv_1x14336x4096(), 8, actblock=True), "hbm")]
@@ -409,6 +427,7 @@ KERNEL_SOURCES = {
     "a8w4_gemm_128x4096x4096": "a8w4_tc.cu",
     "a8w4_gemv_bf16s_1x14336x4096": "a8w4.cu",
     "a8w4_gemv_actblock_1x14336x4096": "a8w4.cu",
+    "a8w4_gemv_asym_1x14336x4096": "a8w4.cu",
 }
 
 
@@ -459,6 +478,15 @@ def oracle_sample(workload, budget_s=12.0, rows_gemm=None, small=False):
         dt = time.perf_counter() - t
         ops += gemm_ops(rows, cols, w["K"]); spent += dt
         parts.append(f"int8 GEMM {rows} row(s) x {cols} cols of 8192x8192x8200")
+    if workload == "a8w4_gemv_asym_1x14336x4096":
+        w = W.a8w4_gemv_1x14336x4096()
+        n = 512 if small else w["N"]
+        zw = (w["sw"][:n] * np.random.default_rng(77).uniform(-8, 8, w["sw"][:n].shape)).astype(np.float32)
+        t = time.perf_counter()
+        oracle.qgemm_a8w4_f32_asym(w["x"], w["qw"][:n], w["sw"][:n], zw, w["bias"][:n], -6.0, 6.0)
+        dt = time.perf_counter() - t
+        ops += a8w4_ops(1, n, w["K"]); spent += dt
+        parts.append(f"A8W4 GEMV (asymmetric weights) {n} of 14336 rows")
     if workload in ("headline", "a8w4_gemv_1x14336x4096", "a8w4_gemv_bf16s_1x14336x4096",
                     "a8w4_gemv_actblock_1x14336x4096"):
         w = W.a8w4_gemv_1x14336x4096()
@@ -538,7 +566,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="headline",
-                    choices=["headline", "int8_gemm_130x70x129", "int8_conv_56x56x64_3x3", "a8w4_gemv_1x14336x4096", "a8w4_gemv_bf16s_1x14336x4096", "a8w4_gemv_actblock_1x14336x4096", "a8w4_gemm_128x4096x4096", "int8_gemm_8192x8192x8200"])
+                    choices=["headline", "int8_gemm_130x70x129", "int8_conv_56x56x64_3x3", "a8w4_gemv_1x14336x4096", "a8w4_gemv_bf16s_1x14336x4096", "a8w4_gemv_actblock_1x14336x4096", "a8w4_gemv_asym_1x14336x4096", "a8w4_gemm_128x4096x4096", "int8_gemm_8192x8192x8200"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=10)
     args = ap.parse_args()

@@ -90,6 +90,10 @@ _sig("qgemm_a8w4_f32", _i32, [_i32, _i32, _i32, _vp, _i64, _vp, _vp, _f32, _f32,
                               _vp, _vp, _vp, _vp, _sz, _vp])
 _sig("qgemm_a8w4_f32_actblock", _i32, [_i32, _i32, _i32, _vp, _i64, _vp, _vp, _f32, _f32, _vp,
                                        _i64, _vp, _vp, _vp, _vp])
+_sig("pack_w4_g32_asym_bytes", _sz, [_i32, _i32])
+_sig("pack_w4_g32_asym", _i32, [_i32, _i32, _vp, _i64, _vp, _vp, _vp, _sz, _vp])
+_sig("qgemm_a8w4_f32_asym", _i32, [_i32, _i32, _i32, _vp, _i64, _vp, _vp, _f32, _f32, _vp,
+                                   _i64, _vp, _vp, _vp, _vp])
 _sig("pack_w4_g32_bf16_bytes", _sz, [_i32, _i32])
 _sig("pack_w4_g32_bf16", _i32, [_i32, _i32, _vp, _i64, _vp, _vp, _sz, _vp])
 _sig("qgemm_a8w4_f32_bf16s", _i32, [_i32, _i32, _i32, _vp, _i64, _vp, _vp, _f32, _f32, _vp,
@@ -219,6 +223,26 @@ def qgemm_a8w4_f32_actblock(x, packed_w, N, bias, clamp_min, clamp_max, y, q_out
                                        float(clamp_min), float(clamp_max), _p(y), _ld(y),
                                        _p(q_out), _p(scale_out), _p(zp_out), _stream(stream)),
            "qgemm_a8w4_f32_actblock")
+
+
+def pack_w4_g32_asym(w, group_scales, group_zeros, packed=None, stream=None):
+    """Pack int4 weights with f32 group scales and f32 group zeros."""
+    N, K = w.shape
+    if packed is None:
+        packed = _empty_bytes(lib.pack_w4_g32_asym_bytes(N, K), w.device)
+    _check(lib.pack_w4_g32_asym(N, K, _p(w), _ld(w), _p(group_scales), _p(group_zeros),
+                                _p(packed), packed.numel(), _stream(stream)), "pack_w4_g32_asym")
+    return packed
+
+
+def qgemm_a8w4_f32_asym(x, packed_w, N, bias, clamp_min, clamp_max, y, q_out=None,
+                        scale_out=None, zp_out=None, stream=None):
+    """A8W4 GEMV (M = 1) with asymmetric int4 weights (pack_w4_g32_asym)."""
+    M, K = x.shape
+    _check(lib.qgemm_a8w4_f32_asym(M, N, K, _p(x), _ld(x), _p(packed_w), _p(bias),
+                                   float(clamp_min), float(clamp_max), _p(y), _ld(y),
+                                   _p(q_out), _p(scale_out), _p(zp_out), _stream(stream)),
+           "qgemm_a8w4_f32_asym")
 
 
 def qgemm_a8w4_f32_bf16s(x, packed_w, N, bias, clamp_min, clamp_max, y, **kw):

@@ -451,10 +451,11 @@ __device__ __forceinline__ void prefetch_l2_interior(const void* p, int64_t byte
   }
 }
 
-template <int GPL, int W, int D, bool SBF, bool ABLK>
+template <int GPL, int W, int D, bool SBF, bool ABLK, bool WZP>
 __global__ void __launch_bounds__(W * 32, 1) a8w4_gemv_stream_kernel(
     int N, int K, int max_rows, const float* __restrict__ x, const uint8_t* __restrict__ wq,
-    const void* __restrict__ wscale, const float* __restrict__ bias, float clamp_lo,
+    const void* __restrict__ wscale, const float* __restrict__ wzero,
+    const float* __restrict__ bias, float clamp_lo,
     float clamp_hi, float* __restrict__ y, int8_t* __restrict__ q_out,
     float* __restrict__ scale_out, int32_t* __restrict__ zp_out, int* status) {
   extern __shared__ __align__(128) uint8_t sm[];
@@ -462,6 +463,7 @@ __global__ void __launch_bounds__(W * 32, 1) a8w4_gemv_stream_kernel(
   __shared__ float part_s[W * GPL];        // partial sums of the split rows
   // ABLK (activations quantized per 32-wide K block): scale and zero-point of
   // each block
+  static_assert(!(ABLK && WZP), "weight zeros are taken with per-row activation scales");
   __shared__ float blk_scale_s[ABLK ? GPL * 32 : 1];
   __shared__ int blk_zp_s[ABLK ? GPL * 32 : 1];
   const int G = K >> 5;
@@ -479,6 +481,7 @@ __global__ void __launch_bounds__(W * 32, 1) a8w4_gemv_stream_kernel(
 
   uint4 wbuf[D][GPL];
   float sbuf[D][GPL];
+  float zbuf[WZP ? D : 1][GPL];  // WZP: f32 weight zero of each group
   // loads of this warp's row j into buffer u (nothing past the last row)
   const uint32_t ssel = (lane & 1) ? 0x3244u : 0x1044u;  // bf16 half of the scale word
   auto load_row = [&](int u, int j) {
@@ -490,6 +493,7 @@ __global__ void __launch_bounds__(W * 32, 1) a8w4_gemv_stream_kernel(
         if (g < G) {
           wbuf[u][i] = ld_stream_u4(wq + (int64_t)r * rowbytes + 16 * g);
           sbuf[u][i] = ld_row_scale<SBF>(wscale, r, G, lane, i, ssel);
+          if constexpr (WZP) zbuf[u][i] = ld_stream_f32(wzero + (int64_t)r * G + g);
         }
       }
     }
@@ -503,13 +507,14 @@ __global__ void __launch_bounds__(W * 32, 1) a8w4_gemv_stream_kernel(
   for (int u = 0; u < D; ++u) load_row(u, u);
   // the first split row this warp takes part in
   uint4 wsplit = make_uint4(0, 0, 0, 0);
-  float ssplit = 0.0f;
+  float ssplit = 0.0f, zsplit = 0.0f;
   auto load_split = [&](int k) {
     const int r = n0 + W * nrows + k;
     const int g = lane + 32 * slot;
     if (g < G) {
       wsplit = ld_stream_u4(wq + (int64_t)r * rowbytes + 16 * g);
       ssplit = ld_row_scale<SBF>(wscale, r, G, lane, slot, ssel);
+      if constexpr (WZP) zsplit = ld_stream_f32(wzero + (int64_t)r * G + g);
     }
   };
   if (warp / GPL < nleft) load_split(warp / GPL);
@@ -549,6 +554,7 @@ __global__ void __launch_bounds__(W * 32, 1) a8w4_gemv_stream_kernel(
       constexpr int64_t sb = SBF ? 2 : 4;  // bytes per scale
       prefetch_l2_interior((const uint8_t*)wscale + (int64_t)r_rest * G * sb,
                            (int64_t)(n1 - r_rest) * G * sb);
+      if (WZP) prefetch_l2_interior(wzero + (int64_t)r_rest * G, (int64_t)(n1 - r_rest) * G * 4);
     }
   }
   RowQuant rq;
@@ -633,6 +639,9 @@ __global__ void __launch_bounds__(W * 32, 1) a8w4_gemv_stream_kernel(
   }
   int a[GPL][8];
   int cseed[GPL];
+  float asum[GPL];  // WZP: the group sums of the centred activation codes
+#pragma unroll
+  for (int i = 0; i < GPL; ++i) asum[i] = 0.0f;
 #pragma unroll
   for (int i = 0; i < GPL; ++i) {
     const int g = lane + 32 * i;
@@ -642,6 +651,12 @@ __global__ void __launch_bounds__(W * 32, 1) a8w4_gemv_stream_kernel(
       a[i][0] = v0.x; a[i][1] = v0.y; a[i][2] = v0.z; a[i][3] = v0.w;
       a[i][4] = v1.x; a[i][5] = v1.y; a[i][6] = v1.z; a[i][7] = v1.w;
       cseed[i] = act_seed(a[i], zag[i]);
+      if constexpr (WZP) {  // S_g = sum_k (qA[k] - zA), exact
+        int sraw = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) sraw = __dp4a(a[i][j], 0x01010101, sraw);
+        asum[i] = (float)(sraw - 32 * zag[i]);
+      }
     } else {
 #pragma unroll
       for (int j = 0; j < 8; ++j) a[i][j] = 0;
@@ -662,6 +677,7 @@ __global__ void __launch_bounds__(W * 32, 1) a8w4_gemv_stream_kernel(
           if (g < G) {
             const float sc = ABLK ? __fmul_rn(sbuf[u][i], sag[i]) : sbuf[u][i];
             acc = fmaf(sc, (float)group_dot(wbuf[u][i], a[i], cseed[i], zag[i]), acc);
+            if constexpr (WZP) acc = fmaf(zbuf[u][i], asum[i], acc);
           }
         }
         load_row(u, j + D);
@@ -686,8 +702,11 @@ __global__ void __launch_bounds__(W * 32, 1) a8w4_gemv_stream_kernel(
 #pragma unroll
       for (int i = 0; i < GPL; ++i)  // static register indexing of a[slot]
         if (i == slot && g < G)
+        {
           part = __fmul_rn(ABLK ? __fmul_rn(ssplit, sag[i]) : ssplit,
                            (float)group_dot(wsplit, a[i], cseed[i], zag[i]));
+          if constexpr (WZP) part = fmaf(zsplit, asum[i], part);
+        }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
       if (lane == 0) part_s[k * GPL + slot] = part;
@@ -706,8 +725,8 @@ __global__ void __launch_bounds__(W * 32, 1) a8w4_gemv_stream_kernel(
   }
 }
 
-template <int GPL, int W, int D, bool SBF, bool ABLK = false>
-static int launch_stream(int N, int K, const float* x, const uint8_t* wq, const void* ws,
+template <int GPL, int W, int D, bool SBF, bool ABLK = false, bool WZP = false>
+static int launch_stream(int N, int K, const float* x, const uint8_t* wq, const void* ws, const float* wz,
                          const float* bias, float lo, float hi, float* y, int8_t* q_out,
                          float* scale_out, int32_t* zp_out, cudaStream_t st) {
   int grid = num_sms();
@@ -725,8 +744,8 @@ static int launch_stream(int N, int K, const float* x, const uint8_t* wq, const 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, a8w4_gemv_stream_kernel<GPL, W, D, SBF, ABLK>, N, K, rows_per_cta,
-                                     x, wq, ws, bias, lo, hi, y, q_out, scale_out, zp_out,
+  cudaError_t e = cudaLaunchKernelEx(&cfg, a8w4_gemv_stream_kernel<GPL, W, D, SBF, ABLK, WZP>, N, K, rows_per_cta,
+                                     x, wq, ws, wz, bias, lo, hi, y, q_out, scale_out, zp_out,
                                      status_word());
   return e == cudaSuccess ? QG_OK : QG_ERR_CUDA;
 }
@@ -742,10 +761,10 @@ static int launch_a8w4_gemv_t(int N, int K, const float* x, const void* packed,
   if (grid > N) grid = N;
   if (K % 128 == 0 && K <= 8192 && ((uintptr_t)x & 15) == 0) {
     int rc;
-    if (G <= 32) rc = launch_stream<1, 16, 3, SBF>(N, K, x, wq, ws, bias, lo, hi, y, q_out, scale_out, zp_out, st);
-    else if (G <= 64) rc = launch_stream<2, 16, 3, SBF>(N, K, x, wq, ws, bias, lo, hi, y, q_out, scale_out, zp_out, st);
-    else if (G <= 128) rc = launch_stream<4, 16, 2, SBF>(N, K, x, wq, ws, bias, lo, hi, y, q_out, scale_out, zp_out, st);
-    else rc = launch_stream<8, 8, 3, SBF>(N, K, x, wq, ws, bias, lo, hi, y, q_out, scale_out, zp_out, st);
+    if (G <= 32) rc = launch_stream<1, 16, 3, SBF>(N, K, x, wq, ws, nullptr, bias, lo, hi, y, q_out, scale_out, zp_out, st);
+    else if (G <= 64) rc = launch_stream<2, 16, 3, SBF>(N, K, x, wq, ws, nullptr, bias, lo, hi, y, q_out, scale_out, zp_out, st);
+    else if (G <= 128) rc = launch_stream<4, 16, 2, SBF>(N, K, x, wq, ws, nullptr, bias, lo, hi, y, q_out, scale_out, zp_out, st);
+    else rc = launch_stream<8, 8, 3, SBF>(N, K, x, wq, ws, nullptr, bias, lo, hi, y, q_out, scale_out, zp_out, st);
     if (rc <= 0) return rc;
   }
   const size_t smem = (size_t)K;
@@ -782,10 +801,29 @@ int launch_a8w4_gemv_actblock(int N, int K, const float* x, const void* packed, 
   const void* ws = wq + (size_t)N * (K / 2);
   const int G = K / 32;
   int rc;
-  if (G <= 32) rc = launch_stream<1, 16, 3, false, true>(N, K, x, wq, ws, bias, lo, hi, y, q_out, scale_out, zp_out, st);
-  else if (G <= 64) rc = launch_stream<2, 16, 3, false, true>(N, K, x, wq, ws, bias, lo, hi, y, q_out, scale_out, zp_out, st);
-  else if (G <= 128) rc = launch_stream<4, 16, 2, false, true>(N, K, x, wq, ws, bias, lo, hi, y, q_out, scale_out, zp_out, st);
-  else rc = launch_stream<8, 8, 3, false, true>(N, K, x, wq, ws, bias, lo, hi, y, q_out, scale_out, zp_out, st);
+  if (G <= 32) rc = launch_stream<1, 16, 3, false, true>(N, K, x, wq, ws, nullptr, bias, lo, hi, y, q_out, scale_out, zp_out, st);
+  else if (G <= 64) rc = launch_stream<2, 16, 3, false, true>(N, K, x, wq, ws, nullptr, bias, lo, hi, y, q_out, scale_out, zp_out, st);
+  else if (G <= 128) rc = launch_stream<4, 16, 2, false, true>(N, K, x, wq, ws, nullptr, bias, lo, hi, y, q_out, scale_out, zp_out, st);
+  else rc = launch_stream<8, 8, 3, false, true>(N, K, x, wq, ws, nullptr, bias, lo, hi, y, q_out, scale_out, zp_out, st);
+  return rc > 0 ? QG_ERR_UNSUPPORTED : rc;
+}
+
+// A8W4 GEMV with asymmetric int4 weights (an f32 zero per 32-wide group
+// after the f32 scales): the streaming kernel only (K % 128 == 0, K <= 8192,
+// x 16-byte aligned), else QG_ERR_UNSUPPORTED.
+int launch_a8w4_gemv_asym(int N, int K, const float* x, const void* packed, const float* bias,
+                          float lo, float hi, float* y, int8_t* q_out, float* scale_out,
+                          int32_t* zp_out, cudaStream_t st) {
+  if (K % 128 != 0 || K > 8192 || ((uintptr_t)x & 15) != 0) return QG_ERR_UNSUPPORTED;
+  const uint8_t* wq = (const uint8_t*)packed;
+  const float* ws = (const float*)(wq + (size_t)N * (K / 2));
+  const float* wz = ws + (size_t)N * (K / 32);
+  const int G = K / 32;
+  int rc;
+  if (G <= 32) rc = launch_stream<1, 16, 3, false, false, true>(N, K, x, wq, ws, wz, bias, lo, hi, y, q_out, scale_out, zp_out, st);
+  else if (G <= 64) rc = launch_stream<2, 16, 3, false, false, true>(N, K, x, wq, ws, wz, bias, lo, hi, y, q_out, scale_out, zp_out, st);
+  else if (G <= 128) rc = launch_stream<4, 16, 2, false, false, true>(N, K, x, wq, ws, wz, bias, lo, hi, y, q_out, scale_out, zp_out, st);
+  else rc = launch_stream<8, 8, 3, false, false, true>(N, K, x, wq, ws, wz, bias, lo, hi, y, q_out, scale_out, zp_out, st);
   return rc > 0 ? QG_ERR_UNSUPPORTED : rc;
 }
 
@@ -794,10 +832,10 @@ static bool setup_a8w4_gemv_t() {
   // up to 64 KiB of activations in shared memory for the plain kernel
   const void* plain[] = {(const void*)a8w4_gemv_kernel<1, SBF>, (const void*)a8w4_gemv_kernel<2, SBF>,
                          (const void*)a8w4_gemv_kernel<4, SBF>};
-  const void* stream[] = {(const void*)a8w4_gemv_stream_kernel<1, 16, 3, SBF, false>,
-                          (const void*)a8w4_gemv_stream_kernel<2, 16, 3, SBF, false>,
-                          (const void*)a8w4_gemv_stream_kernel<4, 16, 2, SBF, false>,
-                          (const void*)a8w4_gemv_stream_kernel<8, 8, 3, SBF, false>};
+  const void* stream[] = {(const void*)a8w4_gemv_stream_kernel<1, 16, 3, SBF, false, false>,
+                          (const void*)a8w4_gemv_stream_kernel<2, 16, 3, SBF, false, false>,
+                          (const void*)a8w4_gemv_stream_kernel<4, 16, 2, SBF, false, false>,
+                          (const void*)a8w4_gemv_stream_kernel<8, 8, 3, SBF, false, false>};
   bool ok = true;
   for (const void* f : plain)
     ok &= cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, 65536) == cudaSuccess;
@@ -809,11 +847,18 @@ static bool setup_a8w4_gemv_t() {
 
 int setup_a8w4_gemv() {
   bool ok = setup_a8w4_gemv_t<false>() && setup_a8w4_gemv_t<true>();
-  const void* blk[] = {(const void*)a8w4_gemv_stream_kernel<1, 16, 3, false, true>,
-                       (const void*)a8w4_gemv_stream_kernel<2, 16, 3, false, true>,
-                       (const void*)a8w4_gemv_stream_kernel<4, 16, 2, false, true>,
-                       (const void*)a8w4_gemv_stream_kernel<8, 8, 3, false, true>};
+  const void* blk[] = {(const void*)a8w4_gemv_stream_kernel<1, 16, 3, false, true, false>,
+                       (const void*)a8w4_gemv_stream_kernel<2, 16, 3, false, true, false>,
+                       (const void*)a8w4_gemv_stream_kernel<4, 16, 2, false, true, false>,
+                       (const void*)a8w4_gemv_stream_kernel<8, 8, 3, false, true, false>};
   for (const void* f : blk)
+    ok &= cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmemMax) ==
+          cudaSuccess;
+  const void* asym[] = {(const void*)a8w4_gemv_stream_kernel<1, 16, 3, false, false, true>,
+                        (const void*)a8w4_gemv_stream_kernel<2, 16, 3, false, false, true>,
+                        (const void*)a8w4_gemv_stream_kernel<4, 16, 2, false, false, true>,
+                        (const void*)a8w4_gemv_stream_kernel<8, 8, 3, false, false, true>};
+  for (const void* f : asym)
     ok &= cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmemMax) ==
           cudaSuccess;
   return ok ? QG_OK : QG_ERR_CUDA;

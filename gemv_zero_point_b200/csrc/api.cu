@@ -25,6 +25,9 @@ int launch_a8w4_gemm_simt(int M, int N, int K, const int8_t* q, const float* sA,
 int launch_a8w4_gemv_actblock(int N, int K, const float* x, const void* packed, const float* bias,
                               float lo, float hi, float* y, int8_t* q_out, float* scale_out,
                               int32_t* zp_out, cudaStream_t st);
+int launch_a8w4_gemv_asym(int N, int K, const float* x, const void* packed, const float* bias,
+                          float lo, float hi, float* y, int8_t* q_out, float* scale_out,
+                          int32_t* zp_out, cudaStream_t st);
 int setup_a8w4_gemv();
 int setup_a8w4_gemm_simt();
 int i8gemm_setup();
@@ -453,4 +456,48 @@ extern "C" int qgemm_a8w4_f32_actblock(int M, int N, int K, const float* x, int6
   if (rc != QG_OK) return rc;
   return launch_a8w4_gemv_actblock(N, K, x, packed_w, bias, clamp_min, clamp_max, y, q_out,
                                    scale_out, zp_out, (cudaStream_t)stream);
+}
+
+extern "C" size_t pack_w4_g32_asym_bytes(int N, int K) {
+  if (N <= 0 || K <= 0 || K % 32) return 0;
+  return pack_w4_g32_bytes(N, K) + (size_t)N * (K / 32) * 4;
+}
+
+extern "C" int pack_w4_g32_asym(int N, int K, const int8_t* w, int64_t ldw,
+                                const float* group_scales, const float* group_zeros,
+                                void* packed, size_t packed_bytes, void* stream) {
+  if (N <= 0 || K <= 0 || ldw < K || !w || !group_scales || !group_zeros || !packed)
+    return QG_ERR_INVALID_ARG;
+  if (K % 32) return QG_ERR_UNSUPPORTED;
+  if (!aligned(packed, 16) || !aligned(group_scales, 4) || !aligned(group_zeros, 4))
+    return QG_ERR_MISALIGNED;
+  if (packed_bytes < pack_w4_g32_asym_bytes(N, K)) return QG_ERR_WORKSPACE;
+  int rc = pack_w4(N, K, w, ldw, group_scales, packed, packed_bytes, false, stream);
+  if (rc != QG_OK) return rc;
+  // the zeros follow the scales as given (f32, [N][K/32])
+  if (cudaMemcpyAsync((char*)packed + pack_w4_g32_bytes(N, K), group_zeros,
+                      (size_t)N * (K / 32) * 4, cudaMemcpyDeviceToDevice,
+                      (cudaStream_t)stream) != cudaSuccess)
+    return QG_ERR_CUDA;
+  return QG_OK;
+}
+
+extern "C" int qgemm_a8w4_f32_asym(int M, int N, int K, const float* x, int64_t ldx,
+                                   const void* packed_w, const float* bias, float clamp_min,
+                                   float clamp_max, float* y, int64_t ldy, int8_t* q_out,
+                                   float* scale_out, int32_t* zp_out, void* stream) {
+  if (M < 0 || N <= 0 || K <= 0 || ldx < K || ldy < N) return QG_ERR_INVALID_ARG;
+  if (K % 32) return QG_ERR_UNSUPPORTED;
+  if (!(clamp_min <= clamp_max)) return QG_ERR_INVALID_ARG;  // also rejects NaN
+  if (M == 0) return QG_OK;
+  if (M != 1) return QG_ERR_UNSUPPORTED;
+  if (!x || !packed_w || !y) return QG_ERR_INVALID_ARG;
+  if (!aligned(packed_w, 16)) return QG_ERR_MISALIGNED;
+  if (!aligned(x, 4) || !aligned(y, 4) || (bias && !aligned(bias, 4))) return QG_ERR_MISALIGNED;
+  if ((scale_out && !aligned(scale_out, 4)) || (zp_out && !aligned(zp_out, 4)))
+    return QG_ERR_MISALIGNED;
+  int rc = device_ready();
+  if (rc != QG_OK) return rc;
+  return launch_a8w4_gemv_asym(N, K, x, packed_w, bias, clamp_min, clamp_max, y, q_out,
+                               scale_out, zp_out, (cudaStream_t)stream);
 }

@@ -283,6 +283,32 @@ int qgemm_a8w4_f32_actblock(int M, int N, int K, const float* x, int64_t ldx,
                             void* stream);
 
 /* ------------------------------------------------------------------------
+ * A8W4 GEMV with asymmetric int4 weights.  [MNN] ConvInt8TiledExecutor,
+ * asymmetric quant info: every (output channel, block) carries a zero and an
+ * alpha, and a weight is alpha * code + zero.  Here:
+ *   w_real[n,k] = sw[n,g] * w[n,k] + zw[n,g]     (w in [-8,7], g = k/32)
+ *   y[n] = clamp(sA * sum_g (sw[n,g]*I[n,g] + zw[n,g]*S[g]) + bias[n])
+ *   I[n,g] = sum_{k in g} (qA[k] - zA) * w[n,k],  S[g] = sum_{k in g} (qA[k] - zA)
+ * (I and S exact integers, the combination in float32).
+ *   pack_w4_g32_asym: pack_w4_g32's layout followed by the f32 zeros
+ *   zw[N][K/32] (row-major, contiguous), copied as given; size from
+ *   pack_w4_g32_asym_bytes (0 when K % 32 != 0).  Checks as pack_w4_g32,
+ *   plus group_zeros non-NULL and 4-byte aligned.
+ *   qgemm_a8w4_f32_asym: M must be 1, K % 128 == 0, K <= 8192 and x 16-byte
+ *   aligned (else QG_ERR_UNSUPPORTED); arguments and outputs as
+ *   qgemm_a8w4_f32 for M == 1, no workspace, and the same stream note.
+ * ------------------------------------------------------------------------ */
+size_t pack_w4_g32_asym_bytes(int N, int K);
+int pack_w4_g32_asym(int N, int K, const int8_t* w, int64_t ldw, const float* group_scales,
+                     const float* group_zeros, void* packed, size_t packed_bytes, void* stream);
+int qgemm_a8w4_f32_asym(int M, int N, int K, const float* x, int64_t ldx,
+                        const void* packed_w, const float* bias,
+                        float clamp_min, float clamp_max,
+                        float* y, int64_t ldy,
+                        int8_t* q_out, float* scale_out, int32_t* zp_out,
+                        void* stream);
+
+/* ------------------------------------------------------------------------
  * qgemm_a8w4_f32 without a workspace.  The pages have no counterpart: this
  * entry point exists for callers that cannot allocate device memory for
  * scratch — a plugin inside a host framework that owns the allocator and

@@ -18,6 +18,7 @@ def test_exports_every_declared_symbol():
     names = qg.exported_symbols()
     for expected in ["quantize_rows_a8", "pack_w4_g32", "qgemm_a8w4_f32", "qgemm_s8s8_requant",
                      "pack_w4_g32_bf16", "qgemm_a8w4_f32_bf16s", "qgemm_a8w4_f32_actblock",
+                     "pack_w4_g32_asym", "qgemm_a8w4_f32_asym",
                      "qconv2d_s8_im2col", "qgemm_pack_b_s8", "qgemm_s8s8_requant_packed",
                      "qg_requant_params", "qg_status_string", "qg_device_status"]:
         assert expected in names
@@ -146,3 +147,17 @@ def test_actblock_gemv_validation():
     assert f(1, 8, 128, FAKE, 128, FAKE, NULL, 1.0, -1.0, FAKE, 8, NULL, NULL, NULL, NULL) == -1  # lo > hi
     assert f(1, 8, 128, FAKE, 127, FAKE, NULL, -1.0, 1.0, FAKE, 8, NULL, NULL, NULL, NULL) == -1  # ldx < K
     assert f(0, 8, 128, FAKE, 128, FAKE, NULL, -1.0, 1.0, FAKE, 8, NULL, NULL, NULL, NULL) == 0   # empty
+
+
+def test_asym_entry_points_validation():
+    assert lib.pack_w4_g32_asym_bytes(14336, 4096) == 14336 * 2048 + 2 * 14336 * 128 * 4
+    assert lib.pack_w4_g32_asym_bytes(10, 33) == 0
+    p = lib.pack_w4_g32_asym
+    assert p(4, 64, FAKE, 64, FAKE, NULL, FAKE, 1 << 20, NULL) == -1      # zeros missing
+    assert p(4, 48, FAKE, 48, FAKE, FAKE, FAKE, 1 << 20, NULL) == -4      # K % 32
+    assert p(4, 64, FAKE, 64, FAKE, ctypes.c_void_p(0x10002), FAKE, 1 << 20, NULL) == -2
+    assert p(4, 64, FAKE, 64, FAKE, FAKE, FAKE, 4 * 32 + 2 * 4 * 2 * 4 - 1, NULL) == -7
+    f = lib.qgemm_a8w4_f32_asym
+    assert f(2, 8, 128, FAKE, 128, FAKE, NULL, -1.0, 1.0, FAKE, 8, NULL, NULL, NULL, NULL) == -4
+    assert f(1, 8, 128, FAKE, 128, FAKE, NULL, 1.0, -1.0, FAKE, 8, NULL, NULL, NULL, NULL) == -1
+    assert f(0, 8, 128, FAKE, 128, FAKE, NULL, -1.0, 1.0, FAKE, 8, NULL, NULL, NULL, NULL) == 0

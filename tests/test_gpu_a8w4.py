@@ -269,3 +269,61 @@ def test_gemv_actblock_rejects_what_it_does_not_cover(lib):
     packed = lib.pack_w4_g32(_dev(w["qw"]), _dev(w["sw"]))
     with pytest.raises(lib.QGError):                       # K % 128 != 0
         lib.qgemm_a8w4_f32_actblock(_dev(w["x"])[:, :96], packed, 64, None, -1.0, 1.0, y[:1])
+
+
+# ---------------------------------------------------------------------------
+# A8W4 GEMV with asymmetric int4 weights (f32 zero per group)
+# ---------------------------------------------------------------------------
+def _asym_zeros(w, seed):
+    rng = np.random.default_rng(seed)
+    return (w["sw"] * rng.uniform(-8, 8, w["sw"].shape)).astype(np.float32)
+
+
+def _check_asym(lib, w, zw):
+    N, K = w["N"], w["K"]
+    packed = lib.pack_w4_g32_asym(_dev(w["qw"]), _dev(w["sw"]), _dev(zw))
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(packed.cpu().numpy(),
+                                  oracle.pack_w4_g32_asym(w["qw"], w["sw"], zw))
+    x = _dev(w["x"])[:, :K]
+    y = torch.full((1, N + 1), 7.0, dtype=torch.float32, device="cuda")
+    q = torch.empty((1, K), dtype=torch.int8, device="cuda")
+    s = torch.empty(1, dtype=torch.float32, device="cuda")
+    z = torch.empty(1, dtype=torch.int32, device="cuda")
+    bias = None if w["bias"] is None else _dev(w["bias"])
+    lib.qgemm_a8w4_f32_asym(x, packed, N, bias, w["clamp_min"], w["clamp_max"], y[:, :N], q, s, z)
+    torch.cuda.synchronize()
+    y_ref, q_ref, s_ref, z_ref = oracle.qgemm_a8w4_f32_asym(
+        w["x"][:, :K], w["qw"], w["sw"], zw, w["bias"], w["clamp_min"], w["clamp_max"])
+    np.testing.assert_array_equal(q.cpu().numpy(), q_ref)
+    np.testing.assert_array_equal(s.cpu().numpy().view(np.int32), s_ref.view(np.int32))
+    np.testing.assert_array_equal(z.cpu().numpy(), z_ref)
+    y_np = y.cpu().numpy()
+    assert (y_np[:, N:] == 7.0).all()
+    assert_a8w4_close(y_np[:, :N], y_ref)
+
+
+def test_gemv_asym_full_size_1x14336x4096(lib):
+    w = workloads.a8w4_gemv_1x14336x4096()
+    _check_asym(lib, w, _asym_zeros(w, 31))
+
+
+@pytest.mark.parametrize("N,K", [(1, 128), (300, 1024), (1000, 2048), (33, 8192), (5000, 4096)])
+def test_gemv_asym_shapes(lib, N, K):
+    w = workloads.a8w4(1, N, K, seed=N * 5 + K, clamp=(-np.inf, np.inf), ldx=K + 3)
+    _check_asym(lib, w, _asym_zeros(w, N + K))
+
+
+def test_gemv_asym_with_zero_zeros_matches_symmetric_entry(lib):
+    w = workloads.a8w4(1, 640, 4096, seed=32)
+    N, K = 640, 4096
+    zw = np.zeros_like(w["sw"])
+    pa = lib.pack_w4_g32_asym(_dev(w["qw"]), _dev(w["sw"]), _dev(zw))
+    ps = lib.pack_w4_g32(_dev(w["qw"]), _dev(w["sw"]))
+    x = _dev(w["x"])[:, :K]
+    ya = torch.empty((1, N), dtype=torch.float32, device="cuda")
+    ys = torch.empty((1, N), dtype=torch.float32, device="cuda")
+    lib.qgemm_a8w4_f32_asym(x, pa, N, _dev(w["bias"]), -6.0, 6.0, ya)
+    lib.qgemm_a8w4_f32(x, ps, N, _dev(w["bias"]), -6.0, 6.0, ys)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(ya.cpu().numpy(), ys.cpu().numpy())
