@@ -39,7 +39,7 @@ class QGError(RuntimeError):
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is not built; run `python -m gemv_zero_point_b200.build` "
+        f"{LIB_PATH} is not built; run `python gemv_zero_point_b200/build.py` "
         "(nvcc with sm_100a) first")
 
 lib = ctypes.CDLL(LIB_PATH)

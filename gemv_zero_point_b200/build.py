@@ -4,7 +4,9 @@ Each ``csrc/*.cu`` is compiled to an object under ``_build/`` (skipped when
 the object is newer than the sources and headers), then linked into
 ``gemv_zero_point_b200/libqgemm.so`` with the CUDA runtime linked statically,
 so the library loads without a GPU and without a CUDA runtime on the loader
-path.  Usage: ``python -m gemv_zero_point_b200.build [-v]``.
+path.  Usage: ``python gemv_zero_point_b200/build.py [-v] [--ptxas-info]`` (run
+as a script: ``-m`` would import the package first, and the package refuses
+to import until the library exists).
 """
 from __future__ import annotations
 
