@@ -21,10 +21,11 @@ Sources (web pages), cited by title and section:
          6 (四级验证, four-level verification).
   [MNN]  MNN source/backend/cpu/compute/ConvInt8TiledExecutor.cpp:
          initializeConvInt8QuantInfo, _computeReorderQuantInfo,
-         BatchAsyDynamicQuant, tileSplitFunction (QuanPostTreatParameters).
+         BatchAsyDynamicQuant, BatchSymDynamicQuant, the low-memory
+         float im2col path, tileSplitFunction (QuanPostTreatParameters).
   [KAI]  pytorch/ao PR #997 "Kleidi 4b blockwise gemv prototype".
 
-Readings where the pages are silent are named R1..R11 here and listed with
+Readings where the pages are silent are named R1..R16 here and listed with
 their justification in the design notes.
 
 Parity pins: every function below is pinned by tests in
@@ -520,3 +521,115 @@ def qgemm_a8w4_f32_asym(x, qw, sw, zw, bias, clamp_min, clamp_max):
         y[m] = np.minimum(np.maximum(comb.astype(np.float32), lo), hi)
     return y, qA, sA, za
 
+
+
+# ---------------------------------------------------------------------------
+# O8: dynamic per-row symmetric int8 activation quantization ([MNN]
+# ConvInt8TiledExecutor, BatchSymDynamicQuant: the absolute maximum of each
+# row gives a quantizing scale and a dequantizing scale, the codes are taken
+# with that scale and the zero-point is 0).
+# READING R15: amax = max_k |x[k]|; dequant scale = amax/127 and quant scale
+# = 127/amax, each one float32 division (both 1 when amax is 0);
+# q = clamp(rne(x * quant scale), -127, 127); zero-point 0.
+# ---------------------------------------------------------------------------
+def quantize_rows_a8_sym(x):
+    """Per row m of x[M][K] (float32):
+        amax = max_k |x[m,k]|   (0 for an empty or all-zero row)
+        dscale = amax / 127, qscale = 127 / amax   (both 1 if amax == 0)
+        q[k] = clamp(rne(x[k] * qscale), -127, 127)
+    every operation in float32 with one rounding each.
+    Returns q int8 [M][K], dscale float32 [M], zp int32 [M] (all zero).
+    """
+    x = np.asarray(x, dtype=np.float32)
+    M, K = x.shape
+    f32 = np.float32
+    q = np.empty((M, K), dtype=np.int8)
+    scale = np.empty(M, dtype=np.float32)
+    for m in range(M):
+        row = x[m]
+        amax = f32(np.abs(row).max()) if K else f32(0.0)
+        if amax == f32(0.0):
+            ds, qs = f32(1.0), f32(1.0)
+        else:
+            ds = f32(amax / f32(127.0))
+            qs = f32(f32(127.0) / amax)
+        r = np.rint((row * qs).astype(np.float32)).astype(np.int64)
+        q[m] = np.clip(r, -127, 127).astype(np.int8)
+        scale[m] = ds
+    return q, scale, np.zeros(M, dtype=np.int32)
+
+
+# ---------------------------------------------------------------------------
+# O9: convolution with a float input quantized on the fly ([MNN]
+# ConvInt8TiledExecutor, low-memory path: the float input of a tile of output
+# pixels is unrolled by im2col, each unrolled row is quantized dynamically,
+# asymmetric (BatchAsyDynamicQuant) or symmetric (BatchSymDynamicQuant), and
+# the int8 rows meet the int4 block-quantized weights; [QG] section 2: a pad
+# tap stands for the real value zero).
+# READING R16: x float32 NHWC [Nb][H][W][Cin]; int4 codes w[Cout][KH][KW][Cin]
+# flattened to K = KH*KW*Cin in (kh, kw, ci) order, one scale per 32
+# consecutive k of that order; the unrolled row of output pixel (n, oh, ow)
+# holds x[n, oh*sh+kh-ph, ow*sw+kw-pw, ci], 0.0 for a tap outside the image;
+# each unrolled row is quantized on its own (R5, or R15 when symmetric) and
+# y[n,oh,ow,:] is O4 on that row, output NHWC float32.
+# ---------------------------------------------------------------------------
+def im2col_f32(x, KH, KW, stride, pad):
+    """Unrolled float input: cols[(n*OH+oh)*OW+ow, (kh*KW+kw)*Cin+ci]."""
+    x = np.asarray(x, dtype=np.float32)
+    Nb, H, W, Cin = x.shape
+    sh, sw = stride
+    ph, pw = pad
+    OH, OW = conv_out_size(H, KH, sh, ph), conv_out_size(W, KW, sw, pw)
+    cols = np.zeros((Nb, OH, OW, KH, KW, Cin), dtype=np.float32)
+    for kh in range(KH):
+        for kw in range(KW):
+            for oh in range(OH):
+                ih = oh * sh + kh - ph
+                if ih < 0 or ih >= H:
+                    continue
+                for ow in range(OW):
+                    iw = ow * sw + kw - pw
+                    if iw < 0 or iw >= W:
+                        continue
+                    cols[:, oh, ow, kh, kw, :] = x[:, ih, iw, :]
+    return cols.reshape(Nb * OH * OW, KH * KW * Cin)
+
+
+def a8w4_from_codes(qA, sA, za, qw, sw, bias, clamp_min, clamp_max):
+    """O4's combination for activations already quantized:
+        y[m,n] = clamp(f32( sum_g sw[n,g]*sA[m]*I[m,n,g] + bias[n] ), lo, hi)
+        I[m,n,g] = sum_{k in group g} (qA[m,k]-za[m]) * qw[n,k]   (exact int)
+    with the combination over groups in float64."""
+    qw = np.asarray(qw, dtype=np.int64)
+    N, K = qw.shape
+    G = K // GROUP
+    M = qA.shape[0]
+    swd = np.asarray(sw, dtype=np.float64)
+    wg = qw.reshape(N, G, GROUP)
+    y = np.empty((M, N), dtype=np.float32)
+    lo, hi = np.float32(clamp_min), np.float32(clamp_max)
+    for m in range(M):
+        a = (qA[m].astype(np.int64) - int(za[m])).reshape(G, GROUP)
+        I = np.einsum("gj,ngj->ng", a, wg)                       # exact
+        comb = (swd * np.float64(sA[m]) * I.astype(np.float64)).sum(axis=1)
+        if bias is not None:
+            comb = comb + np.asarray(bias, np.float64)
+        y[m] = np.minimum(np.maximum(comb.astype(np.float32), lo), hi)
+    return y
+
+
+def qconv2d_f32_dyn_a8w4(x, qw, sw, stride, pad, bias, clamp_min, clamp_max,
+                         symmetric=False):
+    """Float-input convolution with dynamic int8 activations and int4 g32
+    weights (O9, R16).  qw int4 codes [Cout][KH][KW][Cin], sw [Cout][K/32].
+    Returns (y float32 [Nb][OH][OW][Cout], qA int8 [P][K], sA float32 [P],
+    za int32 [P]) with P = Nb*OH*OW unrolled rows."""
+    qw = np.asarray(qw)
+    Cout, KH, KW, Cin = qw.shape
+    Nb, H, W, _ = np.asarray(x).shape
+    OH, OW = conv_out_size(H, KH, stride[0], pad[0]), conv_out_size(W, KW, stride[1], pad[1])
+    cols = im2col_f32(x, KH, KW, stride, pad)
+    qA, sA, za = quantize_rows_a8_sym(cols) if symmetric else quantize_rows_a8(cols)
+    y = a8w4_from_codes(qA, sA, za, qw.reshape(Cout, KH * KW * Cin), sw, bias,
+                        clamp_min, clamp_max)
+    return y.reshape(Nb, OH, OW, Cout), qA, sA, za

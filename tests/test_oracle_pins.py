@@ -503,3 +503,159 @@ def test_p11_pack_layout():
     assert p.size == oracle.pack_w4_g32_asym_bytes(6, 64) == 6 * 32 + 2 * 6 * 2 * 4
     np.testing.assert_array_equal(p[:6 * 32 + 6 * 2 * 4], oracle.pack_w4_g32(w["qw"], w["sw"]))
     np.testing.assert_array_equal(p[6 * 32 + 6 * 2 * 4:].view(np.float32).reshape(6, 2), zw)
+
+
+# ---------------------------------------------------------------------------
+# P12: symmetric dynamic activation quantization (reading R15: amax/127,
+# codes in [-127, 127], zero-point 0)
+# ---------------------------------------------------------------------------
+def test_p12_symmetric_hand_derived_rows():
+    # amax 2: quant scale 63.5, so -1 -> -63.5 (tie, to even -64), 0.5 -> 31.75 -> 32
+    # amax 4: quant scale 31.75, so 1 -> 31.75 -> 32, 3 -> 95.25 -> 95
+    x = np.array([[2.0, -1.0, 0.5, 0.0], [-4.0, 1.0, 3.0, 0.0], [0.0, 0.0, 0.0, 0.0]],
+                 np.float32)
+    q, s, z = oracle.quantize_rows_a8_sym(x)
+    assert q.tolist() == [[127, -64, 32, 0], [-127, 32, 95, 0], [0, 0, 0, 0]]
+    assert s[0] == np.float32(2.0) / np.float32(127.0)
+    assert s[1] == np.float32(4.0) / np.float32(127.0)
+    assert s[2] == 1.0
+    assert z.tolist() == [0, 0, 0]
+
+
+def test_p12_symmetric_invariants():
+    rng = np.random.default_rng(12)
+    x = (rng.standard_normal((16, 96)) * rng.uniform(0.01, 50, (16, 1))).astype(np.float32)
+    q, s, z = oracle.quantize_rows_a8_sym(x)
+    assert (z == 0).all() and q.min() >= -127 and q.max() <= 127
+    # the largest magnitude takes the end code, with its sign
+    am = np.abs(x).argmax(axis=1)
+    assert (q[np.arange(16), am] == np.sign(x[np.arange(16), am]) * 127).all()
+    # odd symmetry: negating the row negates the codes and keeps the scale
+    qn, sn, _ = oracle.quantize_rows_a8_sym(-x)
+    assert (qn == -q).all() and (sn == s).all()
+    # a power-of-two scaling of the row scales the scale and keeps the codes
+    q2, s2, _ = oracle.quantize_rows_a8_sym(x * np.float32(8.0))
+    assert (q2 == q).all() and (s2 == s * np.float32(8.0)).all()
+    # reconstruction within half a step (plus the float32 rounding of the scales)
+    err = np.abs(x.astype(np.float64) - s.astype(np.float64)[:, None] * q)
+    assert (err <= s.astype(np.float64)[:, None] * 0.5001).all()
+
+
+def test_p12_symmetric_brute_force_nearest_code():
+    rng = np.random.default_rng(121)
+    x = rng.uniform(-3, 3, (4, 40)).astype(np.float32)
+    q, _, _ = oracle.quantize_rows_a8_sym(x)
+    for m in range(4):
+        amax = max(abs(float(v)) for v in x[m])
+        for k in range(40):
+            t = float(x[m, k]) * 127.0 / amax
+            if abs(abs(t - math.floor(t)) - 0.5) < 1e-4:
+                continue  # too close to a tie for a float64 search to decide
+            best = min(range(-127, 128), key=lambda c: abs(c - t))
+            assert q[m, k] == best
+
+
+# ---------------------------------------------------------------------------
+# P13: convolution with a float input quantized per unrolled row (reading R16)
+# ---------------------------------------------------------------------------
+def _direct_dyn_conv(x, qw, sw, stride, pad, bias, lo, hi, symmetric):
+    """Brute force by output pixel: read the taps inside the image with
+    explicit bounds tests, quantize that pixel's values (a pad tap is the
+    value 0, which never widens the range), and sum the dequantized products
+    in float64 with the weight group taken from the (kh, kw, ci) position."""
+    Nb, H, W, Cin = x.shape
+    Cout, KH, KW, _ = qw.shape
+    sh, sw_ = stride
+    ph, pw = pad
+    OH = (H + 2 * ph - KH) // sh + 1
+    OW = (W + 2 * pw - KW) // sw_ + 1
+    quant = oracle.quantize_rows_a8_sym if symmetric else oracle.quantize_rows_a8
+    y = np.zeros((Nb, OH, OW, Cout), np.float32)
+    for n in range(Nb):
+        for oh in range(OH):
+            for ow in range(OW):
+                taps = []
+                for kh in range(KH):
+                    for kw in range(KW):
+                        ih, iw = oh * sh + kh - ph, ow * sw_ + kw - pw
+                        if 0 <= ih < H and 0 <= iw < W:
+                            for ci in range(Cin):
+                                taps.append((kh, kw, ci, float(x[n, ih, iw, ci])))
+                vals = np.array([[t[3] for t in taps] + [0.0]], np.float32)
+                q, s, z = quant(vals)
+                for co in range(Cout):
+                    acc = 0.0
+                    for j, (kh, kw, ci, _) in enumerate(taps):
+                        g = ((kh * KW + kw) * Cin + ci) // 32
+                        acc += (float(s[0]) * (int(q[0, j]) - int(z[0]))
+                                * float(sw[co, g]) * int(qw[co, kh, kw, ci]))
+                    if bias is not None:
+                        acc += float(bias[co])
+                    y[n, oh, ow, co] = min(max(np.float32(acc), np.float32(lo)), np.float32(hi))
+    return y
+
+
+def _conv_case(Nb, H, W, Cin, Cout, KH, KW, seed):
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((Nb, H, W, Cin)).astype(np.float32)
+    qw = rng.integers(-8, 8, size=(Cout, KH, KW, Cin)).astype(np.int8)
+    sw = rng.uniform(0.01, 0.1, (Cout, KH * KW * Cin // 32)).astype(np.float32)
+    bias = rng.standard_normal(Cout).astype(np.float32)
+    return x, qw, sw, bias
+
+
+@pytest.mark.parametrize("symmetric", [False, True])
+@pytest.mark.parametrize("H,W,Cin,KH,KW,stride,pad", [
+    (5, 6, 32, 3, 3, (1, 1), (1, 1)),
+    (7, 5, 32, 3, 2, (2, 1), (1, 0)),
+    (4, 4, 64, 1, 1, (2, 2), (0, 0)),
+])
+def test_p13_dynamic_conv_equals_direct_brute_force(symmetric, H, W, Cin, KH, KW, stride, pad):
+    x, qw, sw, bias = _conv_case(2, H, W, Cin, 3, KH, KW, seed=H * 10 + KH)
+    y, _, _, _ = oracle.qconv2d_f32_dyn_a8w4(x, qw, sw, stride, pad, bias, -50.0, 50.0,
+                                             symmetric=symmetric)
+    y_bf = _direct_dyn_conv(x, qw, sw, stride, pad, bias, -50.0, 50.0, symmetric)
+    np.testing.assert_allclose(y, y_bf, rtol=1e-6, atol=1e-6)
+
+
+def test_p13_pointwise_conv_is_the_linear():
+    # a 1x1 conv with unit stride and no pad is the A8W4 linear on [Nb*H*W, Cin]
+    x, qw, sw, bias = _conv_case(2, 3, 4, 64, 5, 1, 1, seed=131)
+    y, qA, sA, za = oracle.qconv2d_f32_dyn_a8w4(x, qw, sw, (1, 1), (0, 0), bias, -6.0, 6.0)
+    y2, qA2, sA2, za2 = oracle.qgemm_a8w4_f32(x.reshape(24, 64), qw.reshape(5, 64), sw, bias,
+                                              -6.0, 6.0)
+    assert (y.reshape(24, 5) == y2).all()
+    assert (qA == qA2).all() and (sA == sA2).all() and (za == za2).all()
+
+
+def test_p13_whole_image_kernel_is_the_linear_on_the_flattened_image():
+    # a kernel the size of the image gives one output pixel: the linear on
+    # the image flattened in (h, w, c) order, which fixes the K order
+    x, qw, sw, bias = _conv_case(3, 2, 3, 32, 4, 2, 3, seed=132)
+    y, _, _, _ = oracle.qconv2d_f32_dyn_a8w4(x, qw, sw, (1, 1), (0, 0), bias, -60.0, 60.0)
+    y2, _, _, _ = oracle.qgemm_a8w4_f32(x.reshape(3, 2 * 3 * 32), qw.reshape(4, 2 * 3 * 32), sw,
+                                        bias, -60.0, 60.0)
+    assert y.shape == (3, 1, 1, 4) and (y.reshape(3, 4) == y2).all()
+
+
+def test_p13_padding_does_not_move_the_quantization_of_a_row():
+    # zero taps never widen the range (0 is always inside it), so an unrolled
+    # row with pad taps has the parameters of its in-image values alone
+    x, _, _, _ = _conv_case(1, 3, 3, 32, 1, 3, 3, seed=133)
+    cols = oracle.im2col_f32(x, 3, 3, (1, 1), (1, 1))
+    corner = cols[0]                                   # output pixel (0, 0): 5 pad taps
+    inside = corner.reshape(3, 3, 32)[1:, 1:].reshape(1, -1)
+    for quant in (oracle.quantize_rows_a8, oracle.quantize_rows_a8_sym):
+        _, s1, z1 = quant(corner[None, :])
+        _, s2, z2 = quant(inside)
+        assert s1[0] == s2[0] and z1[0] == z2[0]
+    assert (corner.reshape(3, 3, 32)[0] == 0).all() and (corner.reshape(3, 3, 32)[:, 0] == 0).all()
+
+
+def test_p13_codes_entry_matches_the_linear():
+    x, qw, sw, bias = _conv_case(1, 4, 8, 32, 6, 1, 1, seed=134)
+    x2 = x.reshape(32, 32)
+    qA, sA, za = oracle.quantize_rows_a8(x2)
+    y = oracle.a8w4_from_codes(qA, sA, za, qw.reshape(6, 32), sw, bias, -6.0, 6.0)
+    y2, _, _, _ = oracle.qgemm_a8w4_f32(x2, qw.reshape(6, 32), sw, bias, -6.0, 6.0)
+    assert (y == y2).all()
