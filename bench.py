@@ -26,7 +26,9 @@ Workloads: int8_gemm_130x70x129, int8_conv_56x56x64_3x3, a8w4_gemv_1x14336x4096,
 a8w4_gemv_bf16s_1x14336x4096 (bf16 group scales), a8w4_gemv_actblock_1x14336x4096
 (activations quantized per 32-wide K block), a8w4_gemv_asym_1x14336x4096
 (asymmetric int4 weights), a8w4_gemm_128x4096x4096,
-int8_gemm_8192x8192x8200.
+int8_gemm_8192x8192x8200, a8w4_conv_f32_56x56x64_3x3 and
+a8w4_conv_f32_sym_56x56x64_3x3 (float-input conv, unrolled rows quantized
+per output pixel, asymmetric or symmetric).
 Under torchrun each rank runs the same work on its own GPU (replicas: the
 path has no exchange step), and value sums all ranks' work.
 """
@@ -389,6 +391,62 @@ class ConvCase:
         return self.d2h_host.numel()
 
 
+class DynConvCase:
+    """Float-input conv: every unrolled row quantized on the fly, int4 weights."""
+
+    def __init__(self, qg, torch, w, sets, symmetric=False):
+        self.qg, self.torch, self.w, self.sym = qg, torch, w, symmetric
+        self.Cout, self.K = w["Cout"], w["K"]
+        self.packed = qg.pack_w4_g32(dev(w["qw"].reshape(self.Cout, self.K), torch),
+                                     dev(w["sw"], torch))
+        x = dev(w["x"], torch)
+        # distinct images (the input shifted along W), together larger than L2
+        self.inputs = [x if s == 0 else torch.roll(x, shifts=s, dims=2) for s in range(sets)]
+        self.bias = dev(w["bias"], torch)
+        self.OH, self.OW = qg.conv_out_hw(w["H"], w["W"], w["KH"], w["KW"], w["stride"], w["pad"])
+        self.P = w["Nb"] * self.OH * self.OW
+        self.y = torch.empty((w["Nb"], self.OH, self.OW, self.Cout), dtype=torch.float32,
+                             device="cuda")
+        wsb = qg.qconv2d_f32_dyn_a8w4_workspace_bytes(x.shape, self.Cout, w["KH"], w["KW"],
+                                                      w["stride"], w["pad"])
+        self.ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+        self.launches = 2        # unroll + quantize, then the CUDA-core A8W4 GEMM
+        self.kernel = "a8w4_gemm_simt_kernel"
+        self.h2d_host = torch.from_numpy(np.ascontiguousarray(w["x"])).pin_memory()
+        self.d2h_host = torch.empty(tuple(self.y.shape), dtype=torch.float32).pin_memory()
+
+    def _call(self, x, stream=None):
+        w = self.w
+        self.qg.qconv2d_f32_dyn_a8w4(x, self.packed, self.Cout, w["KH"], w["KW"], w["stride"],
+                                     w["pad"], self.bias, w["clamp_min"], w["clamp_max"], self.y,
+                                     symmetric=self.sym, workspace=self.ws, stream=stream)
+
+    def run(self, i, stream=None):
+        self._call(self.inputs[i % len(self.inputs)], stream)
+
+    def prep_e2e(self):
+        self.e2e_x = self.torch.empty_like(self.inputs[0])
+
+    def run_e2e(self, i):
+        self.e2e_x.copy_(self.h2d_host, non_blocking=True)
+        self._call(self.e2e_x)
+        self.d2h_host.copy_(self.y, non_blocking=True)
+
+    def ops(self):
+        return a8w4_ops(self.P, self.Cout, self.K)
+
+    def bytes(self):
+        # f32 image + int4 nibbles + f32 group scales + f32 bias + f32 output
+        return (self.inputs[0].numel() * 4 + self.Cout * self.K // 2
+                + self.Cout * (self.K // 32) * 4 + self.Cout * 4 + self.P * self.Cout * 4)
+
+    def h2d(self):
+        return self.h2d_host.numel() * 4
+
+    def d2h(self):
+        return self.d2h_host.numel() * 4
+
+
 def build_cases(workload, qg, torch):
     import workloads as W
     if workload == "headline":
@@ -412,6 +470,10 @@ def build_cases(workload, qg, torch):
         return [("a8w4_gemv_bf16s_1x14336x4096", A8W4Case(qg, torch, W.a8w4_gemv_1x14336x4096(), 9, True), "hbm")]
     if workload == "int8_gemm_8192x8192x8200":
         return [("int8_gemm_8192x8192x8200", GemmCase(qg, torch, W.int8_gemm_8192x8192x8200(), 2), "tensor")]
+    if workload in ("a8w4_conv_f32_56x56x64_3x3", "a8w4_conv_f32_sym_56x56x64_3x3"):
+        # 160 input images of 0.8 MB: 128 MB > L2
+        return [(workload, DynConvCase(qg, torch, W.a8w4_conv_f32_56x56x64_3x3(), 160,
+                                       symmetric="_sym_" in workload), "latency")]
     raise SystemExit(f"unknown workload {workload}")
 
 
@@ -428,6 +490,8 @@ KERNEL_SOURCES = {
     "a8w4_gemv_bf16s_1x14336x4096": "a8w4.cu",
     "a8w4_gemv_actblock_1x14336x4096": "a8w4.cu",
     "a8w4_gemv_asym_1x14336x4096": "a8w4.cu",
+    "a8w4_conv_f32_56x56x64_3x3": "a8w4.cu",
+    "a8w4_conv_f32_sym_56x56x64_3x3": "a8w4.cu",
 }
 
 
@@ -518,6 +582,16 @@ def oracle_sample(workload, budget_s=12.0, rows_gemm=None, small=False):
         dt = time.perf_counter() - t
         ops += gemm_ops(130, 70, 129); spent += dt
         parts.append("int8 GEMM 130x70x129 (whole)")
+    if workload in ("a8w4_conv_f32_56x56x64_3x3", "a8w4_conv_f32_sym_56x56x64_3x3"):
+        w = W.a8w4_conv_f32_56x56x64_3x3()
+        sym = "_sym_" in workload
+        t = time.perf_counter()
+        oracle.qconv2d_f32_dyn_a8w4(w["x"], w["qw"], w["sw"], w["stride"], w["pad"], w["bias"],
+                                    w["clamp_min"], w["clamp_max"], symmetric=sym)
+        dt = time.perf_counter() - t
+        ops += a8w4_ops(3136, 64, 576); spent += dt
+        parts.append(f"float-input dynamic conv ({'symmetric' if sym else 'asymmetric'} rows) "
+                     "1x56x56x64 3x3 (whole)")
     if workload == "int8_conv_56x56x64_3x3":
         w = W.int8_conv_56x56x64_3x3()
         pr = [oracle.requant_params(float(r)) for r in w["ratio"]]
@@ -566,7 +640,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="headline",
-                    choices=["headline", "int8_gemm_130x70x129", "int8_conv_56x56x64_3x3", "a8w4_gemv_1x14336x4096", "a8w4_gemv_bf16s_1x14336x4096", "a8w4_gemv_actblock_1x14336x4096", "a8w4_gemv_asym_1x14336x4096", "a8w4_gemm_128x4096x4096", "int8_gemm_8192x8192x8200"])
+                    choices=["headline", "int8_gemm_130x70x129", "int8_conv_56x56x64_3x3", "a8w4_gemv_1x14336x4096", "a8w4_gemv_bf16s_1x14336x4096", "a8w4_gemv_actblock_1x14336x4096", "a8w4_gemv_asym_1x14336x4096", "a8w4_gemm_128x4096x4096", "int8_gemm_8192x8192x8200",
+                             "a8w4_conv_f32_56x56x64_3x3", "a8w4_conv_f32_sym_56x56x64_3x3"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=10)
     args = ap.parse_args()

@@ -10,7 +10,8 @@ status code.
 The function names are those of the C ABI:
   quantize_rows_a8, pack_w4_g32, qgemm_a8w4_f32,
   qgemm_pack_b_s8, qgemm_s8s8_requant, qgemm_s8s8_requant_packed,
-  qconv2d_s8_im2col, qg_requant_params, qg_device_status
+  qconv2d_s8_im2col, qg_requant_params, qg_device_status,
+  quantize_rows_a8_sym, qconv2d_f32_dyn_a8w4
 plus the *_bytes / *_workspace_bytes size queries.
 """
 from __future__ import annotations
@@ -94,6 +95,10 @@ _sig("pack_w4_g32_asym_bytes", _sz, [_i32, _i32])
 _sig("pack_w4_g32_asym", _i32, [_i32, _i32, _vp, _i64, _vp, _vp, _vp, _sz, _vp])
 _sig("qgemm_a8w4_f32_asym", _i32, [_i32, _i32, _i32, _vp, _i64, _vp, _vp, _f32, _f32, _vp,
                                    _i64, _vp, _vp, _vp, _vp])
+_sig("quantize_rows_a8_sym", _i32, [_i32, _i32, _vp, _i64, _vp, _i64, _vp, _vp])
+_sig("qconv2d_f32_dyn_a8w4_workspace_bytes", _sz, [_i32] * 11)
+_sig("qconv2d_f32_dyn_a8w4", _i32, [_i32] * 11 + [_vp, _vp, _vp, _f32, _f32, _i32, _vp, _vp, _vp,
+                                                  _vp, _vp, _sz, _vp])
 _sig("pack_w4_g32_bf16_bytes", _sz, [_i32, _i32])
 _sig("pack_w4_g32_bf16", _i32, [_i32, _i32, _vp, _i64, _vp, _vp, _sz, _vp])
 _sig("qgemm_a8w4_f32_bf16s", _i32, [_i32, _i32, _i32, _vp, _i64, _vp, _vp, _f32, _f32, _vp,
@@ -324,6 +329,37 @@ def qconv2d_s8_im2col(x, w, y, rq, stride, pad, acc_out=None, workspace=None, st
                                  pad[1], _p(x), _p(w), _p(y), ctypes.byref(rq), _p(acc_out),
                                  _p(workspace), workspace.numel(), _stream(stream)),
            "qconv2d_s8_im2col")
+
+
+def quantize_rows_a8_sym(x, q, scale, stream=None):
+    """Symmetric per-row int8 quantization (zero-point 0)."""
+    M, K = x.shape
+    _check(lib.quantize_rows_a8_sym(M, K, _p(x), _ld(x), _p(q), _ld(q), _p(scale),
+                                    _stream(stream)), "quantize_rows_a8_sym")
+
+
+def qconv2d_f32_dyn_a8w4_workspace_bytes(x_shape, Cout, KH, KW, stride, pad):
+    Nb, H, W, Cin = x_shape
+    return lib.qconv2d_f32_dyn_a8w4_workspace_bytes(Nb, H, W, Cin, Cout, KH, KW, stride[0],
+                                                    stride[1], pad[0], pad[1])
+
+
+def qconv2d_f32_dyn_a8w4(x, packed_w, Cout, KH, KW, stride, pad, bias, clamp_min, clamp_max, y,
+                         symmetric=False, q_out=None, scale_out=None, zp_out=None,
+                         workspace=None, stream=None):
+    """Float NHWC input x [Nb][H][W][Cin], unrolled and quantized per output
+    pixel, times int4 weights packed by pack_w4_g32 from [Cout][KH*KW*Cin];
+    y f32 NHWC [Nb][OH][OW][Cout]."""
+    Nb, H, W, Cin = x.shape
+    assert x.is_contiguous() and y.is_contiguous()
+    if workspace is None:
+        workspace = _empty_bytes(qconv2d_f32_dyn_a8w4_workspace_bytes(x.shape, Cout, KH, KW,
+                                                                      stride, pad), x.device)
+    _check(lib.qconv2d_f32_dyn_a8w4(Nb, H, W, Cin, Cout, KH, KW, stride[0], stride[1], pad[0],
+                                    pad[1], _p(x), _p(packed_w), _p(bias), float(clamp_min),
+                                    float(clamp_max), 1 if symmetric else 0, _p(y), _p(q_out),
+                                    _p(scale_out), _p(zp_out), _p(workspace), workspace.numel(),
+                                    _stream(stream)), "qconv2d_f32_dyn_a8w4")
 
 
 def exported_symbols():

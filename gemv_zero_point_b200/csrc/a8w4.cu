@@ -117,6 +117,128 @@ int launch_quantize_rows(int M, int K, const float* x, int64_t ldx, int8_t* q, i
 }
 
 // ---------------------------------------------------------------------------
+// Gathered rows, quantized on the fly (MNN ConvInt8TiledExecutor, low-memory
+// path: the float input of a tile of output pixels is unrolled and each
+// unrolled row quantized before the int8 product).  One warp per row; a row
+// is `taps` runs of `run` consecutive floats.  CONV: row m is output pixel
+// (n, oh, ow) of an NHWC image, run r = (kh, kw) reads pixel
+// (oh*sh+kh-ph, ow*sw+kw-pw), and a run outside the image is the value 0
+// ([QG] section 2), which is never read and never widens the range (0 is
+// always inside it).  Otherwise row m is x + m*ldx, one run of K.
+// Asymmetric rows take the per-row rule above; symmetric rows
+// (BatchSymDynamicQuant) take amax = max|x|, scale = amax/127, quantizing
+// factor 127/amax (both 1 when amax is 0), codes clamp(rne(x*factor), -127,
+// 127) and zero-point 0.
+// ---------------------------------------------------------------------------
+struct GatherGeom {
+  int H, W, Cin, KH, KW, sh, sw, ph, pw, OH, OW;
+};
+
+constexpr int kGatherWarps = 8;
+
+template <bool SYM, bool CONV>
+__global__ void __launch_bounds__(kGatherWarps * 32) quantize_gathered_rows_kernel(
+    int M, int K, const float* __restrict__ x, int64_t ldx, GatherGeom g,
+    int8_t* __restrict__ q, int64_t ldq, float* __restrict__ scale,
+    int32_t* __restrict__ zero_point) {
+  const int lane = threadIdx.x & 31;
+  const int64_t m = (int64_t)blockIdx.x * kGatherWarps + (threadIdx.x >> 5);
+  if (m >= M) return;
+  const int taps = CONV ? g.KH * g.KW : 1;
+  const int run = CONV ? g.Cin : K;
+  int64_t n = 0;
+  int oh = 0, ow = 0;
+  if (CONV) {
+    ow = (int)(m % g.OW);
+    const int64_t t = m / g.OW;
+    oh = (int)(t % g.OH);
+    n = t / g.OH;
+  }
+  // start of run t of this row, or nullptr for a run outside the image
+  auto run_ptr = [&](int t) -> const float* {
+    if (!CONV) return x + m * ldx;
+    const int kh = t / g.KW, kw = t - kh * g.KW;
+    const int ih = oh * g.sh + kh - g.ph, iw = ow * g.sw + kw - g.pw;
+    if (ih < 0 || ih >= g.H || iw < 0 || iw >= g.W) return nullptr;
+    return x + ((n * g.H + ih) * g.W + iw) * (int64_t)g.Cin;
+  };
+  float mn = 0.0f, mx = 0.0f;
+  for (int t = 0; t < taps; ++t) {
+    const float* p = run_ptr(t);
+    if (!p) continue;
+    for (int c = lane; c < run; c += 32) {
+      const float v = __ldg(p + c);
+      if (SYM) {
+        mx = fmaxf(mx, fabsf(v));
+      } else {
+        mn = fminf(mn, v);
+        mx = fmaxf(mx, v);
+      }
+    }
+  }
+  for (int o = 16; o > 0; o >>= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
+  RowQuant r;
+  if (SYM) {
+    r.scale = mx == 0.0f ? 1.0f : __fdiv_rn(mx, 127.0f);
+    r.inv = mx == 0.0f ? 1.0f : __fdiv_rn(127.0f, mx);
+    r.zp = 0;
+  } else {
+    r = row_quant_params(mn, mx);
+  }
+  int8_t* qr = q + m * ldq;
+  for (int t = 0; t < taps; ++t) {
+    const float* p = run_ptr(t);
+    int8_t* qt = qr + (int64_t)t * run;
+    for (int c = lane; c < run; c += 32) {
+      const float v = p ? __ldg(p + c) : 0.0f;
+      int code;
+      if (SYM)
+        code = min(max(__float2int_rn(__fmul_rn(v, r.inv)), -127), 127);
+      else
+        code = quant_one(v, r);
+      qt[c] = (int8_t)code;
+    }
+  }
+  if (lane == 0) {
+    scale[m] = r.scale;
+    if (zero_point) zero_point[m] = r.zp;
+  }
+}
+
+int launch_quantize_rows_sym(int M, int K, const float* x, int64_t ldx, int8_t* q, int64_t ldq,
+                             float* scale, int32_t* zp, cudaStream_t st) {
+  if (M == 0) return QG_OK;
+  const GatherGeom g{};
+  quantize_gathered_rows_kernel<true, false>
+      <<<(unsigned)cdiv(M, kGatherWarps), kGatherWarps * 32, 0, st>>>(M, K, x, ldx, g, q, ldq,
+                                                                      scale, zp);
+  return launch_status();
+}
+
+// Unrolled rows of an NHWC float image: P = Nb*OH*OW rows of K = KH*KW*Cin
+// codes, row-major with ld K.
+int launch_im2col_quantize(int Nb, int H, int W, int Cin, int KH, int KW, int sh, int sw, int ph,
+                           int pw, const float* x, bool symmetric, int8_t* q, float* scale,
+                           int32_t* zp, cudaStream_t st) {
+  const int OH = (H + 2 * ph - KH) / sh + 1, OW = (W + 2 * pw - KW) / sw + 1;
+  const int64_t P = (int64_t)Nb * OH * OW;
+  const int K = KH * KW * Cin;
+  if (P == 0) return QG_OK;
+  const GatherGeom g{H, W, Cin, KH, KW, sh, sw, ph, pw, OH, OW};
+  const unsigned grid = (unsigned)cdiv(P, kGatherWarps);
+  if (symmetric)
+    quantize_gathered_rows_kernel<true, true>
+        <<<grid, kGatherWarps * 32, 0, st>>>((int)P, K, x, 0, g, q, K, scale, zp);
+  else
+    quantize_gathered_rows_kernel<false, true>
+        <<<grid, kGatherWarps * 32, 0, st>>>((int)P, K, x, 0, g, q, K, scale, zp);
+  return launch_status();
+}
+
+// ---------------------------------------------------------------------------
 // W4 pack: one thread per output 32-bit word (8 consecutive k of a row).
 // word j of row n: byte b = (w[8j+b]+8) | (w[8j+4+b]+8) << 4.
 // ---------------------------------------------------------------------------

@@ -28,6 +28,11 @@ int launch_a8w4_gemv_actblock(int N, int K, const float* x, const void* packed, 
 int launch_a8w4_gemv_asym(int N, int K, const float* x, const void* packed, const float* bias,
                           float lo, float hi, float* y, int8_t* q_out, float* scale_out,
                           int32_t* zp_out, cudaStream_t st);
+int launch_quantize_rows_sym(int M, int K, const float* x, int64_t ldx, int8_t* q, int64_t ldq,
+                             float* scale, int32_t* zp, cudaStream_t st);
+int launch_im2col_quantize(int Nb, int H, int W, int Cin, int KH, int KW, int sh, int sw, int ph,
+                           int pw, const float* x, bool symmetric, int8_t* q, float* scale,
+                           int32_t* zp, cudaStream_t st);
 int setup_a8w4_gemv();
 int setup_a8w4_gemm_simt();
 int i8gemm_setup();
@@ -500,4 +505,96 @@ extern "C" int qgemm_a8w4_f32_asym(int M, int N, int K, const float* x, int64_t 
   if (rc != QG_OK) return rc;
   return launch_a8w4_gemv_asym(N, K, x, packed_w, bias, clamp_min, clamp_max, y, q_out,
                                scale_out, zp_out, (cudaStream_t)stream);
+}
+
+// ---------------------------------------------------------------------------
+// Symmetric row quantization; float-input convolution with dynamic int8
+// activations and int4 weights
+// ---------------------------------------------------------------------------
+extern "C" int quantize_rows_a8_sym(int M, int K, const float* x, int64_t ldx, int8_t* q,
+                                    int64_t ldq, float* scale, void* stream) {
+  if (M < 0 || K <= 0 || ldx < K || ldq < K) return QG_ERR_INVALID_ARG;
+  if (M == 0) return QG_OK;
+  if (!x || !q || !scale) return QG_ERR_INVALID_ARG;
+  if (!aligned(x, 4) || !aligned(scale, 4)) return QG_ERR_MISALIGNED;
+  int rc = device_ready();
+  if (rc != QG_OK) return rc;
+  return launch_quantize_rows_sym(M, K, x, ldx, q, ldq, scale, nullptr, (cudaStream_t)stream);
+}
+
+// The conv's GEMM runs on the CUDA-core A8W4 kernel: 8 unrolled rows per CTA
+// row of the grid (at most 65535 of them) and 8*K bytes of shared memory.
+static const int64_t kDynConvMaxRows = 65535 * 8;
+
+// Unrolled-matrix shape of a float-input conv: QG_OK with P rows of K, or
+// the status the call returns.
+static int dynconv_shape(int Nb, int H, int W, int Cin, int Cout, int KH, int KW, int sh, int sw,
+                         int ph, int pw, int64_t* P, int* K) {
+  if (Nb <= 0 || H <= 0 || W <= 0 || Cin <= 0 || Cout <= 0 || KH <= 0 || KW <= 0 || sh <= 0 ||
+      sw <= 0 || ph < 0 || pw < 0)
+    return QG_ERR_INVALID_ARG;
+  if ((int64_t)H + 2 * (int64_t)ph < KH || (int64_t)W + 2 * (int64_t)pw < KW)
+    return QG_ERR_INVALID_ARG;
+  const int64_t k = (int64_t)KH * KW * Cin;
+  if (k % 32) return QG_ERR_UNSUPPORTED;
+  if (k > kSimtMaxK) return QG_ERR_UNSUPPORTED;
+  const int64_t OH = ((int64_t)H + 2 * (int64_t)ph - KH) / sh + 1;
+  const int64_t OW = ((int64_t)W + 2 * (int64_t)pw - KW) / sw + 1;
+  const int64_t p = (int64_t)Nb * OH * OW;
+  if (p > kDynConvMaxRows) return QG_ERR_UNSUPPORTED;
+  *P = p;
+  *K = (int)k;
+  return QG_OK;
+}
+
+extern "C" size_t qconv2d_f32_dyn_a8w4_workspace_bytes(int Nb, int H, int W, int Cin, int Cout,
+                                                       int KH, int KW, int stride_h,
+                                                       int stride_w, int pad_h, int pad_w) {
+  int64_t P = 0;
+  int K = 0;
+  if (dynconv_shape(Nb, H, W, Cin, Cout, KH, KW, stride_h, stride_w, pad_h, pad_w, &P, &K) !=
+      QG_OK)
+    return 0;
+  return a8w4_ws_layout((int)P, K, nullptr, nullptr);
+}
+
+extern "C" int qconv2d_f32_dyn_a8w4(int Nb, int H, int W, int Cin, int Cout, int KH, int KW,
+                                    int stride_h, int stride_w, int pad_h, int pad_w,
+                                    const float* x, const void* packed_w, const float* bias,
+                                    float clamp_min, float clamp_max, int symmetric, float* y,
+                                    int8_t* q_out, float* scale_out, int32_t* zp_out,
+                                    void* workspace, size_t workspace_bytes, void* stream) {
+  int64_t P = 0;
+  int K = 0;
+  int rc = dynconv_shape(Nb, H, W, Cin, Cout, KH, KW, stride_h, stride_w, pad_h, pad_w, &P, &K);
+  if (rc != QG_OK) return rc;
+  if (symmetric != 0 && symmetric != 1) return QG_ERR_INVALID_ARG;
+  if (!(clamp_min <= clamp_max)) return QG_ERR_INVALID_ARG;  // also rejects NaN
+  if (!x || !packed_w || !y) return QG_ERR_INVALID_ARG;
+  if (!aligned(packed_w, 16)) return QG_ERR_MISALIGNED;
+  if (!aligned(x, 4) || !aligned(y, 4) || (bias && !aligned(bias, 4))) return QG_ERR_MISALIGNED;
+  if ((scale_out && !aligned(scale_out, 4)) || (zp_out && !aligned(zp_out, 4)))
+    return QG_ERR_MISALIGNED;
+  size_t off_s = 0, off_z = 0;
+  const size_t need = a8w4_ws_layout((int)P, K, &off_s, &off_z);
+  if (!workspace || workspace_bytes < need) return QG_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return QG_ERR_MISALIGNED;
+  rc = device_ready();
+  if (rc != QG_OK) return rc;
+  cudaStream_t st = (cudaStream_t)stream;
+  int8_t* q = (int8_t*)workspace;
+  float* sA = (float*)((char*)workspace + off_s);
+  int32_t* zA = (int32_t*)((char*)workspace + off_z);
+  rc = launch_im2col_quantize(Nb, H, W, Cin, KH, KW, stride_h, stride_w, pad_h, pad_w, x,
+                              symmetric != 0, q, sA, zA, st);
+  if (rc != QG_OK) return rc;
+  if (q_out && cudaMemcpyAsync(q_out, q, (size_t)P * K, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    return QG_ERR_CUDA;
+  if (scale_out &&
+      cudaMemcpyAsync(scale_out, sA, (size_t)P * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    return QG_ERR_CUDA;
+  if (zp_out && cudaMemcpyAsync(zp_out, zA, (size_t)P * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    return QG_ERR_CUDA;
+  return launch_a8w4_gemm_simt((int)P, Cout, K, q, sA, zA, packed_w, bias, clamp_min, clamp_max, y,
+                               Cout, false, st);
 }

@@ -309,6 +309,55 @@ int qgemm_a8w4_f32_asym(int M, int N, int K, const float* x, int64_t ldx,
                         void* stream);
 
 /* ------------------------------------------------------------------------
+ * Dynamic per-row symmetric int8 activation quantization.  [MNN]
+ * ConvInt8TiledExecutor, BatchSymDynamicQuant: the absolute maximum of each
+ * row gives a quantizing and a dequantizing scale, and the zero-point is 0.
+ * All float32, one rounding per operation:
+ *   amax = max_k |x[k]|
+ *   scale = amax/127 and factor = 127/amax, both 1 if amax is 0
+ *   q[k] = clamp(rne(x[k]*factor), -127, 127)
+ *   x: f32 [M][ldx] (ldx >= K); q: int8 [M][ldq] (ldq >= K); scale: f32 [M].
+ * Non-finite x is out of contract.
+ * ------------------------------------------------------------------------ */
+int quantize_rows_a8_sym(int M, int K, const float* x, int64_t ldx,
+                         int8_t* q, int64_t ldq, float* scale, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Convolution of a float input quantized on the fly, with int4 weights.
+ * [MNN] ConvInt8TiledExecutor, low-memory path: the float input of a tile of
+ * output pixels is unrolled (im2col) and every unrolled row is quantized
+ * dynamically, asymmetric (BatchAsyDynamicQuant) or symmetric
+ * (BatchSymDynamicQuant), before the int8 x int4 block-quantized product;
+ * [QG] section 2: a tap in the padding stands for the real value 0.
+ *
+ *   x: f32 NHWC [Nb][H][W][Cin], 4-byte aligned
+ *   packed_w: pack_w4_g32 of the int4 codes [Cout][KH][KW][Cin] read as
+ *     [Cout][K], K = KH*KW*Cin in (kh, kw, ci) order, one scale per 32
+ *     consecutive k of that order (K % 32 == 0, else QG_ERR_UNSUPPORTED)
+ *   bias: f32 [Cout] or NULL;  y: f32 NHWC [Nb][OH][OW][Cout],
+ *     OH = (H+2*pad_h-KH)/stride_h + 1 (same for W)
+ * Unrolled row p = (n*OH+oh)*OW+ow holds x[n, oh*stride_h+kh-pad_h,
+ * ow*stride_w+kw-pad_w, ci], 0 for a tap outside the image.  It is quantized
+ * by quantize_rows_a8's rule (symmetric = 0) or quantize_rows_a8_sym's
+ * (symmetric = 1, zero-point 0), and
+ *   y[p, co] = clamp(sA[p] * sum_g sw[co,g] * I[p,co,g] + bias[co])
+ *   I[p,co,g] = sum_{k in g} (qA[p,k] - zA[p]) * w[co,k]   (exact integer)
+ * as qgemm_a8w4_f32.  q_out [P][K] int8 / scale_out [P] / zp_out [P] int32
+ * (P = Nb*OH*OW): optional, receive the unrolled row quantization.
+ * Workspace: qconv2d_f32_dyn_a8w4_workspace_bytes (256-byte aligned).
+ * Limits: K <= 25600 and P <= 524280 (else QG_ERR_UNSUPPORTED).
+ * ------------------------------------------------------------------------ */
+size_t qconv2d_f32_dyn_a8w4_workspace_bytes(int Nb, int H, int W, int Cin, int Cout,
+                                            int KH, int KW, int stride_h, int stride_w,
+                                            int pad_h, int pad_w);
+int qconv2d_f32_dyn_a8w4(int Nb, int H, int W, int Cin, int Cout, int KH, int KW,
+                         int stride_h, int stride_w, int pad_h, int pad_w,
+                         const float* x, const void* packed_w, const float* bias,
+                         float clamp_min, float clamp_max, int symmetric, float* y,
+                         int8_t* q_out, float* scale_out, int32_t* zp_out,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * qgemm_a8w4_f32 without a workspace.  The pages have no counterpart: this
  * entry point exists for callers that cannot allocate device memory for
  * scratch — a plugin inside a host framework that owns the allocator and

@@ -19,6 +19,8 @@ def test_exports_every_declared_symbol():
     for expected in ["quantize_rows_a8", "pack_w4_g32", "qgemm_a8w4_f32", "qgemm_s8s8_requant",
                      "pack_w4_g32_bf16", "qgemm_a8w4_f32_bf16s", "qgemm_a8w4_f32_actblock",
                      "pack_w4_g32_asym", "qgemm_a8w4_f32_asym",
+                     "quantize_rows_a8_sym", "qconv2d_f32_dyn_a8w4",
+                     "qconv2d_f32_dyn_a8w4_workspace_bytes",
                      "qconv2d_s8_im2col", "qgemm_pack_b_s8", "qgemm_s8s8_requant_packed",
                      "qg_requant_params", "qg_status_string", "qg_device_status"]:
         assert expected in names
@@ -161,3 +163,47 @@ def test_asym_entry_points_validation():
     assert f(2, 8, 128, FAKE, 128, FAKE, NULL, -1.0, 1.0, FAKE, 8, NULL, NULL, NULL, NULL) == -4
     assert f(1, 8, 128, FAKE, 128, FAKE, NULL, 1.0, -1.0, FAKE, 8, NULL, NULL, NULL, NULL) == -1
     assert f(0, 8, 128, FAKE, 128, FAKE, NULL, -1.0, 1.0, FAKE, 8, NULL, NULL, NULL, NULL) == 0
+
+
+def test_symmetric_quantization_validation():
+    f = lib.quantize_rows_a8_sym
+    assert f(0, 16, NULL, 16, NULL, 16, NULL, NULL) == 0                  # empty
+    assert f(-1, 16, FAKE, 16, FAKE, 16, FAKE, NULL) == -1
+    assert f(2, 16, FAKE, 15, FAKE, 16, FAKE, NULL) == -1                 # ldx < K
+    assert f(2, 16, FAKE, 16, FAKE, 15, FAKE, NULL) == -1                 # ldq < K
+    assert f(2, 16, NULL, 16, FAKE, 16, FAKE, NULL) == -1
+    assert f(2, 16, ctypes.c_void_p(0x10002), 16, FAKE, 16, FAKE, NULL) == -2
+
+
+def test_dynamic_conv_workspace_and_validation():
+    ws = lib.qconv2d_f32_dyn_a8w4_workspace_bytes
+    # 56x56x64 3x3 pad 1: 3136 unrolled rows of K = 576 codes, scales, zero-points
+    assert ws(1, 56, 56, 64, 64, 3, 3, 1, 1, 1, 1) >= 3136 * 576 + 2 * 3136 * 4
+    assert ws(1, 56, 56, 60, 64, 3, 3, 1, 1, 1, 1) == 0                   # K % 32
+    assert ws(1, 4, 4, 32, 8, 5, 5, 1, 1, 0, 0) == 0                      # kernel larger than image
+    assert ws(1, 8, 8, 1024, 8, 5, 5, 1, 1, 2, 2) > 0                     # K = 25600: the limit
+    assert ws(1, 8, 8, 25632, 8, 1, 1, 1, 1, 0, 0) == 0                   # K = 25632: over it
+    f = lib.qconv2d_f32_dyn_a8w4
+    geo = [1, 8, 8, 32, 16, 3, 3, 1, 1, 1, 1]
+    big = 1 << 30
+
+    def call(g=geo, x=FAKE, w=FAKE, lo=-1.0, hi=1.0, sym=0, y=FAKE, ws_=FAKE, wsb=big, s=NULL):
+        return f(*g, x, w, NULL, lo, hi, sym, y, NULL, s, NULL, ws_, wsb, NULL)
+
+    assert call(g=[1, 8, 8, 30, 16, 3, 3, 1, 1, 1, 1]) == -4             # K = 270, not % 32
+    assert call(g=[1, 8, 8, 32, 16, 3, 3, 0, 1, 1, 1]) == -1             # stride 0
+    assert call(g=[1, 8, 8, 32, 16, 3, 3, 1, 1, -1, 1]) == -1            # negative pad
+    assert call(g=[1, 2, 8, 32, 16, 5, 3, 1, 1, 1, 1]) == -1             # KH > H + 2*pad
+    assert call(g=[1, 8, 8, 3200, 16, 3, 3, 1, 1, 1, 1]) == -4           # K = 28800 > 25600
+    assert call(g=[200, 56, 56, 32, 16, 1, 1, 1, 1, 0, 0]) == -4         # 627200 unrolled rows
+    assert call(sym=2) == -1
+    assert call(lo=1.0, hi=-1.0) == -1
+    assert call(lo=float("nan")) == -1
+    assert call(x=NULL) == -1 and call(w=NULL) == -1 and call(y=NULL) == -1
+    assert call(w=ctypes.c_void_p(0x10008)) == -2                        # packed 16-byte aligned
+    assert call(x=ctypes.c_void_p(0x10002)) == -2
+    assert call(s=ctypes.c_void_p(0x10002)) == -2
+    assert call(ws_=NULL) == -7
+    need = ws(*geo)
+    assert call(wsb=need - 1) == -7
+    assert call(ws_=ctypes.c_void_p(0x10080)) == -2                     # workspace 256-byte aligned

@@ -6,8 +6,8 @@ quantization, no requantization, no packing, no matmul).  Both the CPU oracle
 tests and the GPU tests / benchmark take their inputs from here, so the two
 sides see identical data.
 
-Generator: ``numpy.random.default_rng(seed)`` (PCG64).  Seeds 1001..1005 are
-the five standard workloads in the order listed in ``WORKLOADS``.
+Generator: ``numpy.random.default_rng(seed)`` (PCG64).  Seeds 1001..1006 are
+the standard workloads listed in ``WORKLOADS``.
 
 Workload shapes follow the quantized GEMM case study (xidianedu, "量化 GEMM：
 数值契约、SRAM、DMA 与结果验证", "明确范围": M=130, N=70, K=129) and the A8W4
@@ -142,10 +142,34 @@ def a8w4_gemm_128x4096x4096(seed=1004):
     return a8w4(128, 4096, 4096, seed)
 
 
+def a8w4_conv_f32(Nb, H, W, Cin, Cout, KH, KW, stride, pad, seed, *, clamp=(-6.0, 6.0)):
+    """f32 NHWC input N(0,1) [Nb][H][W][Cin]; int4 weight codes uniform in
+    [-8,7] stored one per int8 as qw[Cout][KH][KW][Cin]; f32 group scales
+    sw[Cout][KH*KW*Cin/32] log-uniform [1e-3, 1e-1]; f32 bias N(0, 0.1);
+    output clamp."""
+    K = KH * KW * Cin
+    assert K % 32 == 0
+    rng = _rng(seed)
+    x = rng.standard_normal((Nb, H, W, Cin), dtype=np.float32)
+    qw = _int8(rng, (Cout, KH, KW, Cin), -8, 7)
+    sw = _log_uniform(rng, (Cout, K // 32), 1e-3, 1e-1)
+    bias = rng.normal(0.0, 0.1, size=Cout).astype(np.float32)
+    return dict(Nb=Nb, H=H, W=W, Cin=Cin, Cout=Cout, KH=KH, KW=KW, stride=tuple(stride),
+                pad=tuple(pad), K=K, x=x, qw=qw, sw=sw, bias=bias,
+                clamp_min=float(clamp[0]), clamp_max=float(clamp[1]))
+
+
+def a8w4_conv_f32_56x56x64_3x3(seed=1006):
+    """Float-input dynamic conv: Nb=1, 56x56, Cin=Cout=64, 3x3, stride 1,
+    pad 1 (the INT8 conv's shape, K = 576)."""
+    return a8w4_conv_f32(1, 56, 56, 64, 64, 3, 3, (1, 1), (1, 1), seed)
+
+
 WORKLOADS = {
     "int8_gemm_130x70x129": int8_gemm_130x70x129,
     "int8_conv_56x56x64_3x3": int8_conv_56x56x64_3x3,
     "a8w4_gemv_1x14336x4096": a8w4_gemv_1x14336x4096,
     "a8w4_gemm_128x4096x4096": a8w4_gemm_128x4096x4096,
     "int8_gemm_8192x8192x8200": int8_gemm_8192x8192x8200,
+    "a8w4_conv_f32_56x56x64_3x3": a8w4_conv_f32_56x56x64_3x3,
 }
