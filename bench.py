@@ -523,14 +523,25 @@ def traffic_for(kernel):
 # ---------------------------------------------------------------------------
 # CPU oracle timing (bounded sample)
 # ---------------------------------------------------------------------------
+_WORKLOAD_CACHE = {}
+
+
+def _inputs(name):
+    """The seeded inputs of a workload, drawn once per process (drawing the
+    8192x8200 GEMM's operands takes longer than the sample it feeds)."""
+    if name not in _WORKLOAD_CACHE:
+        import workloads
+        _WORKLOAD_CACHE[name] = getattr(workloads, name)()
+    return _WORKLOAD_CACHE[name]
+
+
 def oracle_sample(workload, budget_s=12.0, rows_gemm=None, small=False):
     """Time the CPU oracle, as it stands, on a bounded sample of the workload.
     Returns (ops per second, seconds spent, description)."""
     import oracle
-    import workloads as W
     ops, spent, parts = 0.0, 0.0, []
     if workload in ("headline", "int8_gemm_8192x8192x8200"):
-        w = W.int8_gemm_8192x8192x8200()
+        w = _inputs("int8_gemm_8192x8192x8200")
         m0 = np.array([oracle.requant_params(float(r))[0] for r in w["ratio"]])
         sh = np.array([oracle.requant_params(float(r))[1] for r in w["ratio"]])
         cols = 512 if small else w["N"]
@@ -543,7 +554,7 @@ def oracle_sample(workload, budget_s=12.0, rows_gemm=None, small=False):
         ops += gemm_ops(rows, cols, w["K"]); spent += dt
         parts.append(f"int8 GEMM {rows} row(s) x {cols} cols of 8192x8192x8200")
     if workload == "a8w4_gemv_asym_1x14336x4096":
-        w = W.a8w4_gemv_1x14336x4096()
+        w = _inputs("a8w4_gemv_1x14336x4096")
         n = 512 if small else w["N"]
         zw = (w["sw"][:n] * np.random.default_rng(77).uniform(-8, 8, w["sw"][:n].shape)).astype(np.float32)
         t = time.perf_counter()
@@ -553,7 +564,7 @@ def oracle_sample(workload, budget_s=12.0, rows_gemm=None, small=False):
         parts.append(f"A8W4 GEMV (asymmetric weights) {n} of 14336 rows")
     if workload in ("headline", "a8w4_gemv_1x14336x4096", "a8w4_gemv_bf16s_1x14336x4096",
                     "a8w4_gemv_actblock_1x14336x4096"):
-        w = W.a8w4_gemv_1x14336x4096()
+        w = _inputs("a8w4_gemv_1x14336x4096")
         n = 512 if small else w["N"]
         t = time.perf_counter()
         fn = {"a8w4_gemv_bf16s_1x14336x4096": oracle.qgemm_a8w4_f32_bf16s,
@@ -566,7 +577,7 @@ def oracle_sample(workload, budget_s=12.0, rows_gemm=None, small=False):
                "a8w4_gemv_actblock_1x14336x4096": " (per-block activations)"}.get(workload, "")
         parts.append(f"A8W4 GEMV{tag} {n} of 14336 rows")
     if workload == "a8w4_gemm_128x4096x4096":
-        w = W.a8w4_gemm_128x4096x4096()
+        w = _inputs("a8w4_gemm_128x4096x4096")
         rows = 1 if small else 4
         t = time.perf_counter()
         oracle.qgemm_a8w4_f32(w["x"][:rows], w["qw"], w["sw"], w["bias"], -6.0, 6.0)
@@ -574,7 +585,7 @@ def oracle_sample(workload, budget_s=12.0, rows_gemm=None, small=False):
         ops += a8w4_ops(rows, w["N"], w["K"]); spent += dt
         parts.append(f"A8W4 GEMM {rows} of 128 rows")
     if workload == "int8_gemm_130x70x129":
-        w = W.int8_gemm_130x70x129()
+        w = _inputs("int8_gemm_130x70x129")
         m0, sh = oracle.requant_params(float(w["ratio"][0]))
         t = time.perf_counter()
         oracle.qgemm_s8s8_requant(w["A"], w["B"], w["za"], w["zb"], w["bias"], m0, sh,
@@ -583,7 +594,7 @@ def oracle_sample(workload, budget_s=12.0, rows_gemm=None, small=False):
         ops += gemm_ops(130, 70, 129); spent += dt
         parts.append("int8 GEMM 130x70x129 (whole)")
     if workload in ("a8w4_conv_f32_56x56x64_3x3", "a8w4_conv_f32_sym_56x56x64_3x3"):
-        w = W.a8w4_conv_f32_56x56x64_3x3()
+        w = _inputs("a8w4_conv_f32_56x56x64_3x3")
         sym = "_sym_" in workload
         t = time.perf_counter()
         oracle.qconv2d_f32_dyn_a8w4(w["x"], w["qw"], w["sw"], w["stride"], w["pad"], w["bias"],
@@ -593,7 +604,7 @@ def oracle_sample(workload, budget_s=12.0, rows_gemm=None, small=False):
         parts.append(f"float-input dynamic conv ({'symmetric' if sym else 'asymmetric'} rows) "
                      "1x56x56x64 3x3 (whole)")
     if workload == "int8_conv_56x56x64_3x3":
-        w = W.int8_conv_56x56x64_3x3()
+        w = _inputs("int8_conv_56x56x64_3x3")
         pr = [oracle.requant_params(float(r)) for r in w["ratio"]]
         m0 = np.array([p[0] for p in pr]); sh = np.array([p[1] for p in pr])
         t = time.perf_counter()
