@@ -1,12 +1,14 @@
-// A8W4 path: dynamic per-row int8 activation quantization, int4 group-32
-// weight packing, and the A8W4 linear (fused M=1 GEMV; M>1 GEMM).
+// A8W4 path: dynamic per-row int8 activation quantization (asymmetric, and
+// symmetric or gathered from an unrolled conv input), int4 group-32 weight
+// packing, and the A8W4 linear (fused M=1 GEMV; M>1 GEMM).
 //
 // Sources: pytorch/ao PR #997 "Kleidi 4b blockwise gemv prototype"
 // (matmul_clamp_f32_qai8dxp_qsi4c32p: int8 dynamic per-row asymmetric
 // activations, int4 symmetric weights with one scale per 32 K, f32 output
 // clamped after the bias); MNN ConvInt8TiledExecutor.cpp
-// (BatchAsyDynamicQuant min/max quantization; int4 weights stored with an
-// offset of 8 in _computeReorderQuantInfo).
+// (BatchAsyDynamicQuant min/max quantization, BatchSymDynamicQuant absolute
+// maximum quantization, the low-memory float im2col path; int4 weights
+// stored with an offset of 8 in _computeReorderQuantInfo).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <math.h>

@@ -6,7 +6,8 @@
  *         numeric contract, SRAM, DMA and result verification), sections 1-5.
  *   [MNN] MNN source/backend/cpu/compute/ConvInt8TiledExecutor.cpp
  *         (initializeConvInt8QuantInfo, reorderWeight, _computeReorderQuantInfo,
- *          BatchAsyDynamicQuant, tileSplitFunction / QuanPostTreatParameters).
+ *          BatchAsyDynamicQuant, BatchSymDynamicQuant, the low-memory float
+ *          im2col path, tileSplitFunction / QuanPostTreatParameters).
  *   [KAI] pytorch/ao PR #997, "Kleidi 4b blockwise gemv prototype"
  *         (matmul_clamp_f32_qai8dxp_qsi4c32p micro-kernels and their wrapper).
  *
