@@ -447,6 +447,13 @@ class DynConvCase:
         return self.d2h_host.numel() * 4
 
 
+WORKLOAD_NAMES = ["headline", "int8_gemm_130x70x129", "int8_conv_56x56x64_3x3",
+                  "a8w4_gemv_1x14336x4096", "a8w4_gemv_bf16s_1x14336x4096",
+                  "a8w4_gemv_actblock_1x14336x4096", "a8w4_gemv_asym_1x14336x4096",
+                  "a8w4_gemm_128x4096x4096", "int8_gemm_8192x8192x8200",
+                  "a8w4_conv_f32_56x56x64_3x3", "a8w4_conv_f32_sym_56x56x64_3x3"]
+
+
 def build_cases(workload, qg, torch):
     import workloads as W
     if workload == "headline":
@@ -650,9 +657,7 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="headline",
-                    choices=["headline", "int8_gemm_130x70x129", "int8_conv_56x56x64_3x3", "a8w4_gemv_1x14336x4096", "a8w4_gemv_bf16s_1x14336x4096", "a8w4_gemv_actblock_1x14336x4096", "a8w4_gemv_asym_1x14336x4096", "a8w4_gemm_128x4096x4096", "int8_gemm_8192x8192x8200",
-                             "a8w4_conv_f32_56x56x64_3x3", "a8w4_conv_f32_sym_56x56x64_3x3"])
+    ap.add_argument("--workload", default="headline", choices=WORKLOAD_NAMES)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=10)
     args = ap.parse_args()
