@@ -38,7 +38,8 @@ def test_status_strings_and_version():
 def test_requant_params_match_oracle_bit_exact():
     rng = np.random.default_rng(0)
     ratios = list(np.exp(rng.uniform(np.log(1e-9), np.log(0.9999), 2000)))
-    ratios += [0.5, 0.25, 0.75, 2.0 ** -10, 2.0 ** -31, 0.999999999, 1e-4, 1e-2]
+    ratios += [0.5, 0.25, 0.75, 2.0 ** -10, 2.0 ** -31, 0.999999999, 1e-4, 1e-2,
+               0.5 - 2.0 ** -34, 0.25 - 2.0 ** -35, 0.5 - 2.0 ** -31]
     for r in ratios:
         try:
             ref = oracle.requant_params(r)

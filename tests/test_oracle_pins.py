@@ -229,6 +229,15 @@ def test_requant_params_closed_forms():
             oracle.requant_params(bad)
 
 
+def test_requant_params_carry_into_the_next_power_of_two():
+    # f = 1 - 2^-33 rounds to 2^31 at 31 bits, which does not fit int32: the
+    # multiplier becomes 2^30 one binade up, i.e. exactly 0.5 (resp. 0.25)
+    assert oracle.requant_params(0.5 - 2.0 ** -34) == (2 ** 30, 0)
+    assert oracle.requant_params(0.25 - 2.0 ** -35) == (2 ** 30, 1)
+    # one step further from the power of two stays below it
+    assert oracle.requant_params(0.5 - 2.0 ** -31) == (2 ** 31 - 2, 1)
+
+
 def test_requant_round_half_even_cases():
     m0, sh = oracle.requant_params(0.5)            # divides by exactly 2
     acc = np.array([3, 5, 7, -3, -5, -7, 1, -1, 4])
