@@ -71,6 +71,7 @@ def _sig(name, res, args):
 _sig("qg_status_string", ctypes.c_char_p, [_i32])
 _sig("qg_version", _i32, [])
 _sig("qg_device_status", _i32, [_i32])
+_sig("qg_test_arm_stall", _i32, [_i32])
 _sig("qg_requant_params", _i32, [_f64, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32)])
 _sig("qgemm_s8s8_workspace_bytes", _sz, [_i32, _i32, _i32])
 _sig("qgemm_s8s8_requant", _i32, [_i32, _i32, _i32, _vp, _i64, _vp, _i64, _vp, _i64,
@@ -138,6 +139,13 @@ def _empty_bytes(n, device):
 # ---------------------------------------------------------------------------
 def qg_device_status(reset=True):
     return lib.qg_device_status(1 if reset else 0)
+
+
+def qg_test_arm_stall(which):
+    """Test hook: arm one stalled pipeline for the next launch of a kernel
+    family (1 = INT8 GEMM one-CTA kernel, 2 = A8W4 tensor-core kernel, 0 =
+    disarm); see include/qgemm.h."""
+    _check(lib.qg_test_arm_stall(int(which)), "qg_test_arm_stall")
 
 
 def qg_requant_params(ratio):

@@ -5,6 +5,7 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "qg_internal.cuh"
@@ -118,6 +119,15 @@ static int device_ready() {
 // Per-device set-up status for entry points defined in other files.
 int device_setup_status() { return device_ready(); }
 
+// One-shot stall armed by qg_test_arm_stall: the next launch of the named
+// kernel family takes it (and only that launch).
+static std::atomic<int> g_stall_armed{kStallNone};
+
+bool take_stall(int target) {
+  int expected = target;
+  return target != kStallNone && g_stall_armed.compare_exchange_strong(expected, kStallNone);
+}
+
 }  // namespace qg
 
 using namespace qg;
@@ -153,6 +163,13 @@ extern "C" int qg_device_status(int reset) {
     if (cudaMemset(status_word(), 0, sizeof(int)) != cudaSuccess) return QG_ERR_CUDA;
   }
   return v;
+}
+
+extern "C" int qg_test_arm_stall(int which) {
+  if (which != kStallNone && which != kStallInt8Gemm && which != kStallA8W4TC)
+    return QG_ERR_INVALID_ARG;
+  g_stall_armed.store(which);
+  return QG_OK;
 }
 
 extern "C" int qg_requant_params(double ratio, int32_t* m0, int32_t* shift) {

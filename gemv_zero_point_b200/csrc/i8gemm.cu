@@ -142,6 +142,8 @@ struct EpiArgs {
   int64_t ldc;
   int32_t* acc_out;
   int64_t ld_acc;
+  int stall;        // test hook (one-CTA kernel): skip the loads of K block 1 of the first tile
+  uint32_t spin;    // poll limit of the pipeline waits
 };
 
 __global__ void __launch_bounds__(THREADS, 1)
@@ -155,7 +157,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
-  uint32_t* tmem_slot = (uint32_t*)(tempty + 2);
+  uint64_t* drain = tempty + 2;                 // MMA completion after a failed wait
+  uint32_t* tmem_slot = (uint32_t*)(drain + 1);
   int32_t* c_term = (int32_t*)(tmem_slot + 4);  // [BN] per-column constant
   int32_t* c_m0 = c_term + BN;                   // [BN]
   int32_t* c_sh = c_m0 + BN;                     // [BN]
@@ -172,6 +175,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&tfull[b], 1);
       mbar_init(&tempty[b], 4);
     }
+    mbar_init(drain, 1);
     fence_mbar_init();
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
@@ -190,20 +194,29 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
+      uint32_t issued = 0, last_ph = 0;  // per slot: loads issued, parity of the last issue
       for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
         const int tm = t % tiles_m, tn = t / tiles_m;
         for (int kb = 0; kb < num_kb; ++kb) {
-          if (!mbar_poll(&empty[stage], phase ^ 1, status)) goto producer_done;
-          mbar_arrive_expect_tx(&full[stage], A_STAGE + B_STAGE);
-          tma_load_2d(sA + stage * A_STAGE, &tmA, kb * BK, tm * BM, &full[stage]);
-          tma_load_2d(sB + stage * B_STAGE, &tmB, kb * BK, tn * BN, &full[stage]);
+          if (!mbar_poll(&empty[stage], phase ^ 1, status, ep.spin)) goto producer_done;
+          if (!(ep.stall && t == (int)blockIdx.x && kb == 1)) {
+            mbar_arrive_expect_tx(&full[stage], A_STAGE + B_STAGE);
+            tma_load_2d(sA + stage * A_STAGE, &tmA, kb * BK, tm * BM, &full[stage]);
+            tma_load_2d(sB + stage * B_STAGE, &tmB, kb * BK, tn * BN, &full[stage]);
+            issued |= 1u << stage;
+            last_ph = (last_ph & ~(1u << stage)) | (phase << stage);
+          }
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
           }
         }
       }
-    producer_done:;
+    producer_done:
+      // every copy this thread issued has landed before the CTA may exit
+      // (after a normal run these phases completed long ago)
+      for (int st = 0; st < STAGES; ++st)
+        if ((issued >> st) & 1u) mbar_poll(&full[st], (last_ph >> st) & 1u, status);
     }
   } else if (warp == 1) {
     // ------------------------- MMA issuer -------------------------
@@ -211,14 +224,21 @@ __global__ void __launch_bounds__(THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       int local = 0;
-      for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++local) {
+      bool failed = false;
+      for (int t = blockIdx.x; t < tiles && !failed; t += gridDim.x, ++local) {
         const int buf = local & 1;
         const uint32_t use = (uint32_t)(local >> 1);
-        if (!mbar_poll(&tempty[buf], (use & 1) ^ 1, status)) goto mma_done;
+        if (!mbar_poll(&tempty[buf], (use & 1) ^ 1, status, ep.spin)) {
+          failed = true;
+          break;
+        }
         tc_fence_after();
         const uint32_t d = tmem_base + (uint32_t)(buf * BN);
         for (int kb = 0; kb < num_kb; ++kb) {
-          if (!mbar_poll(&full[stage], phase, status)) goto mma_done;
+          if (!mbar_poll(&full[stage], phase, status, ep.spin)) {
+            failed = true;
+            break;
+          }
           tc_fence_after();
           const uint32_t a0 = smem_u32(sA + stage * A_STAGE);
           const uint32_t b0 = smem_u32(sB + stage * B_STAGE);
@@ -232,9 +252,13 @@ __global__ void __launch_bounds__(THREADS, 1)
             phase ^= 1;
           }
         }
-        mma_commit(&tfull[buf]);  // accumulator ready for the epilogue
+        if (!failed) mma_commit(&tfull[buf]);  // accumulator ready for the epilogue
       }
-    mma_done:;
+      if (failed) {
+        // MMAs already issued finish before TMEM is freed
+        mma_commit(drain);
+        mbar_poll(drain, 0, status);
+      }
     }
   } else {
     // ------------------------- epilogue -------------------------
@@ -262,7 +286,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int m = tm * BM + row_in_tile;
       const bool row_ok = m < ep.M;
       const int32_t r_term = (ep.rowsum && row_ok) ? -ep.zb * ep.rowsum[m] : 0;
-      const bool ok = epi_bar_and(mbar_wait(&tfull[buf], use & 1, status));
+      const bool ok = epi_bar_and(mbar_wait(&tfull[buf], use & 1, status, ep.spin));
       tc_fence_after();
       if (ok) {
         for (int ch = 0; ch < BN / 32; ++ch) {
@@ -525,7 +549,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int m = tm * 256 + (int)rank * BM + row_in_tile;
       const bool row_ok = m < ep.M;
       const int32_t r_term = (ep.rowsum && row_ok) ? -ep.zb * ep.rowsum[m] : 0;
-      const bool ok = epi_bar_and(mbar_wait(&tfull[buf], use & 1, status));
+      const bool ok = epi_bar_and(mbar_wait(&tfull[buf], use & 1, status, ep.spin));
       tc_fence_after();
       if (ok) {
         for (int ch = 0; ch < BN / 32; ++ch) {
@@ -873,6 +897,8 @@ int i8gemm_run_packed(int M, int N, int K, const int8_t* A, int64_t lda, const v
   ep.m0v = rq.multiplier; ep.shv = rq.shift;
   ep.C = C; ep.ldc = ldc; ep.acc_out = acc_out; ep.ld_acc = ld_acc;
   const int num_kb = (int)(d.Kp / BK);
+  ep.stall = (M <= BM && num_kb > 1 && take_stall(kStallInt8Gemm)) ? 1 : 0;
+  ep.spin = ep.stall ? kStallSpinLimit : kSpinLimit;
   if (pair_path) {
     // 2-CTA pairs on 256 x 256 tiles, one resident pair per SM pair
     const int tiles_m = (int)cdiv(M, 256), tiles_n = (int)cdiv(N, BN);

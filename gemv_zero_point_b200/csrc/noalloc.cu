@@ -9,11 +9,16 @@
 // memory that the library declares itself.  Every GPU that loads the library
 // holds that array (kScratchBytes) until the process exits.
 //
-// The arithmetic is exactly that of qgemm_a8w4_f32: the same kernels run,
-// only the scratch comes from the array instead of the caller's workspace.
+// The arithmetic is that of qgemm_a8w4_f32, and the results agree with it
+// within the A8W4 tolerance.  M == 1 runs the same fused GEMV (its scratch
+// lives in shared memory, so the array is not touched).  M > 1 always runs
+// the CUDA-core GEMM on activations quantized into the array, where the
+// workspace entry point may take the tensor-core kernel instead; the two
+// combine the same exact group dots in a different float order.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "qg_internal.cuh"
@@ -45,27 +50,32 @@ constexpr int kSimtMaxK = 25600;
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kScratchBytes];
 
 // The host-side name g_noalloc_scratch is only a stand-in for the symbol; the
-// kernels need its device address, looked up once per device.
+// kernels need its device address, looked up once per device (with that
+// device current) and published with release/acquire ordering, so a thread
+// that sees the pointer also sees the completed lookup.
 constexpr int kMaxDevices = 64;
-uint8_t* g_scratch_ptr[kMaxDevices] = {nullptr};
+std::atomic<uint8_t*> g_scratch_ptr[kMaxDevices];
 std::mutex g_scratch_mu;
 
 int scratch_for_current_device(uint8_t** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return QG_ERR_NO_DEVICE;
-  if (!g_scratch_ptr[dev]) {
+  uint8_t* p = g_scratch_ptr[dev].load(std::memory_order_acquire);
+  if (!p) {
     std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (!g_scratch_ptr[dev]) {
-      void* p = nullptr;
-      cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-      if (e != cudaSuccess || !p) {
+    p = g_scratch_ptr[dev].load(std::memory_order_relaxed);
+    if (!p) {
+      void* sym = nullptr;
+      cudaError_t e = cudaGetSymbolAddress(&sym, g_noalloc_scratch);
+      if (e != cudaSuccess || !sym) {
         cudaGetLastError();
         return QG_ERR_CUDA;
       }
-      g_scratch_ptr[dev] = static_cast<uint8_t*>(p);
+      p = static_cast<uint8_t*>(sym);
+      g_scratch_ptr[dev].store(p, std::memory_order_release);
     }
   }
-  *out = g_scratch_ptr[dev];
+  *out = p;
   return QG_OK;
 }
 

@@ -77,10 +77,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Wait for phase `parity` of `bar` to complete, at most kSpinLimit polls.
+// Wait for phase `parity` of `bar` to complete, at most `limit` polls.
 // Returns false (after recording QG_ERR_TIMEOUT) if it never completed.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status) {
-  for (uint32_t i = 0; i < kSpinLimit; ++i) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status,
+                                          uint32_t limit = kSpinLimit) {
+  for (uint32_t i = 0; i < limit; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
   }
   record_error(status, QG_ERR_TIMEOUT);
@@ -102,13 +103,22 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-__device__ __forceinline__ bool mbar_poll(uint64_t* bar, uint32_t parity, int* status) {
-  for (uint32_t i = 0; i < (kSpinLimit << 4); ++i) {
+__device__ __forceinline__ bool mbar_poll(uint64_t* bar, uint32_t parity, int* status,
+                                          uint32_t limit = kSpinLimit) {
+  for (uint32_t i = 0; i < (limit << 4); ++i) {
     if (mbar_test(bar, parity)) return true;
   }
   record_error(status, QG_ERR_TIMEOUT);
   return false;
 }
+
+// Test hook (qg_test_arm_stall): which kernel family the next launch should
+// stall, consumed by that launch.  Kernels given a stall skip one pipeline
+// stage and wait with kStallSpinLimit polls, so their bounded waits run out
+// quickly.
+enum StallTarget { kStallNone = 0, kStallInt8Gemm = 1, kStallA8W4TC = 2 };
+bool take_stall(int target);  // true once after qg_test_arm_stall(target)
+constexpr uint32_t kStallSpinLimit = 1u << 12;
 
 // ---------------------------------------------------------------------------
 // Bulk copies (TMA engine)

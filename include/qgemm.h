@@ -66,6 +66,27 @@ int qg_version(void);
  */
 int qg_device_status(int reset);
 
+/*
+ * Test hook for the bounded waits; the pages have no counterpart.  Every
+ * pipeline wait in the tensor-core kernels gives up after a poll limit,
+ * records QG_ERR_TIMEOUT in the device status word and lets the kernel
+ * return (it first waits for its own copies and MMAs in flight and frees its
+ * tensor memory), so a stalled pipeline never hangs the GPU.  This arms one
+ * stall for the next launch of a kernel family, so that path can be
+ * exercised on purpose: that launch skips one pipeline stage (nothing is
+ * issued for it, so no copy is left in flight) and waits with a short poll
+ * limit.  The call itself still returns QG_OK; qg_device_status() then
+ * reports QG_ERR_TIMEOUT, the call's outputs are unspecified, and the next
+ * call runs normally.
+ *   which: 1 = INT8 GEMM one-CTA kernel (a call with M <= 128 and K > 128),
+ *          2 = A8W4 tensor-core kernel (an M > 1 call that takes it),
+ *          0 = disarm.
+ * Returns QG_OK, or QG_ERR_INVALID_ARG for another value.  Not for
+ * production use: one process-wide flag, taken by whichever thread launches
+ * that kernel family next.
+ */
+int qg_test_arm_stall(int which);
+
 /* ------------------------------------------------------------------------
  * Requantization parameters of the affine INT8 contract.
  *
@@ -365,12 +386,16 @@ int qconv2d_f32_dyn_a8w4(int Nb, int H, int W, int Cin, int Cout, int KH, int KW
  * exposes none, or a serving loop that must not call cudaMalloc after
  * start-up because it can synchronise the device.
  *
- * Same arguments and results as qgemm_a8w4_f32 (without the optional
- * quantization outputs).  The scratch (per-row int8 activations, scales and
+ * Same arguments as qgemm_a8w4_f32 (without the optional quantization
+ * outputs), and the same results within the A8W4 tolerance: M == 1 runs the
+ * same fused GEMV; M > 1 always runs the CUDA-core GEMM (qgemm_a8w4_f32 may
+ * take the tensor-core kernel there, which adds the same exact group dots in
+ * another float order).  The scratch (per-row int8 activations, scales and
  * zero-points) lives in a fixed array in device global memory owned by the
  * library: 4 MiB + 64 KiB, held on every GPU that loads the library until
- * the process exits.  Limits: M <= 8192 and M*K <= 4194304 when M > 1;
- * larger calls return QG_ERR_WORKSPACE and launch nothing.  It never calls
+ * the process exits.  Limits when M > 1: M <= 8192 and M*K <= 4194304, else
+ * QG_ERR_WORKSPACE; K <= 25600, else QG_ERR_UNSUPPORTED (8 rows of codes
+ * sit in shared memory).  A rejected call launches nothing.  It never calls
  * cudaMalloc/cudaFree or any allocating routine.
  *
  * The first call on each device looks up the array's device address

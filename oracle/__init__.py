@@ -25,8 +25,15 @@ Sources (web pages), cited by title and section:
          float im2col path, tileSplitFunction (QuanPostTreatParameters).
   [KAI]  pytorch/ao PR #997 "Kleidi 4b blockwise gemv prototype".
 
-Readings where the pages are silent are named R1..R16 here and listed with
-their justification in the design notes.
+Where the pages are silent the oracle takes the plainest reading and names
+it R1..R16 at the function that uses it, stating the reading in that
+function's docstring or the comment above it: R1 requant rounding (one
+round-half-even on the exact 64-bit product), R2 bias in accumulator scale
+added once after all of K, R5 min/max dynamic quantization in float32 with
+one rounding per operation, R6 the packed int4 layout, R8 clamp after bias,
+R12 bf16 scales rounded to nearest even, R13 one activation block per 32-wide
+weight group, R14 an f32 zero per weight group, R15 absolute-maximum
+symmetric quantization, R16 the unrolled float input of the dynamic conv.
 
 Parity pins: every function below is pinned by tests in
 ``tests/test_oracle_pins.py`` against the pages' printed numbers, closed
@@ -139,6 +146,38 @@ def int8_gemm_acc(A, B, za, zb, bias=None):
     if bias is not None:
         acc = acc + np.asarray(bias, dtype=np.int64)[None, :]
     return acc
+
+
+F64_EXACT_LIMIT = 2 ** 53  # every integer of magnitude <= 2^53 is a float64
+
+
+def int8_gemm_acc_f64(A, B, za, zb, bias=None, row_block=1024):
+    """The accumulator of int8_gemm_acc computed with a float64 matrix
+    product, for sizes where the int64 product is too slow to check every
+    output.
+
+    Each factor (A[m,k]-za)(B[k,n]-zb) is an integer of magnitude at most
+    255*255 = 65025 ([QG] section 4), so every partial sum of any summation
+    order has magnitude at most K*65025.  While K*65025 <= 2^53 each partial
+    sum is an integer that float64 represents, every addition is exact, and
+    the product equals the int64 definition whatever blocking the BLAS
+    routine uses.  Larger K is refused.  Returns int64 [M, N], bias added in
+    int64 after the product (R2).
+    """
+    A = np.asarray(A)
+    B = np.asarray(B)
+    K = A.shape[1]
+    if K * worst_zp_corrected_magnitude() ** 2 > F64_EXACT_LIMIT:
+        raise ValueError("K too large for an exact float64 accumulation")
+    Bf = B.astype(np.float64) - float(zb)
+    blocks = [np.zeros((0, B.shape[1]), np.int64)]
+    for r0 in range(0, A.shape[0], row_block):
+        Af = A[r0:r0 + row_block].astype(np.float64) - float(za)
+        blocks.append((Af @ Bf).astype(np.int64))
+    out = np.concatenate(blocks)
+    if bias is not None:
+        out += np.asarray(bias, dtype=np.int64)[None, :]
+    return out
 
 
 def qgemm_s8s8_requant(A, B, za, zb, bias, m0, shift, out_zp, clamp_min,

@@ -1,30 +1,24 @@
 """GPU parity of the A8W4 path against the CPU oracle, through the C ABI.
 
 Quantized activations (q, scale, zero-point) and packed weights must match
-bit-exactly; f32 outputs within |y - y_ref| <= 1e-4 * max(|y_ref|, 1)
-(relative 1e-4 for |y| >= 1, absolute 1e-4 below; see the tolerance reading
-in the design notes)."""
+bit-exactly.  f32 outputs must satisfy |y - y_ref| <= 1e-4 * max(|y_ref|, 1)
+against the float64 oracle: relative 1e-4 where |y| >= 1, absolute 1e-4
+below, because the float32 rounding of a sum of group terms is set by the
+size of the terms, not of y (tests/a8w4_tol.py; the observed errors are
+printed at the end of the run)."""
 import numpy as np
 import pytest
 
 import oracle
 import workloads
+from a8w4_tol import assert_a8w4_close
 
 pytestmark = pytest.mark.gpu
 torch = pytest.importorskip("torch")
 
-TOL = 1e-4
-
 
 def _dev(a):
     return torch.from_numpy(np.ascontiguousarray(a)).cuda()
-
-
-def assert_a8w4_close(y, y_ref):
-    err = np.abs(y.astype(np.float64) - y_ref.astype(np.float64)) / np.maximum(np.abs(y_ref), 1.0)
-    i = int(np.argmax(err))
-    assert err.flat[i] <= TOL, f"max err {err.flat[i]:.3e} at {np.unravel_index(i, y.shape)}: " \
-                               f"{y.flat[i]} vs {y_ref.flat[i]}"
 
 
 @pytest.fixture(autouse=True)
@@ -126,7 +120,9 @@ def _check_a8w4(lib, w, bf16=False, **kw):
     np.testing.assert_array_equal(q, q_ref)
     np.testing.assert_array_equal(s.view(np.int32), s_ref.view(np.int32))
     np.testing.assert_array_equal(z, z_ref)
-    assert_a8w4_close(y, y_ref)
+    M, N, K = w["M"], w["N"], w["K"]
+    kind = "gemv" if M == 1 else ("tc" if K % 128 == 0 and N % 4 == 0 else "simt")
+    assert_a8w4_close(y, y_ref, f"a8w4{'_bf16s' if bf16 else ''} {kind} {M}x{N}x{K}")
     return y, y_ref
 
 
@@ -184,7 +180,7 @@ def test_gemv_chain_on_one_stream(lib):
         y_ref = oracle.qgemm_a8w4_f32(xin, w["qw"], w["sw"], w["bias"], w["clamp_min"],
                                       w["clamp_max"])[0]
         y_np = y.cpu().numpy()
-        assert_a8w4_close(y_np, y_ref)
+        assert_a8w4_close(y_np, y_ref, "a8w4 gemv chain")
         xin = y_np
 
 
@@ -242,7 +238,7 @@ def _check_actblock(lib, w):
     np.testing.assert_array_equal(z.cpu().numpy(), z_ref[0])
     y_np = y.cpu().numpy()
     assert (y_np[:, N:] == 7.0).all()
-    assert_a8w4_close(y_np[:, :N], y_ref)
+    assert_a8w4_close(y_np[:, :N], y_ref, f"actblock 1x{N}x{K}")
 
 
 def test_gemv_actblock_full_size_1x14336x4096(lib):
@@ -300,7 +296,7 @@ def _check_asym(lib, w, zw):
     np.testing.assert_array_equal(z.cpu().numpy(), z_ref)
     y_np = y.cpu().numpy()
     assert (y_np[:, N:] == 7.0).all()
-    assert_a8w4_close(y_np[:, :N], y_ref)
+    assert_a8w4_close(y_np[:, :N], y_ref, f"asym 1x{N}x{K}")
 
 
 def test_gemv_asym_full_size_1x14336x4096(lib):

@@ -3,28 +3,21 @@ convolution (unrolled rows quantized per output pixel, int4 weights) against
 the CPU oracle, through the C ABI.
 
 Quantized rows (codes, scales, zero-points) must match bit-exactly; f32
-outputs within |y - y_ref| <= 1e-4 * max(|y_ref|, 1), as the A8W4 linear."""
+outputs within |y - y_ref| <= 1e-4 * max(|y_ref|, 1), as the A8W4 linear
+(tests/a8w4_tol.py)."""
 import numpy as np
 import pytest
 
 import oracle
 import workloads
+from a8w4_tol import assert_a8w4_close
 
 pytestmark = pytest.mark.gpu
 torch = pytest.importorskip("torch")
 
-TOL = 1e-4
-
 
 def _dev(a):
     return torch.from_numpy(np.ascontiguousarray(a)).cuda()
-
-
-def _assert_close(y, y_ref):
-    err = np.abs(y.astype(np.float64) - y_ref.astype(np.float64)) / np.maximum(np.abs(y_ref), 1.0)
-    i = int(np.argmax(err))
-    assert err.flat[i] <= TOL, f"max err {err.flat[i]:.3e} at {np.unravel_index(i, y.shape)}: " \
-                               f"{y.flat[i]} vs {y_ref.flat[i]}"
 
 
 @pytest.fixture(autouse=True)
@@ -79,7 +72,9 @@ def _run_dynconv(lib, w, symmetric):
     np.testing.assert_array_equal(q.cpu().numpy(), q_ref)
     np.testing.assert_array_equal(s.cpu().numpy().view(np.int32), s_ref.view(np.int32))
     np.testing.assert_array_equal(z.cpu().numpy(), z_ref)
-    _assert_close(y.cpu().numpy(), y_ref)
+    assert_a8w4_close(y.cpu().numpy(), y_ref,
+                      f"dynconv {'sym' if symmetric else 'asym'} {Nb}x{H}x{W}x{Cin}->{Cout} "
+                      f"{KH}x{KW}")
     return y_ref
 
 

@@ -140,11 +140,33 @@ def test_gemm_deterministic(lib):
 
 
 def test_gemm_8192x8192x8200_sampled_rows(lib):
+    # direct int64 definition on rows at tile edges (the full check below
+    # goes through the exact float64 route)
     w = workloads.int8_gemm_8192x8192x8200()
     rows = np.array([0, 1, 127, 128, 129, 2047, 4096, 5000, 8063, 8064, 8190, 8191])
     C, C_ref = check_gemm(lib, w, packed=True, rows=rows)
     # every column of the sampled rows is checked; outputs are not all saturated
     assert np.mean(np.abs(C_ref.astype(int)) < 127) > 0.05
+
+
+@pytest.mark.parametrize("packed", [True, False])
+def test_gemm_8192x8192x8200_every_output(lib, packed):
+    """All 67,108,864 outputs (int8 C and the int32 accumulators) of the
+    8192x8192x8200 GEMM against the oracle's exact float64 accumulation
+    (pinned to the int64 definition on the CPU) and its requantization.
+    packed=True is the weights-stationary call the benchmark times."""
+    w = workloads.int8_gemm_8192x8192x8200()
+    C, acc, m0, sh = run_gemm(lib, w, packed=packed)
+    K, N = w["K"], w["N"]
+    B = w["B"][:, :N]
+    for r0 in range(0, w["M"], 2048):
+        rows = slice(r0, r0 + 2048)
+        acc_ref = oracle.int8_gemm_acc_f64(w["A"][rows, :K], B, w["za"], w["zb"], w["bias"])
+        bad = np.argwhere(acc[rows] != acc_ref)
+        assert bad.size == 0, f"first accumulator mismatch at row {r0 + bad[0][0]}, col {bad[0][1]}"
+        C_ref = oracle.requantize(acc_ref, m0, sh, w["out_zp"], w["clamp_min"], w["clamp_max"])
+        bad = np.argwhere(C[rows] != C_ref)
+        assert bad.size == 0, f"first output mismatch at row {r0 + bad[0][0]}, col {bad[0][1]}"
 
 
 # ---------------------------------------------------------------------------

@@ -72,6 +72,18 @@ CASES = {
     "output zero-point dropped": (
         "y = np.clip(q + int(out_zp),", "y = np.clip(q,", None,
         [("test_requant_round_half_even_cases", {})]),
+    "float64 route drops the activation zero-point": (
+        "Af = A[r0:r0 + row_block].astype(np.float64) - float(za)",
+        "Af = A[r0:r0 + row_block].astype(np.float64)", None,
+        [("test_p5_float64_accumulation_is_exact_against_int64_loops", {})]),
+    "float64 route in float32": (
+        "blocks.append((Af @ Bf).astype(np.int64))",
+        "blocks.append((Af.astype(np.float32) @ Bf.astype(np.float32)).astype(np.int64))",
+        None, [("test_p5_float64_accumulation_is_exact_against_int64_loops", {})]),
+    "float64 route skips the last row block": (
+        "for r0 in range(0, A.shape[0], row_block):",
+        "for r0 in range(0, A.shape[0] - row_block, row_block):", None,
+        [("test_p5_float64_accumulation_is_exact_against_int64_loops", {})]),
     "weight zero-point dropped": (
         "B = np.asarray(B, dtype=np.int64) - int(zb)", "B = np.asarray(B, dtype=np.int64)", None,
         [("test_p5_float_dequant_reference", {})]),

@@ -188,6 +188,43 @@ def test_p5_gemm_brute_force_loops():
     np.testing.assert_array_equal(oracle.int8_gemm_acc(A, B, za, zb, bias), np.array(ref))
 
 
+def test_p5_float64_accumulation_is_exact_against_int64_loops():
+    # The float64 route equals the int64 definition on random blocks with
+    # several row blocks, zero-points and a bias, and on the all-worst-case
+    # operands at K = 8200, where every product is -65025 and the sum reaches
+    # -533,205,000: far past float32's exact range (2^24), inside float64's.
+    rng = np.random.default_rng(21)
+    for M, N, K, za, zb in [(37, 29, 8200, 7, 0), (300, 64, 1000, -20, 13), (5, 3, 1, 0, 0)]:
+        A = rng.integers(-128, 128, (M, K)).astype(np.int8)
+        B = rng.integers(-128, 128, (K, N)).astype(np.int8)
+        bias = rng.integers(-5000, 5001, N).astype(np.int32)
+        ref = oracle.int8_gemm_acc(A, B, za, zb, bias)
+        np.testing.assert_array_equal(oracle.int8_gemm_acc_f64(A, B, za, zb, bias, row_block=16),
+                                      ref)
+    K = 8200
+    A = np.full((3, K), 127, np.int8)
+    B = np.full((K, 4), -128, np.int8)
+    acc = oracle.int8_gemm_acc_f64(A, B, za=-128, zb=127)
+    assert (acc == -K * 65025).all()
+    # that sum is not a float32 value: an accumulation in float32 would fail here
+    assert int(np.float32(K * 65025)) != K * 65025
+    # a few brute-force entries with plain Python integers
+    A = rng.integers(-128, 128, (4, 50)).astype(np.int8)
+    B = rng.integers(-128, 128, (50, 6)).astype(np.int8)
+    f = oracle.int8_gemm_acc_f64(A, B, 3, -5)
+    for m in range(4):
+        for n in range(6):
+            assert f[m, n] == sum((int(A[m, k]) - 3) * (int(B[k, n]) + 5) for k in range(50))
+
+
+def test_p5_float64_accumulation_refuses_k_past_the_exact_range():
+    K = 2 ** 53 // 65025 + 1
+    A = np.broadcast_to(np.int8(0), (1, K))        # views: nothing of size K is allocated
+    B = np.broadcast_to(np.int8(0), (K, 1))
+    with pytest.raises(ValueError):
+        oracle.int8_gemm_acc_f64(A, B, 0, 0)
+
+
 def test_p5_float_dequant_reference():
     w = workloads.int8_gemm(37, 23, 129, seed=5)
     A, B = w["A"], w["B"]
