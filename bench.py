@@ -15,10 +15,14 @@ Timing: W untimed warm-up steps, then exactly K steps bracketed by a barrier
 and cudaDeviceSynchronize on both sides, CUDA events on the launching stream,
 max over ranks.  The K timed steps (C-ABI calls) are captured once into a
 CUDA graph and replayed, so Python/ctypes launch cost stays out of the kernel
-numbers; per-kernel times come from graphs of K back-to-back calls of each
-part.  The end-to-end leg is eager, one API call at a time.  L2 (126 MB) is defeated by rotating input sets larger than
-it: 2 GEMM sets (A + packed B = 135 MB each) and 8 GEMV weight sets (36.8 MB
-each, 295 MB in all).
+numbers.  Per-call and per-kernel times come from graphs of back-to-back
+calls of one part lasting at least 8 ms (up to 200 calls, at least K),
+replayed 5 times after idle pauses, median reported: graph start-up is spread
+over hundreds of the microsecond calls whatever K is, and each replay is a
+burst, not a power-capped loop.  The end-to-end leg is eager, one API call at
+a time.  L2 (126 MB) is defeated by rotating input sets larger than it: 2
+GEMM sets (A + packed B = 135 MB each) and 8 GEMV weight sets (36.8 MB each,
+295 MB in all).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
                   [--workload headline|<one workload name below>] [--no-cpu-baseline]
@@ -36,6 +40,7 @@ from __future__ import annotations
 
 import argparse
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -53,8 +58,9 @@ PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 INT8_OVER_BF16 = 2.0  # nominal dense ratio (4.5 POPS int8 vs 2.25 PFLOPS bf16)
 NOMINAL_INT8_TOPS = 4500.0  # B200 dense int8 spec figure, reported beside the measured-derived peak
-PART_CALLS = 200     # calls per per-part timing graph, whatever --steps is
-PART_REPLAYS = 5     # replays per per-part graph (median reported)
+PART_CALLS = 200     # most calls per per-part timing graph
+PART_GRAPH_MS = 8.0  # a per-part graph lasts at least this long (or PART_CALLS calls)
+PART_REPLAYS = 5     # replays per per-part graph, each after an idle pause (median reported)
 
 
 def load_peaks():
@@ -822,20 +828,26 @@ def main():
         return g
 
     def part_ms(fn):
-        """Median per-call time of a graph of PART_CALLS back-to-back calls
-        (independent of --steps, so graph start-up is spread over as many
-        calls as a long run has), over at least PART_REPLAYS replays, with
-        the clocks sampled while they run."""
-        n = max(PART_CALLS, args.steps)
+        """Median per-call time of a call timed alone.  The graph holds enough
+        back-to-back calls to last PART_GRAPH_MS (at least --steps calls, at
+        most PART_CALLS), so graph start-up is spread over hundreds of short
+        calls whatever --steps is; it is replayed PART_REPLAYS times, each
+        replay after an idle pause so every replay is a burst (a kernel timed
+        alone) rather than a power-capped loop; clocks are sampled meanwhile."""
+        probe = capture_n([fn], 10)
+        probe.replay()
+        torch.cuda.synchronize()
+        call_ms = replay_ms(probe) / 10
+        del probe
+        n = max(args.steps, min(PART_CALLS, int(math.ceil(PART_GRAPH_MS / max(call_ms, 1e-4)))))
         g = capture_n([fn], n)
         g.replay()
         torch.cuda.synchronize()
-        time.sleep(0.5)
         clk = Clocks(dist.local)
         clk.start()
-        time.sleep(0.1)
-        times, t_end = [], time.perf_counter() + 0.3
-        while len(times) < PART_REPLAYS or (time.perf_counter() < t_end and len(times) < 50):
+        times = []
+        for _ in range(PART_REPLAYS):
+            time.sleep(0.2)
             times.append(dist.max(replay_ms(g)) / n)
         c = clk.stop()
         del g
@@ -923,9 +935,12 @@ def main():
             part["frac_of_int8_peak"] = part["TOPS"] / tensor_peak_tops
             part["frac_of_int8_peak_burst"] = part["TOPS"] / tensor_peak_burst
             part["frac_of_int8_peak_sustained"] = part["TOPS"] / tensor_peak_sust
-            # The kernel alone is timed after an idle pause over steps*kernel_ms
-            # (well under a second): the burst figure is its fair peak.
-            k_sust = kernel_ms[j] * args.steps > 1000.0
+            # The kernel alone is timed in bursts after idle pauses: the burst
+            # figure is its fair peak, unless the power limiter still showed
+            # while it ran.
+            kt_info = kernel_timing[j] or part_timing[j]
+            k_clk = (kt_info or {}).get("clocks") or {}
+            k_sust = "sw_power_cap" in k_clk.get("reasons", [])
             k_peak = tensor_peak_sust if k_sust else tensor_peak_burst
             part["frac_of_nominal_int8"] = part["TOPS"] / NOMINAL_INT8_TOPS
             rooflines[name] = {"bound": "tensor", "achieved": kt, "peak": k_peak,
