@@ -281,8 +281,8 @@ class A8W4Case:
         self.M, self.N, self.K = w["M"], w["N"], w["K"]
         self.qg, self.torch = qg, torch
         self.bf16 = bf16_scales
-        self.actblock = actblock  # activations quantized per 32-wide K block (M = 1)
-        self.asym = asym          # asymmetric int4 weights: an f32 zero per group (M = 1)
+        self.actblock = actblock  # activations quantized per 32-wide K block
+        self.asym = asym          # asymmetric int4 weights: an f32 zero per group
         qw = dev(w["qw"], torch)
         sw = dev(w["sw"], torch)
         self.packed = []
@@ -310,11 +310,13 @@ class A8W4Case:
     def run(self, i, stream=None):
         if self.asym:
             self.qg.qgemm_a8w4_f32_asym(self.x, self.packed[i % len(self.packed)], self.N,
-                                        self.bias, self.lo, self.hi, self.y, stream=stream)
+                                        self.bias, self.lo, self.hi, self.y, workspace=self.ws,
+                                        stream=stream)
             return
         if self.actblock:
             self.qg.qgemm_a8w4_f32_actblock(self.x, self.packed[i % len(self.packed)], self.N,
-                                            self.bias, self.lo, self.hi, self.y, stream=stream)
+                                            self.bias, self.lo, self.hi, self.y,
+                                            workspace=self.ws, stream=stream)
             return
         self.qg.qgemm_a8w4_f32(self.x, self.packed[i % len(self.packed)], self.N, self.bias,
                                self.lo, self.hi, self.y, workspace=self.ws, stream=stream,
@@ -327,10 +329,10 @@ class A8W4Case:
         self.e2e_x.copy_(self.h2d_host, non_blocking=True)
         if self.asym:
             self.qg.qgemm_a8w4_f32_asym(self.e2e_x, self.packed[0], self.N, self.bias, self.lo,
-                                        self.hi, self.y)
+                                        self.hi, self.y, workspace=self.ws)
         elif self.actblock:
             self.qg.qgemm_a8w4_f32_actblock(self.e2e_x, self.packed[0], self.N, self.bias,
-                                            self.lo, self.hi, self.y)
+                                            self.lo, self.hi, self.y, workspace=self.ws)
         else:
             self.qg.qgemm_a8w4_f32(self.e2e_x, self.packed[0], self.N, self.bias, self.lo,
                                    self.hi, self.y, workspace=self.ws, bf16_scales=self.bf16)
@@ -459,6 +461,7 @@ class DynConvCase:
 WORKLOAD_NAMES = ["headline", "int8_gemm_130x70x129", "int8_conv_56x56x64_3x3",
                   "a8w4_gemv_1x14336x4096", "a8w4_gemv_bf16s_1x14336x4096",
                   "a8w4_gemv_actblock_1x14336x4096", "a8w4_gemv_asym_1x14336x4096",
+                  "a8w4_gemm_actblock_128x4096x4096", "a8w4_gemm_asym_128x4096x4096",
                   "a8w4_gemm_128x4096x4096", "int8_gemm_8192x8192x8200",
                   "a8w4_conv_f32_56x56x64_3x3", "a8w4_conv_f32_sym_56x56x64_3x3"]
 
@@ -479,6 +482,12 @@ def build_cases(workload, qg, torch):
     if workload == "a8w4_gemv_asym_1x14336x4096":   # asymmetric int4 weights (44 MB per set)
         return [("a8w4_gemv_asym_1x14336x4096",
                  A8W4Case(qg, torch, W.a8w4_gemv_1x14336x4096(), 7, asym=True), "hbm")]
+    if workload == "a8w4_gemm_actblock_128x4096x4096":
+        return [("a8w4_gemm_actblock_128x4096x4096",
+                 A8W4Case(qg, torch, W.a8w4_gemm_128x4096x4096(), 16, actblock=True), "hbm")]
+    if workload == "a8w4_gemm_asym_128x4096x4096":
+        return [("a8w4_gemm_asym_128x4096x4096",
+                 A8W4Case(qg, torch, W.a8w4_gemm_128x4096x4096(), 12, asym=True), "hbm")]
     if workload == "a8w4_gemv_actblock_1x14336x4096":   # activations quantized per K block
         return [("a8w4_gemv_actblock_1x14336x4096",
                  A8W4Case(qg, torch, W.a8w4_gemv_1x14336x4096(), 8, actblock=True), "hbm")]
@@ -505,6 +514,8 @@ KERNEL_SOURCES = {
     "a8w4_gemm_128x4096x4096": "a8w4_tc.cu",
     "a8w4_gemv_bf16s_1x14336x4096": "a8w4.cu",
     "a8w4_gemv_actblock_1x14336x4096": "a8w4.cu",
+    "a8w4_gemm_actblock_128x4096x4096": "a8w4_tc.cu",
+    "a8w4_gemm_asym_128x4096x4096": "a8w4_tc.cu",
     "a8w4_gemv_asym_1x14336x4096": "a8w4.cu",
     "a8w4_conv_f32_56x56x64_3x3": "a8w4.cu",
     "a8w4_conv_f32_sym_56x56x64_3x3": "a8w4.cu",
@@ -592,14 +603,21 @@ def oracle_sample(workload, budget_s=12.0, rows_gemm=None, small=False):
         tag = {"a8w4_gemv_bf16s_1x14336x4096": " (bf16 scales)",
                "a8w4_gemv_actblock_1x14336x4096": " (per-block activations)"}.get(workload, "")
         parts.append(f"A8W4 GEMV{tag} {n} of 14336 rows")
-    if workload == "a8w4_gemm_128x4096x4096":
+    if workload in ("a8w4_gemm_128x4096x4096", "a8w4_gemm_actblock_128x4096x4096",
+                    "a8w4_gemm_asym_128x4096x4096"):
         w = _inputs("a8w4_gemm_128x4096x4096")
         rows = 1 if small else 4
         t = time.perf_counter()
-        oracle.qgemm_a8w4_f32(w["x"][:rows], w["qw"], w["sw"], w["bias"], -6.0, 6.0)
+        if workload == "a8w4_gemm_asym_128x4096x4096":
+            zw = (w["sw"] * np.random.default_rng(77).uniform(-8, 8, w["sw"].shape)).astype(np.float32)
+            oracle.qgemm_a8w4_f32_asym(w["x"][:rows], w["qw"], w["sw"], zw, w["bias"], -6.0, 6.0)
+        elif workload == "a8w4_gemm_actblock_128x4096x4096":
+            oracle.qgemm_a8w4_f32_actblock(w["x"][:rows], w["qw"], w["sw"], w["bias"], -6.0, 6.0)
+        else:
+            oracle.qgemm_a8w4_f32(w["x"][:rows], w["qw"], w["sw"], w["bias"], -6.0, 6.0)
         dt = time.perf_counter() - t
         ops += a8w4_ops(rows, w["N"], w["K"]); spent += dt
-        parts.append(f"A8W4 GEMM {rows} of 128 rows")
+        parts.append(f"{workload.rsplit('_', 1)[0]} {rows} of 128 rows")
     if workload == "int8_gemm_130x70x129":
         w = _inputs("int8_gemm_130x70x129")
         m0, sh = oracle.requant_params(float(w["ratio"][0]))

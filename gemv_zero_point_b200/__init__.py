@@ -91,11 +91,11 @@ _sig("qgemm_a8w4_workspace_bytes", _sz, [_i32, _i32, _i32])
 _sig("qgemm_a8w4_f32", _i32, [_i32, _i32, _i32, _vp, _i64, _vp, _vp, _f32, _f32, _vp, _i64,
                               _vp, _vp, _vp, _vp, _sz, _vp])
 _sig("qgemm_a8w4_f32_actblock", _i32, [_i32, _i32, _i32, _vp, _i64, _vp, _vp, _f32, _f32, _vp,
-                                       _i64, _vp, _vp, _vp, _vp])
+                                       _i64, _vp, _vp, _vp, _vp, _sz, _vp])
 _sig("pack_w4_g32_asym_bytes", _sz, [_i32, _i32])
 _sig("pack_w4_g32_asym", _i32, [_i32, _i32, _vp, _i64, _vp, _vp, _vp, _sz, _vp])
 _sig("qgemm_a8w4_f32_asym", _i32, [_i32, _i32, _i32, _vp, _i64, _vp, _vp, _f32, _f32, _vp,
-                                   _i64, _vp, _vp, _vp, _vp])
+                                   _i64, _vp, _vp, _vp, _vp, _sz, _vp])
 _sig("quantize_rows_a8_sym", _i32, [_i32, _i32, _vp, _i64, _vp, _i64, _vp, _vp])
 _sig("qconv2d_f32_dyn_a8w4_workspace_bytes", _sz, [_i32] * 11)
 _sig("qconv2d_f32_dyn_a8w4", _i32, [_i32] * 11 + [_vp, _vp, _vp, _f32, _f32, _i32, _vp, _vp, _vp,
@@ -227,14 +227,24 @@ def qgemm_a8w4_f32(x, packed_w, N, bias, clamp_min, clamp_max, y, q_out=None, sc
               0 if workspace is None else workspace.numel(), _stream(stream)), fn.__name__)
 
 
+def _a8w4_workspace(M, N, K, workspace, device):
+    wsb = lib.qgemm_a8w4_workspace_bytes(M, N, K)
+    if wsb and workspace is None:
+        workspace = _empty_bytes(wsb, device)
+    return workspace
+
+
 def qgemm_a8w4_f32_actblock(x, packed_w, N, bias, clamp_min, clamp_max, y, q_out=None,
-                            scale_out=None, zp_out=None, stream=None):
-    """A8W4 GEMV (M = 1) with the activations quantized per 32-wide K block;
-    scale_out / zp_out, when given, receive K/32 values."""
+                            scale_out=None, zp_out=None, workspace=None, stream=None):
+    """A8W4 linear with the activations quantized per 32-wide K block;
+    scale_out / zp_out, when given, receive [M][K/32] values."""
     M, K = x.shape
+    workspace = _a8w4_workspace(M, N, K, workspace, x.device)
     _check(lib.qgemm_a8w4_f32_actblock(M, N, K, _p(x), _ld(x), _p(packed_w), _p(bias),
                                        float(clamp_min), float(clamp_max), _p(y), _ld(y),
-                                       _p(q_out), _p(scale_out), _p(zp_out), _stream(stream)),
+                                       _p(q_out), _p(scale_out), _p(zp_out), _p(workspace),
+                                       0 if workspace is None else workspace.numel(),
+                                       _stream(stream)),
            "qgemm_a8w4_f32_actblock")
 
 
@@ -249,12 +259,15 @@ def pack_w4_g32_asym(w, group_scales, group_zeros, packed=None, stream=None):
 
 
 def qgemm_a8w4_f32_asym(x, packed_w, N, bias, clamp_min, clamp_max, y, q_out=None,
-                        scale_out=None, zp_out=None, stream=None):
-    """A8W4 GEMV (M = 1) with asymmetric int4 weights (pack_w4_g32_asym)."""
+                        scale_out=None, zp_out=None, workspace=None, stream=None):
+    """A8W4 linear with asymmetric int4 weights (pack_w4_g32_asym)."""
     M, K = x.shape
+    workspace = _a8w4_workspace(M, N, K, workspace, x.device)
     _check(lib.qgemm_a8w4_f32_asym(M, N, K, _p(x), _ld(x), _p(packed_w), _p(bias),
                                    float(clamp_min), float(clamp_max), _p(y), _ld(y),
-                                   _p(q_out), _p(scale_out), _p(zp_out), _stream(stream)),
+                                   _p(q_out), _p(scale_out), _p(zp_out), _p(workspace),
+                                   0 if workspace is None else workspace.numel(),
+                                   _stream(stream)),
            "qgemm_a8w4_f32_asym")
 
 

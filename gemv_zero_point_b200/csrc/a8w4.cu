@@ -18,33 +18,6 @@
 
 namespace qg {
 
-// ---------------------------------------------------------------------------
-// Per-row quantization parameters (float32, one IEEE rounding per operation,
-// no contraction): rmin = min(0, min x), rmax = max(0, max x),
-// scale = (rmax-rmin)/255 (1 if 0), inv = 1/scale,
-// zp = clamp(rne(-128 - rmin*inv), -128, 127).
-// ---------------------------------------------------------------------------
-struct RowQuant {
-  float scale, inv;
-  int zp;
-};
-
-__device__ __forceinline__ RowQuant row_quant_params(float rmin, float rmax) {
-  RowQuant r;
-  float s = __fdiv_rn(__fsub_rn(rmax, rmin), 255.0f);
-  if (s == 0.0f) s = 1.0f;
-  r.scale = s;
-  r.inv = __fdiv_rn(1.0f, s);
-  float t = __fsub_rn(-128.0f, __fmul_rn(rmin, r.inv));
-  int z = __float2int_rn(t);
-  r.zp = min(max(z, -128), 127);
-  return r;
-}
-
-__device__ __forceinline__ int quant_one(float x, const RowQuant& r) {
-  int v = __float2int_rn(__fmul_rn(x, r.inv)) + r.zp;
-  return min(max(v, -128), 127);
-}
 
 // Block-wide min/max of one row (blockDim.x threads, multiple of 32, <= 1024).
 __device__ __forceinline__ void block_minmax(float& mn, float& mx, float* red /* [64] */) {

@@ -1,30 +1,51 @@
-// A8W4 linear for M > 1 on the 5th-generation tensor cores.
+// A8W4 linear for M > 1 on the 5th-generation tensor cores, and the same
+// contraction for the unrolled rows of the float-input convolution.
 //
-// Source: pytorch/ao PR #997 "Kleidi 4b blockwise gemv prototype"
+// Sources: pytorch/ao PR #997 "Kleidi 4b blockwise gemv prototype"
 // (matmul_clamp_f32_qai8dxp_qsi4c32p: int8 dynamic per-row asymmetric
-// activations, int4 symmetric weights with one f32 scale per 32-wide K group,
-// f32 output clamped after the bias; m > 1 tests).
+// activations, int4 symmetric weights with one scale per 32-wide K group,
+// f32 output clamped after the bias; m > 1 tests); MNN
+// ConvInt8TiledExecutor.cpp (dynamic-quant option 2: the input quantized per
+// K block; asymmetric weight quant info, w_real = alpha*code + zero; the
+// low-memory float im2col path, symmetric or asymmetric rows).
 //
-//   y[m,n] = clamp(sA[m] * sum_g sw[n,g] * I[m,n,g] + bias[n])
-//   I[m,n,g] = sum_{k in g} (qA[m,k] - zA[m]) * w[n,k]
+//   y[m,n] = clamp(sA[m] * sum_g (sw[n,g]*I[m,n,g] + zw[n,g]*S[m,g]) + bias[n])
+//   I[m,n,g] = sum_{k in g} (qA[m,k] - zA[m]) * w[n,k],  S[m,g] = sum_{k in g}(qA[m,k] - zA[m])
+// (zw = 0 for symmetric weights; with per-block activations sA and zA are
+// per (m, g) and sA moves inside the sum).
 //
-// Exactness: qA - zA lies in [-255,255] and w in [-8,7], both exact in bf16,
-// and every partial sum of one group is an integer below 2^24, so one
-// kind::f16 MMA pair (K = 2 x 16) per group leaves the exact I[m,n,g] in an
-// f32 TMEM accumulator.  Only the combination over groups is rounded (f32).
+// Exactness: qA - zA lies in [-255,255] and w in [-8,7], both exact in
+// bf16, and every partial sum of one group is an integer below 2^24, so the
+// two K = 16 bf16 MMAs of a group leave the exact I[m,n,g] in an f32 TMEM
+// accumulator.  Only the combination over groups is rounded (f32).
 //
-// Roles (448 threads, one CTA per SM, tile 128 x 128 over a K range):
-//   warp 0      TMA: the CTA's nibble slice once, then (after waiting for the
-//               quantization grid) bf16 A' stages (128 rows x 64 K, 128B
-//               swizzle)
-//   warp 1      TMEM allocation; MMA issue, one 128-column TMEM buffer per
-//               group, 4 buffers
-//   warps 2..5  expand nibbles into the swizzled bf16 B' stage
-//   warps 6..13 per group: tcgen05.ld the exact group dots, release the
-//               buffer, acc += sw * I with packed fma.rn.f32x2; then the
-//               split-K partial, and the last CTA of a tile reduces the
-//               partials in split order (deterministic) and writes y.
+// Two launches per call:
+//  1. a8w4_quant_tiles_kernel quantizes each activation row (per row or per
+//     32-wide block, asymmetric or symmetric; plain rows or the unrolled rows
+//     of an NHWC image) and writes the centred codes qA - zA as bf16 in the
+//     exact byte image the tensor cores read: for every 128-row tile and
+//     every 64-wide K block, 128 rows of 128 bytes with the 16-byte chunks of
+//     row r permuted by r % 8 (the 128-byte swizzle).  One stage of the GEMM
+//     is then one contiguous 16 KiB bulk copy.
+//  2. a8w4_tc_kernel (programmatic dependent launch after 1) computes a tile
+//     of 128 weight rows (MMA M, TMEM lanes) x 128 activation rows (MMA N,
+//     TMEM columns) over a K range; the K ranges of one tile form a cluster
+//     and their partial tiles are reduced through distributed shared memory
+//     in a fixed order.
+//
+// Roles of a8w4_tc_kernel (448 threads, one CTA per SM):
+//   warp 0      bulk copies of the activation stages (after the grid
+//               dependency wait)
+//   warp 1      TMEM allocation; MMA issue: per 32-wide group two K = 16
+//               MMAs into one of 4 rotating 128-column TMEM buffers
+//   warps 2..5  weight nibbles: a ring of 64-wide K slices of the CTA's 128
+//               rows (tensor copies, issued before the grid dependency wait),
+//               expanded to bf16 w = u - 8 in the swizzled stage layout
+//   warps 6..13 per group: tcgen05.ld of the exact group dots, release of the
+//               buffer, acc += scale * I with packed f32x2 FMAs; then the
+//               partial tile, the cluster reduction and y
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 #include <stdint.h>
@@ -39,33 +60,46 @@ int make_tmap_generic(CUtensorMap* tm, CUtensorMapDataType dt, const void* base,
 
 namespace {
 
-constexpr int BM = 128;
-constexpr int BN = 128;
-constexpr int KS = 64;              // K (bf16 elements) per stage = one 128B swizzle row
+constexpr int TW = 128;                 // weight rows per CTA (MMA M, TMEM lanes)
+constexpr int TM = 128;                 // activation rows per CTA (MMA N, TMEM columns)
+constexpr int KS = 64;                  // K per stage: one 128-byte swizzle row of bf16
+constexpr int STAGE_BYTES = 128 * KS * 2;  // 16 KiB, both operands
 constexpr int STAGES = 4;
-constexpr int NBUF = 4;             // TMEM group buffers of BN columns
-constexpr int KR_MAX = 1024;        // K range per CTA
+constexpr int NRING = 8;                // weight nibble stages in flight
+constexpr int NIB_BYTES = TW * KS / 2;  // 4 KiB of nibbles per stage
+constexpr int NBUF = 4;                 // TMEM group buffers of TM columns
+constexpr int KR_MAX = 1024;            // K range per CTA
 constexpr int GR_MAX = KR_MAX / 32;
-constexpr int A_STAGE = BM * KS * 2;   // 16 KiB
-constexpr int B_STAGE = BN * KS * 2;   // 16 KiB
-constexpr int THREADS = 22 * 32;     // TMA, MMA, 4 converter, 16 epilogue warps
-constexpr int CONV_THREADS = 4 * 32;
+constexpr int MAX_SPLITS = 8;
+constexpr int THREADS = 14 * 32;
+constexpr int CONV_WARP0 = 2;
+constexpr int NCONV = 128;              // converter threads
 constexpr int EPI_WARP0 = 6;
-constexpr int EPI_THREADS = 16 * 32;
-constexpr int PST = BN + 4;          // row stride (floats) of the split-K partial in smem
-constexpr size_t SMEM_BYTES = 1024 + STAGES * (A_STAGE + B_STAGE) + (size_t)BN * KR_MAX / 2 +
-                              (size_t)BN * GR_MAX * 4 + 512;
+constexpr int NEPI = 256;               // epilogue threads
+constexpr int PST = TW + 4;             // row stride (floats) of the partial tile [m][n]
 
-// kind::f16 instruction descriptor: D f32, A bf16, B bf16, both K-major, N = BN, M = BM.
-constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
-                           ((uint32_t)(BM >> 4) << 24);
+// shared-memory map (offsets from the 1024-byte aligned base)
+constexpr size_t OFF_A = 0;                                        // activation stages
+constexpr size_t OFF_W = OFF_A + (size_t)STAGES * STAGE_BYTES;     // weight stages
+constexpr size_t OFF_N = OFF_W + (size_t)STAGES * STAGE_BYTES;     // nibble ring
+constexpr size_t OFF_SCL = OFF_N + (size_t)NRING * NIB_BYTES;      // [GR][TW] weight scales
+constexpr size_t OFF_ZW = OFF_SCL + (size_t)GR_MAX * TW * 4;       // [GR][TW] weight zeros
+constexpr size_t OFF_ACT = OFF_ZW + (size_t)GR_MAX * TW * 4;       // [GR][TM] act scales / sums
+constexpr size_t OFF_BAR = OFF_ACT + (size_t)GR_MAX * TM * 4;
+constexpr size_t SMEM_BYTES = 1024 + OFF_BAR + 512;
+static_assert((size_t)TM * PST * 4 <= OFF_N, "partial tile reuses the stage buffers");
+
+// kind::f16 instruction descriptor: D f32, A bf16, B bf16, both K-major,
+// N = TM, M = TW.
+constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(TM >> 3) << 17) |
+                           ((uint32_t)(TW >> 4) << 24);
 
 __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr) {
   uint64_t d = (uint64_t)((saddr & 0x3FFFFu) >> 4);
-  d |= (uint64_t)1 << 16;
-  d |= (uint64_t)(1024 >> 4) << 32;
-  d |= (uint64_t)1 << 46;
-  d |= (uint64_t)2 << 61;
+  d |= (uint64_t)1 << 16;            // leading byte offset (unused with 128B swizzle)
+  d |= (uint64_t)(1024 >> 4) << 32;  // stride byte offset between 8-row groups
+  d |= (uint64_t)1 << 46;            // descriptor version
+  d |= (uint64_t)2 << 61;            // SWIZZLE_128B
   return d;
 }
 __device__ __forceinline__ void tc_fence_before() {
@@ -114,25 +148,40 @@ __device__ __forceinline__ uint32_t bf16x2_minus136(uint32_t v) {
   asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(v), "r"(0x43084308u));
   return d;
 }
-__device__ __forceinline__ void ffma2(unsigned long long& acc, unsigned long long a,
-                                      unsigned long long b) {
+typedef unsigned long long f32x2;
+__device__ __forceinline__ f32x2 pack2(float lo, float hi) {
+  return ((f32x2)__float_as_uint(hi) << 32) | __float_as_uint(lo);
+}
+__device__ __forceinline__ f32x2 pack2u(uint32_t lo, uint32_t hi) {
+  return ((f32x2)hi << 32) | lo;
+}
+__device__ __forceinline__ void ffma2(f32x2& acc, f32x2 a, f32x2 b) {
   asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(a), "l"(b));
 }
-__device__ __forceinline__ unsigned long long pack2(uint32_t lo, uint32_t hi) {
-  return ((unsigned long long)hi << 32) | lo;
+__device__ __forceinline__ f32x2 fmul2(f32x2 a, f32x2 b) {
+  f32x2 d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
 }
-__device__ __forceinline__ void epi_sync(int id) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "n"(EPI_THREADS) : "memory");
-}
-__device__ __forceinline__ bool epi_and(bool v) {
+__device__ __forceinline__ float lo_f(f32x2 v) { return __uint_as_float((uint32_t)v); }
+__device__ __forceinline__ float hi_f(f32x2 v) { return __uint_as_float((uint32_t)(v >> 32)); }
+
+// Named barriers with an AND over a predicate, so every thread of a role
+// takes the same decision after a bounded wait.
+template <int ID, int N>
+__device__ __forceinline__ bool bar_and(bool v) {
   uint32_t r;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.and.pred q, 3, %2, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+      "bar.red.and.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
       : "=r"(r)
-      : "r"((uint32_t)v), "n"(EPI_THREADS)
+      : "r"((uint32_t)v), "n"(ID), "n"(N)
       : "memory");
   return r != 0;
+}
+template <int ID, int N>
+__device__ __forceinline__ void bar_sync() {
+  asm volatile("bar.sync %0, %1;" ::"n"(ID), "n"(N) : "memory");
 }
 
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -158,69 +207,293 @@ __device__ __forceinline__ float4 ld_dsmem_f4(uint32_t addr) {
   return v;
 }
 
-struct Args {
-  int M, N, K, Kr, splits, n_tiles;
-  const void* wscale;   // packed group scales [N][K/32], f32 or bf16
+// ---------------------------------------------------------------------------
+// 1. Quantization of the activation rows into swizzled bf16 tiles.
+// ---------------------------------------------------------------------------
+enum QuantMode { kRowAsym = 0, kBlockAsym = 1, kRowSym = 2 };
+
+struct RowSource {
+  const float* x;
+  int64_t ldx;  // plain rows: row m at x + m*ldx
+  // unrolled NHWC rows: row m = output pixel (n, oh, ow), k = (kh*KW + kw)*Cin + ci
+  int H, W, Cin, KH, KW, sh, sw, ph, pw, OH, OW;
+};
+
+struct QuantArgs {
+  int M, K, Mpad;
+  RowSource src;
+  int vec4;             // the 8 floats of a chunk can be read as two aligned float4
+  uint16_t* atile;      // [Mpad/128][K/64][128][64] bf16 (qA - zA), swizzled
+  float* sA;            // per-row scale [Mpad], or per-block [Mpad][K/32]
+  float* Sg;            // per-block sums of qA - zA [Mpad][K/32] (weight zeros), or NULL
+  int8_t* q_out;        // optional [M][K] codes
+  int q_vec;            // q_out is 8-byte aligned
+  float* scale_out;     // optional [M] (per row) or [M][K/32] (per block)
+  int32_t* zp_out;      // optional, same shape as scale_out
+};
+
+constexpr int QT = 256;   // threads per quantization CTA
+constexpr int QCH = 4;    // most 8-wide chunks per thread (K <= 32 * threads per row)
+
+template <bool CONV>
+__device__ __forceinline__ void load_chunk(const QuantArgs& a, int64_t m, int c, int pn, int poh,
+                                           int pow_, float (&v)[8]) {
+  const RowSource& s = a.src;
+  if (!CONV) {
+    const float* p = s.x + m * s.ldx + 8 * c;
+    if (a.vec4) {
+      const float4 u0 = __ldg(reinterpret_cast<const float4*>(p));
+      const float4 u1 = __ldg(reinterpret_cast<const float4*>(p) + 1);
+      v[0] = u0.x; v[1] = u0.y; v[2] = u0.z; v[3] = u0.w;
+      v[4] = u1.x; v[5] = u1.y; v[6] = u1.z; v[7] = u1.w;
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v[e] = __ldg(p + e);
+    }
+    return;
+  }
+  if (a.vec4) {  // Cin % 8 == 0: the chunk lies in one tap
+    const int k = 8 * c;
+    const int tap = k / s.Cin, ci = k - tap * s.Cin;
+    const int kh = tap / s.KW, kw = tap - kh * s.KW;
+    const int ih = poh * s.sh + kh - s.ph, iw = pow_ * s.sw + kw - s.pw;
+    if (ih < 0 || ih >= s.H || iw < 0 || iw >= s.W) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v[e] = 0.0f;  // a pad tap is the real value 0
+      return;
+    }
+    const float* p = s.x + (((int64_t)pn * s.H + ih) * s.W + iw) * s.Cin + ci;
+    const float4 u0 = __ldg(reinterpret_cast<const float4*>(p));
+    const float4 u1 = __ldg(reinterpret_cast<const float4*>(p) + 1);
+    v[0] = u0.x; v[1] = u0.y; v[2] = u0.z; v[3] = u0.w;
+    v[4] = u1.x; v[5] = u1.y; v[6] = u1.z; v[7] = u1.w;
+    return;
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const int k = 8 * c + e;
+    const int tap = k / s.Cin, ci = k - tap * s.Cin;
+    const int kh = tap / s.KW, kw = tap - kh * s.KW;
+    const int ih = poh * s.sh + kh - s.ph, iw = pow_ * s.sw + kw - s.pw;
+    v[e] = (ih < 0 || ih >= s.H || iw < 0 || iw >= s.W)
+               ? 0.0f
+               : __ldg(s.x + (((int64_t)pn * s.H + ih) * s.W + iw) * s.Cin + ci);
+  }
+}
+
+// R rows per CTA, QT/R threads per row; thread t of a row owns the 8-wide K
+// chunks t, t + QT/R, ... (at most QCH of them).
+template <int MODE, bool CONV>
+__global__ void __launch_bounds__(QT) a8w4_quant_tiles_kernel(QuantArgs a, int R) {
+  // the GEMM grid may start its prologue now; it waits for this grid before
+  // it reads anything written here
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  __shared__ float red[2][QT / 32];
+  const int T = QT / R;
+  const int sub = threadIdx.x / T, t = threadIdx.x - sub * T;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t m = (int64_t)blockIdx.x * R + sub;
+  const int K = a.K, G = K >> 5, nchunk = K >> 3, nkb = K >> 6;
+  const bool live = m < a.M;
+  int pn = 0, poh = 0, pow_ = 0;
+  if (CONV && live) {
+    pow_ = (int)(m % a.src.OW);
+    const int64_t tt = m / a.src.OW;
+    poh = (int)(tt % a.src.OH);
+    pn = (int)(tt / a.src.OH);
+  }
+  float v[QCH][8];
+  float mn = 0.0f, mx = 0.0f;  // min(0, .), max(0, .); mx is max|x| when symmetric
+#pragma unroll
+  for (int i = 0; i < QCH; ++i) {
+    const int c = t + i * T;
+    if (live && c < nchunk) {
+      load_chunk<CONV>(a, m, c, pn, poh, pow_, v[i]);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v[i][e] = 0.0f;
+    }
+  }
+  RowQuant rowq;
+  if (MODE != kBlockAsym) {
+#pragma unroll
+    for (int i = 0; i < QCH; ++i)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        if (MODE == kRowSym) {
+          mx = fmaxf(mx, fabsf(v[i][e]));
+        } else {
+          mn = fminf(mn, v[i][e]);
+          mx = fmaxf(mx, v[i][e]);
+        }
+      }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    }
+    if (T > 32) {  // combine the warps of this row
+      if (lane == 0) {
+        red[0][warp] = mn;
+        red[1][warp] = mx;
+      }
+      __syncthreads();
+      const int w0 = (sub * T) >> 5, nw = T >> 5;
+      mn = red[0][w0];
+      mx = red[1][w0];
+      for (int i = 1; i < nw; ++i) {
+        mn = fminf(mn, red[0][w0 + i]);
+        mx = fmaxf(mx, red[1][w0 + i]);
+      }
+    }
+    rowq = MODE == kRowSym ? row_quant_params_sym(mx) : row_quant_params(mn, mx);
+  }
+  const int mt = (int)(m >> 7), r = (int)(m & 127);
+#pragma unroll
+  for (int i = 0; i < QCH; ++i) {
+    const int c = t + i * T;
+    RowQuant q = rowq;
+    if (MODE == kBlockAsym) {
+      // the 4 chunks of a 32-wide block sit in 4 consecutive threads
+      float bmn = 0.0f, bmx = 0.0f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        bmn = fminf(bmn, v[i][e]);
+        bmx = fmaxf(bmx, v[i][e]);
+      }
+#pragma unroll
+      for (int o = 1; o < 4; o <<= 1) {
+        bmn = fminf(bmn, __shfl_xor_sync(0xffffffffu, bmn, o));
+        bmx = fmaxf(bmx, __shfl_xor_sync(0xffffffffu, bmx, o));
+      }
+      q = row_quant_params(bmn, bmx);
+    }
+    int code[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      code[e] = MODE == kRowSym ? quant_one_sym(v[i][e], q) : quant_one(v[i][e], q);
+    // block sums of the centred codes (exact; only read with weight zeros)
+    int csum = 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) csum += code[e] - q.zp;
+    if (a.Sg) {
+#pragma unroll
+      for (int o = 1; o < 4; o <<= 1) csum += __shfl_xor_sync(0xffffffffu, csum, o);
+    }
+    if (c >= nchunk || m >= a.Mpad) continue;
+    uint32_t h[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float f0 = live ? (float)(code[2 * e] - q.zp) : 0.0f;
+      const float f1 = live ? (float)(code[2 * e + 1] - q.zp) : 0.0f;
+      // |code - zp| <= 255: exact in bf16
+      h[e] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(f0)) |
+             ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(f1)) << 16);
+    }
+    const int kb = c >> 3, j = c & 7;
+    uint8_t* dst = reinterpret_cast<uint8_t*>(a.atile) +
+                   (((int64_t)mt * nkb + kb) * 128 + r) * 128 + ((j ^ (r & 7)) << 4);
+    *reinterpret_cast<uint4*>(dst) = make_uint4(h[0], h[1], h[2], h[3]);
+    if (!live) continue;
+    if (a.q_out) {
+      uint32_t lo = 0, hi = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        lo |= ((uint32_t)code[e] & 0xFFu) << (8 * e);
+        hi |= ((uint32_t)code[4 + e] & 0xFFu) << (8 * e);
+      }
+      int8_t* qo = a.q_out + m * K + 8 * c;
+      if (a.q_vec) {
+        *reinterpret_cast<uint2*>(qo) = make_uint2(lo, hi);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) qo[e] = (int8_t)code[e];
+      }
+    }
+    if (MODE == kBlockAsym && (t & 3) == 0) {
+      const int64_t b = m * G + (c >> 2);
+      a.sA[b] = q.scale;
+      if (a.scale_out) a.scale_out[b] = q.scale;
+      if (a.zp_out) a.zp_out[b] = q.zp;
+    }
+    if (a.Sg && (t & 3) == 0) a.Sg[m * G + (c >> 2)] = (float)csum;
+  }
+  if (MODE != kBlockAsym && t == 0 && m < a.Mpad) {
+    a.sA[m] = live ? rowq.scale : 0.0f;
+    if (live && a.scale_out) a.scale_out[m] = rowq.scale;
+    if (live && a.zp_out) a.zp_out[m] = rowq.zp;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// 2. The tensor-core contraction.
+// ---------------------------------------------------------------------------
+struct GemmArgs {
+  int M, N, K, Kr, splits, n_tiles, nkb;
+  const uint16_t* atile;   // activation tiles from the quantization kernel
+  const void* wscale;      // [N][K/32] f32, or bf16 when scale_bf16
   int scale_bf16;
-  const float* sA;
+  const float* wzero;      // [N][K/32] f32 weight zeros (WZP)
+  const float* sA;         // [Mpad] or [Mpad][K/32] (ABLK)
+  const float* Sg;         // [Mpad][K/32] (WZP)
   const float* bias;
   float lo, hi;
   float* y;
   int64_t ldy;
+  int stall;               // test hook: the activation stage 1 is never issued
+  uint32_t spin;           // poll limit of the pipeline waits
 };
 
+template <bool ABLK, bool WZP>
 __global__ void __launch_bounds__(THREADS, 1)
-    a8w4_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW,
-                   Args a, int* status) {
+    a8w4_tc_kernel(const __grid_constant__ CUtensorMap tmW, GemmArgs a, int* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint8_t* sA = smem;
-  uint8_t* sB = sA + STAGES * A_STAGE;
-  uint8_t* sN = sB + STAGES * B_STAGE;                         // [BN][Kr/2] nibbles of this CTA
-  float* scl_t = (float*)(sN + (size_t)BN * KR_MAX / 2);      // [Gr][BN] group scales
-  uint64_t* ld_full = (uint64_t*)(scl_t + BN * GR_MAX);
-  uint64_t* cv_full = ld_full + STAGES;
-  uint64_t* empty = cv_full + STAGES;
-  uint64_t* tfull = empty + STAGES;
+  uint8_t* sA = smem + OFF_A;
+  uint8_t* sW = smem + OFF_W;
+  uint8_t* sN = smem + OFF_N;
+  float* scl = reinterpret_cast<float*>(smem + OFF_SCL);   // [g][n]
+  float* zws = reinterpret_cast<float*>(smem + OFF_ZW);    // [g][n]
+  float* actp = reinterpret_cast<float*>(smem + OFF_ACT);  // [g][m]
+  uint64_t* a_full = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+  uint64_t* w_full = a_full + STAGES;
+  uint64_t* empty = w_full + STAGES;
+  uint64_t* nib_full = empty + STAGES;
+  uint64_t* tfull = nib_full + NRING;
   uint64_t* tempty = tfull + NBUF;
-  uint64_t* nib_full = tempty + NBUF;
-  uint32_t* tmem_slot = (uint32_t*)(nib_full + 1);
-  float* part = reinterpret_cast<float*>(smem);  // [BM][PST], reuses the A' stages after the mainloop
+  uint64_t* drain = tempty + NBUF;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  float* part = reinterpret_cast<float*>(smem);  // [TM][PST], after the mainloop
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int split = a.splits > 1 ? (int)cluster_rank() : 0;
   const int tile = blockIdx.x / a.splits;
   const int tn = tile % a.n_tiles, tm = tile / a.n_tiles;
-  const int m0 = tm * BM, n0 = tn * BN;
+  const int n0 = tn * TW, m0 = tm * TM;
   const int k0 = split * a.Kr;
-  const int Gr = a.Kr / 32;
-  const int nstages = a.Kr / KS;
-  // The N tiles of one split all read the same A' K range; each tile walks its
-  // stages in a rotated order so concurrent CTAs fetch different A' tiles
-  // instead of hammering the same L2 lines.  Stage position s holds K block
-  // kb(s) = (s + rot) % nstages (every group's dot is exact, only the f32
-  // combination order depends on it, and it is fixed per tile).
-  const int rot = (tn * 7) % nstages;
+  const int G = a.K >> 5, g0 = k0 >> 5;
+  const int Gr = a.Kr >> 5;
+  const int nst = a.Kr / KS;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&ld_full[s], 1);
-      mbar_init(&cv_full[s], CONV_THREADS / 32);
+      mbar_init(&a_full[s], 1);
+      mbar_init(&w_full[s], 1);
       mbar_init(&empty[s], 1);
     }
+    for (int s = 0; s < NRING; ++s) mbar_init(&nib_full[s], 1);
     for (int b = 0; b < NBUF; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], EPI_THREADS / 32);
+      mbar_init(&tempty[b], NEPI / 32);
     }
-    mbar_init(nib_full, 1);
+    mbar_init(drain, 1);
     fence_mbar_init();
-    prefetch_tmap(&tmA);
     prefetch_tmap(&tmW);
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_u32(tmem_slot)),
-                 "r"(NBUF * BN)
+                 "r"(NBUF * TM)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
@@ -230,75 +503,91 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint32_t tmem_base = *tmem_slot;
 
   if (warp == 0) {
-    // ------------------------- TMA producer -------------------------
+    // ---------------- activation stages (bulk copies) ----------------
     if (lane == 0) {
-      // this CTA's whole nibble slice (BN rows x Kr/2 bytes) in one box
-      mbar_arrive_expect_tx(nib_full, (uint32_t)(BN * a.Kr / 2));
-      tma_load_2d(sN, &tmW, k0 / 8, n0, nib_full);
-      // The activation codes come from the quantization grid just before
-      // this one (programmatic dependent launch): wait for it from here on.
+      uint32_t issued = 0, last_ph = 0;
+      // the activation tiles come from the quantization grid
       asm volatile("griddepcontrol.wait;" ::: "memory");
-      for (int s = 0; s < nstages; ++s) {
+      const uint8_t* src = reinterpret_cast<const uint8_t*>(a.atile) +
+                           ((int64_t)tm * a.nkb + (k0 / KS)) * STAGE_BYTES;
+      for (int s = 0; s < nst; ++s) {
         const int slot = s % STAGES;
-        if (s >= STAGES && !mbar_poll(&empty[slot], ((s / STAGES) - 1) & 1, status)) break;
-        const int kb = (s + rot) % nstages;
-        mbar_arrive_expect_tx(&ld_full[slot], (uint32_t)A_STAGE);
-        tma_load_2d(sA + slot * A_STAGE, &tmA, k0 + KS * kb, m0, &ld_full[slot]);
+        if (s >= STAGES && !mbar_poll(&empty[slot], ((s / STAGES) - 1) & 1, status, a.spin)) break;
+        if (a.stall && s == 1) continue;
+        mbar_arrive_expect_tx(&a_full[slot], STAGE_BYTES);
+        bulk_g2s(sA + slot * STAGE_BYTES, src + (int64_t)s * STAGE_BYTES, STAGE_BYTES,
+                 &a_full[slot]);
+        issued |= 1u << slot;
+        last_ph = (last_ph & ~(1u << slot)) | ((uint32_t)((s / STAGES) & 1) << slot);
       }
+      // every copy issued here has landed before the CTA may exit
+      for (int st = 0; st < STAGES; ++st)
+        if ((issued >> st) & 1u) mbar_poll(&a_full[st], (last_ph >> st) & 1u, status);
     }
   } else if (warp == 1) {
-    // ------------------------- MMA issuer -------------------------
+    // ---------------- MMA issue ----------------
     if (lane == 0) {
-      bool ok = true;
-      for (int s = 0; s < nstages && ok; ++s) {
+      bool failed = false;
+      for (int s = 0; s < nst && !failed; ++s) {
         const int slot = s % STAGES;
         const uint32_t par = (uint32_t)(s / STAGES) & 1;
-        if (!mbar_poll(&ld_full[slot], par, status) || !mbar_poll(&cv_full[slot], par, status)) break;
+        if (!mbar_poll(&a_full[slot], par, status, a.spin) ||
+            !mbar_poll(&w_full[slot], par, status, a.spin)) {
+          failed = true;
+          break;
+        }
         tc_fence_after();
-        const uint32_t a0 = smem_u32(sA + slot * A_STAGE);
-        const uint32_t b0 = smem_u32(sB + slot * B_STAGE);
+        const uint32_t wa = smem_u32(sW + slot * STAGE_BYTES);
+        const uint32_t xa = smem_u32(sA + slot * STAGE_BYTES);
 #pragma unroll
         for (int gi = 0; gi < 2; ++gi) {
           const int g = 2 * s + gi;
           const int buf = g % NBUF;
-          const uint32_t use = (uint32_t)(g / NBUF);
-          if (!mbar_poll(&tempty[buf], (use & 1) ^ 1, status)) {
-            ok = false;
+          if (!mbar_poll(&tempty[buf], ((uint32_t)(g / NBUF) & 1) ^ 1, status, a.spin)) {
+            failed = true;
             break;
           }
           tc_fence_after();
-          const uint32_t d = tmem_base + (uint32_t)(buf * BN);
-          mma_bf16(d, sdesc_sw128(a0 + 64 * gi), sdesc_sw128(b0 + 64 * gi), 0);
-          mma_bf16(d, sdesc_sw128(a0 + 64 * gi + 32), sdesc_sw128(b0 + 64 * gi + 32), 1);
+          const uint32_t d = tmem_base + (uint32_t)(buf * TM);
+          mma_bf16(d, sdesc_sw128(wa + 64 * gi), sdesc_sw128(xa + 64 * gi), 0);
+          mma_bf16(d, sdesc_sw128(wa + 64 * gi + 32), sdesc_sw128(xa + 64 * gi + 32), 1);
           mma_commit(&tfull[buf]);
         }
-        mma_commit(&empty[slot]);
+        if (!failed) mma_commit(&empty[slot]);
+      }
+      if (failed) {
+        // MMAs already issued finish before their operands or TMEM go away
+        mma_commit(drain);
+        mbar_poll(drain, 0, status);
       }
     }
   } else if (warp < EPI_WARP0) {
-    // ------------------------- nibble -> bf16 converters -------------------------
-    // Stage s, row r takes nibble words 8s..8s+7 of row r's slice; word c becomes
-    // the 16-byte chunk c of the row in the 128B-swizzled bf16 tile.
-    const int ctid = threadIdx.x - 64;  // 0..127
-    const int wpr = a.Kr / 8;           // nibble words per row
-    const uint32_t* nib = (const uint32_t*)sN;
-    bool ok = mbar_wait(nib_full, 0, status);
-    for (int s = 0; s < nstages && ok; ++s) {
-      const int slot = s % STAGES;
-      if (s >= STAGES && !mbar_wait(&empty[slot], ((s / STAGES) - 1) & 1, status)) break;
-      uint8_t* dst = sB + slot * B_STAGE;
-      const int kb = (s + rot) % nstages;
-      uint32_t w[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int idx = ctid + u * CONV_THREADS;  // 0..1023 = row * 8 + word
-        w[u] = nib[(idx >> 3) * wpr + 8 * kb + (idx & 7)];
+    // ---------------- weight nibbles -> bf16 stages ----------------
+    const int ctid = threadIdx.x - CONV_WARP0 * 32;  // 0..127
+    uint32_t issued = 0, last_ph = 0;                 // nibble ring (thread 0 only)
+    if (ctid == 0) {
+      for (int s = 0; s < nst && s < NRING; ++s) {
+        mbar_arrive_expect_tx(&nib_full[s], NIB_BYTES);
+        tma_load_2d(sN + s * NIB_BYTES, &tmW, (k0 + KS * s) / 8, n0, &nib_full[s]);
+        issued |= 1u << s;
       }
+    }
+    bool ok = true;
+    for (int s = 0; s < nst; ++s) {
+      const int slot = s % STAGES, ns = s % NRING;
+      bool w = true;
+      if (s >= STAGES) w = mbar_wait(&empty[slot], ((s / STAGES) - 1) & 1, status, a.spin);
+      w = w && mbar_wait(&nib_full[ns], (s / NRING) & 1, status, a.spin);
+      ok = bar_and<2, NCONV>(w);
+      if (!ok) break;
+      const uint32_t* nib = reinterpret_cast<const uint32_t*>(sN + ns * NIB_BYTES);
+      uint8_t* dst = sW + slot * STAGE_BYTES;
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
-        const int idx = ctid + u * CONV_THREADS;
+        const int idx = ctid + u * NCONV;  // row * 8 + word
         const int r = idx >> 3, c = idx & 7;
-        const uint32_t L = w[u] & 0x0F0F0F0Fu, H = (w[u] >> 4) & 0x0F0F0F0Fu;
+        const uint32_t wd = nib[idx];
+        const uint32_t L = wd & 0x0F0F0F0Fu, H = (wd >> 4) & 0x0F0F0F0Fu;
         uint4 o;
         o.x = bf16x2_minus136(prmt(L, 0x43434343u, 0x5140u));
         o.y = bf16x2_minus136(prmt(L, 0x43434343u, 0x5342u));
@@ -307,322 +596,311 @@ __global__ void __launch_bounds__(THREADS, 1)
         *reinterpret_cast<uint4*>(dst + r * 128 + ((c ^ (r & 7)) << 4)) = o;
       }
       fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&cv_full[slot]);
+      bar_sync<2, NCONV>();  // every converter is done with this nibble stage
+      if (ctid == 0) {
+        mbar_arrive(&w_full[slot]);
+        const int sn = s + NRING;
+        if (sn < nst) {
+          mbar_arrive_expect_tx(&nib_full[ns], NIB_BYTES);
+          tma_load_2d(sN + ns * NIB_BYTES, &tmW, (k0 + KS * sn) / 8, n0, &nib_full[ns]);
+          last_ph = (last_ph & ~(1u << ns)) | ((uint32_t)((sn / NRING) & 1) << ns);
+        }
+      }
+    }
+    if (ctid == 0) {
+      for (int st = 0; st < NRING; ++st)
+        if ((issued >> st) & 1u) mbar_poll(&nib_full[st], (last_ph >> st) & 1u, status);
     }
   } else {
-    // ------------------------- epilogue -------------------------
-    const int etid = threadIdx.x - EPI_WARP0 * 32;  // 0..511
+    // ---------------- epilogue ----------------
+    const int etid = threadIdx.x - EPI_WARP0 * 32;  // 0..255
     const int q = warp & 3;                         // TMEM lane quarter
-    const int cb = (warp - EPI_WARP0) >> 2;         // 32-column block
-    const int row = 32 * q + lane;
-    const int m = m0 + row;
-    bool ok = true;
-    {
-      // group scales of this tile, transposed to [g][n] (rows past N read as 0)
-      const int G = a.K / 32, g0 = k0 / 32;
-      for (int i = etid; i < BN * Gr; i += EPI_THREADS) {
-        const int n = i / Gr, g = i - n * Gr;
-        const int64_t idx = (int64_t)(n0 + n) * G + g0 + g;
-        float v = 0.0f;
-        if (n0 + n < a.N)  // a bf16 scale widens to f32 exactly
-          v = a.scale_bf16
-                  ? __uint_as_float((uint32_t)__ldg(reinterpret_cast<const unsigned short*>(a.wscale) + idx) << 16)
-                  : __ldg(reinterpret_cast<const float*>(a.wscale) + idx);
-        scl_t[g * BN + n] = v;
+    const int cb = (warp - EPI_WARP0) >> 2;         // 64-column half
+    const int nl = 32 * q + lane;                   // weight row within the tile
+    // group scales (and zeros) of this CTA's rows and K range, as [g][n]
+    for (int i = etid; i < Gr * TW; i += NEPI) {
+      const int g = i / TW, n = i - g * TW;
+      const int64_t idx = (int64_t)(n0 + n) * G + g0 + g;
+      float v = 0.0f, z = 0.0f;
+      if (n0 + n < a.N) {
+        v = a.scale_bf16
+                ? __uint_as_float((uint32_t)__ldg(reinterpret_cast<const unsigned short*>(a.wscale) + idx) << 16)
+                : __ldg(reinterpret_cast<const float*>(a.wscale) + idx);
+        if (WZP) z = __ldg(a.wzero + idx);
+      }
+      scl[i] = v;
+      if (WZP) zws[i] = z;
+    }
+    // activation scales per block / group sums come from the quantization grid
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (ABLK || WZP) {
+      const float* src = ABLK ? a.sA : a.Sg;
+      for (int i = etid; i < Gr * TM; i += NEPI) {
+        const int g = i / TM, mm = i - g * TM;
+        actp[i] = src[(int64_t)(m0 + mm) * G + g0 + g];
       }
     }
-    epi_sync(1);
-    // sA (read after the mainloop) comes from the quantization grid
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    unsigned long long acc[16];
+    bar_sync<1, NEPI>();
+    f32x2 acc[32];
 #pragma unroll
-    for (int j = 0; j < 16; ++j) acc[j] = 0ull;
+    for (int j = 0; j < 32; ++j) acc[j] = 0ull;
+    bool ok = true;
     for (int g = 0; g < Gr && ok; ++g) {
       const int buf = g % NBUF;
-      const uint32_t use = (uint32_t)(g / NBUF);
-      ok = mbar_wait(&tfull[buf], use & 1, status);
+      // warp-uniform decision: the TMEM loads below are .sync.aligned
+      ok = __all_sync(0xffffffffu, mbar_wait(&tfull[buf], (uint32_t)(g / NBUF) & 1, status, a.spin));
+      if (!ok) break;
       tc_fence_after();
-      uint32_t p[32];
-      tmem_ld32(tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * BN + 32 * cb), p);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[buf]);
-      const int gg = 2 * (((g >> 1) + rot) % nstages) + (g & 1);  // K group held by buffer
-      const float4* sc = reinterpret_cast<const float4*>(scl_t + gg * BN + 32 * cb);
+      const float sw = scl[g * TW + nl];
+      const f32x2 s2 = pack2(sw, sw);
+      const f32x2* ap = reinterpret_cast<const f32x2*>(actp + g * TM + 64 * cb);
+      const uint32_t taddr = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * TM + 64 * cb);
+      // the two 32-column halves one after the other (32 staging registers)
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const float4 s4 = sc[j];
-        ffma2(acc[2 * j], pack2(p[4 * j], p[4 * j + 1]),
-              pack2(__float_as_uint(s4.x), __float_as_uint(s4.y)));
-        ffma2(acc[2 * j + 1], pack2(p[4 * j + 2], p[4 * j + 3]),
-              pack2(__float_as_uint(s4.z), __float_as_uint(s4.w)));
-      }
-    }
-    ok = epi_and(ok);
-    float v[32];
+      for (int h = 0; h < 2; ++h) {
+        uint32_t p[32];
+        tmem_ld32(taddr + 32 * h, p);
+        tmem_wait_ld();
+        if (h == 1) {  // both halves read: hand the buffer back to the MMA warp
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[buf]);
+        }
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      v[2 * j] = __uint_as_float((uint32_t)(acc[j] & 0xFFFFFFFFull));
-      v[2 * j + 1] = __uint_as_float((uint32_t)(acc[j] >> 32));
-    }
-    const int nb = n0 + 32 * cb;
-    if (a.splits == 1) {
-      // N % 4 == 0 on this path: every float4 chunk is fully in or out of range
-      if (ok && m < a.M) {
-        const float s = a.sA[m];
-        float* yr = a.y + (int64_t)m * a.ldy;
-        const bool vec = ((a.ldy & 3) == 0) && ((reinterpret_cast<uintptr_t>(a.y) & 15) == 0);
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const int n = nb + 4 * c;
-          if (n < a.N) {
-            float t[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              t[e] = __fmul_rn(s, v[4 * c + e]);
-              if (a.bias) t[e] = __fadd_rn(t[e], a.bias[n + e]);
-              t[e] = fminf(fmaxf(t[e], a.lo), a.hi);
-            }
-            if (vec) {
-              *reinterpret_cast<float4*>(yr + n) = make_float4(t[0], t[1], t[2], t[3]);
-            } else {
-#pragma unroll
-              for (int e = 0; e < 4; ++e) yr[n + e] = t[e];
-            }
-          }
+        for (int j = 0; j < 16; ++j) {
+          const f32x2 d = pack2u(p[2 * j], p[2 * j + 1]);
+          if (ABLK)
+            ffma2(acc[16 * h + j], d, fmul2(s2, ap[16 * h + j]));
+          else
+            ffma2(acc[16 * h + j], d, s2);
         }
       }
-    } else {
-      // park this split's partial tile in shared memory for the cluster reduction
-      float4* dst = reinterpret_cast<float4*>(part + row * PST + 32 * cb);
+      if (WZP) {
+        const float zw = zws[g * TW + nl];
+        const f32x2 z2 = pack2(zw, zw);
+        const f32x2* sp = reinterpret_cast<const f32x2*>(actp + g * TM + 64 * cb);
 #pragma unroll
-      for (int c = 0; c < 8; ++c)
-        dst[c] = make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+        for (int j = 0; j < 32; ++j) ffma2(acc[j], sp[j], z2);
+      }
+    }
+    ok = bar_and<1, NEPI>(ok);
+    // park the partial tile as [m][n]; every MMA has completed (the last
+    // group's accumulator was waited for), so the stage buffers are free
+    if (ok) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        part[(64 * cb + 2 * j) * PST + nl] = lo_f(acc[j]);
+        part[(64 * cb + 2 * j + 1) * PST + nl] = hi_f(acc[j]);
+      }
     }
   }
 
+  // Split-K reduction over the cluster (one CTA per K range): after the
+  // first cluster barrier every partial is visible; CTA `split` sums its
+  // share of the rows over all ranks in rank order (deterministic) and
+  // writes y; the second barrier keeps every CTA's shared memory alive until
+  // its peers have read it.
   __syncwarp();
-  if (a.splits > 1) {
-    // Split-K reduction over the cluster (one CTA per K range): after the
-    // first cluster barrier every partial is visible; CTA `split` sums its
-    // share of the rows over all ranks in rank order (deterministic) and
-    // writes y; the second barrier keeps every CTA's shared memory alive
-    // until its peers have read it.
-    cluster_sync_all();
-    if (warp >= EPI_WARP0) {
-      const int etid = threadIdx.x - EPI_WARP0 * 32;
-      const int rows_per = BM / a.splits;
-      const uint32_t part_s = smem_u32(part);
-      for (int i = etid; i < rows_per * (BN / 4); i += EPI_THREADS) {
-        const int r = split * rows_per + i / (BN / 4);
-        const int c = i % (BN / 4);
-        const int m = m0 + r, n = n0 + 4 * c;
-        const uint32_t off = (uint32_t)((r * PST + 4 * c) * 4);
-        float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int j = 0; j < a.splits; ++j) {
-          const float4 t = ld_dsmem_f4(mapa(part_s + off, (uint32_t)j));
-          sum.x = __fadd_rn(sum.x, t.x);
-          sum.y = __fadd_rn(sum.y, t.y);
-          sum.z = __fadd_rn(sum.z, t.z);
-          sum.w = __fadd_rn(sum.w, t.w);
-        }
-        if (m < a.M && n < a.N) {
-          const float s = a.sA[m];
-          float t4[4] = {sum.x, sum.y, sum.z, sum.w};
+  cluster_sync_all();
+  if (warp >= EPI_WARP0) {
+    const int etid = threadIdx.x - EPI_WARP0 * 32;
+    const int rows_per = (TM + a.splits - 1) / a.splits;
+    const int r0 = split * rows_per, r1 = min(TM, r0 + rows_per);
+    const uint32_t part_s = smem_u32(part);
+    const bool vec = ((a.ldy & 3) == 0) && ((reinterpret_cast<uintptr_t>(a.y) & 15) == 0);
+    for (int i = etid; i < (r1 - r0) * (TW / 4); i += NEPI) {
+      const int mm = r0 + i / (TW / 4);
+      const int c = i % (TW / 4);
+      const int m = m0 + mm, n = n0 + 4 * c;
+      if (m >= a.M || n >= a.N) continue;
+      const uint32_t off = (uint32_t)((mm * PST + 4 * c) * 4);
+      float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int j = 0; j < a.splits; ++j) {
+        const float4 t = ld_dsmem_f4(mapa(part_s + off, (uint32_t)j));
+        sum.x = __fadd_rn(sum.x, t.x);
+        sum.y = __fadd_rn(sum.y, t.y);
+        sum.z = __fadd_rn(sum.z, t.z);
+        sum.w = __fadd_rn(sum.w, t.w);
+      }
+      const float s = ABLK ? 1.0f : a.sA[m];
+      float t4[4] = {sum.x, sum.y, sum.z, sum.w};
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            t4[e] = __fmul_rn(s, t4[e]);
-            if (a.bias) t4[e] = __fadd_rn(t4[e], a.bias[n + e]);
-            t4[e] = fminf(fmaxf(t4[e], a.lo), a.hi);
-          }
-          float* yr = a.y + (int64_t)m * a.ldy + n;
-          if (((a.ldy & 3) == 0) && ((reinterpret_cast<uintptr_t>(a.y) & 15) == 0)) {
-            *reinterpret_cast<float4*>(yr) = make_float4(t4[0], t4[1], t4[2], t4[3]);
-          } else {
+      for (int e = 0; e < 4; ++e) {
+        if (!ABLK) t4[e] = __fmul_rn(s, t4[e]);
+        if (a.bias && n + e < a.N) t4[e] = __fadd_rn(t4[e], a.bias[n + e]);
+        t4[e] = fminf(fmaxf(t4[e], a.lo), a.hi);
+      }
+      float* yr = a.y + (int64_t)m * a.ldy + n;
+      if (vec && n + 3 < a.N) {
+        *reinterpret_cast<float4*>(yr) = make_float4(t4[0], t4[1], t4[2], t4[3]);
+      } else {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) yr[e] = t4[e];
-          }
-        }
+        for (int e = 0; e < 4; ++e)
+          if (n + e < a.N) yr[e] = t4[e];
       }
     }
-    __syncwarp();
-    cluster_sync_all();
   }
+  __syncwarp();
+  cluster_sync_all();
 
-  // Reconverge every warp (lane 0 of the TMA and MMA warps ran their loops
-  // alone) so the CTA barrier below counts complete warps only after all
-  // of their work, in particular before TMEM is freed.
+  // Reconverge every warp (single lanes ran the copy and MMA loops) so the
+  // CTA barrier below counts complete warps, then free TMEM.
   __syncwarp();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
-                 "r"(NBUF * BN)
+                 "r"(NBUF * TM)
                  : "memory");
   }
 }
 
-// Per-row quantization into bf16 (q - zp) for the tensor-core operand, plus
-// the scale/zero-point and (optionally) the int8 codes.
-__global__ void __launch_bounds__(256) quantize_rows_centered_kernel(
-    int K, const float* __restrict__ x, int64_t ldx, uint16_t* __restrict__ qc,
-    int8_t* __restrict__ q_opt, float* __restrict__ scale, int32_t* __restrict__ zero_point) {
-  __shared__ float red[16];
-  const int64_t m = blockIdx.x;
-  // let the GEMM grid start its prologue (it waits before reading our outputs)
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  const float* xr = x + m * ldx;
-  float mn = 0.0f, mx = 0.0f;
-  int k = threadIdx.x;
-  for (; k + 7 * 256 < K; k += 8 * 256) {
-    float v[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) v[u] = xr[k + u * 256];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      mn = fminf(mn, v[u]);
-      mx = fmaxf(mx, v[u]);
-    }
-  }
-  for (; k < K; k += 256) {
-    mn = fminf(mn, xr[k]);
-    mx = fmaxf(mx, xr[k]);
-  }
-  for (int o = 16; o > 0; o >>= 1) {
-    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  }
-  if ((threadIdx.x & 31) == 0) {
-    red[threadIdx.x >> 5] = mn;
-    red[8 + (threadIdx.x >> 5)] = mx;
-  }
-  __syncthreads();
-  mn = red[0];
-  mx = red[8];
-  for (int i = 1; i < 8; ++i) {
-    mn = fminf(mn, red[i]);
-    mx = fmaxf(mx, red[8 + i]);
-  }
-  // scale = (rmax - rmin)/255 (1 if 0), inv = 1/scale, zp = clamp(rne(-128 - rmin*inv))
-  float sc = __fdiv_rn(__fsub_rn(mx, mn), 255.0f);
-  if (sc == 0.0f) sc = 1.0f;
-  const float inv = __fdiv_rn(1.0f, sc);
-  const int zp = min(max(__float2int_rn(__fsub_rn(-128.0f, __fmul_rn(mn, inv))), -128), 127);
-  uint16_t* qr = qc + m * K;
-  // (v - zp) in [-255, 255] is exact in bf16: built through f32 (exact), then truncated
-  k = threadIdx.x;
-  for (; k + 7 * 256 < K; k += 8 * 256) {
-    float xv[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) xv[u] = xr[k + u * 256];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int v = min(max(__float2int_rn(__fmul_rn(xv[u], inv)) + zp, -128), 127);
-      qr[k + u * 256] = (uint16_t)(__float_as_uint((float)(v - zp)) >> 16);
-      if (q_opt) q_opt[m * K + k + u * 256] = (int8_t)v;
-    }
-  }
-  for (; k < K; k += 256) {
-    const int v = min(max(__float2int_rn(__fmul_rn(xr[k], inv)) + zp, -128), 127);
-    qr[k] = (uint16_t)(__float_as_uint((float)(v - zp)) >> 16);
-    if (q_opt) q_opt[m * K + k] = (int8_t)v;
-  }
-  if (threadIdx.x == 0) {
-    scale[m] = sc;
-    zero_point[m] = zp;
-  }
-}
-
-}  // namespace
-
-size_t a8w4_tc_workspace_bytes(int M, int N, int K, int splits) {
-  (void)N;
-  (void)splits;
-  return (size_t)(round_up((int64_t)M * K * 2, 256) + 2 * round_up((int64_t)M * 4, 256));
-}
-
-// Split count s in {1, 2, 4, 8} (one cluster of s CTAs per output tile, K
-// range K/s a multiple of 128 and <= 1024): the largest with tiles*s no more
-// than the SM count, at least the smallest valid one.
-int a8w4_tc_splits(int M, int N, int K, int sms) {
-  const int64_t tiles = cdiv(M, BM) * cdiv(N, BN);
+// Split count s (a cluster of s CTAs per output tile): K/s a multiple of 64
+// and at most KR_MAX; the largest s with tiles * s within the SM count, else
+// the smallest valid one; -1 if none.
+int choose_splits(int64_t tiles, int K, int sms) {
   int best = -1;
-  for (int s = 1; s <= 8; s *= 2) {
-    if (K % s) continue;
-    const int kr = K / s;
-    if (kr % 128 || kr > KR_MAX) continue;  // scale tile rows must be 16-byte multiples
+  for (int s = 1; s <= MAX_SPLITS; ++s) {
+    if (K % (KS * s)) continue;
+    if (K / s > KR_MAX) continue;
     if (best < 0) best = s;
     if (tiles * s <= sms) best = s;
   }
   return best;
 }
 
-bool a8w4_tc_supported(int M, int N, int K) {
-  return K % 128 == 0 && N % 4 == 0 && a8w4_tc_splits(M, N, K, 1 << 30) > 0;
+struct TcPlan {
+  int m_tiles, n_tiles, splits, R;
+  int64_t Mpad;
+  size_t off_sA, off_Sg, bytes;
+};
+
+TcPlan plan_tc(int64_t M, int N, int K, int sms) {
+  TcPlan p{};
+  p.m_tiles = (int)cdiv(M, TM);
+  p.n_tiles = (int)cdiv(N, TW);
+  p.Mpad = (int64_t)p.m_tiles * TM;
+  p.splits = choose_splits((int64_t)p.m_tiles * p.n_tiles, K, sms);
+  int R = 1;
+  while (R < 8 && (int64_t)K * 2 * R <= (int64_t)32 * QT) R *= 2;  // K <= 32 * (QT / R)
+  p.R = R;
+  const int G = K / 32;
+  p.off_sA = (size_t)round_up(p.Mpad * K * 2, 256);
+  p.off_Sg = p.off_sA + (size_t)round_up(p.Mpad * G * 4, 256);
+  p.bytes = p.off_Sg + (size_t)round_up(p.Mpad * G * 4, 256);
+  return p;
+}
+
+template <int MODE, bool CONV>
+int launch_quant(const QuantArgs& qa, int grid, int R, cudaStream_t st) {
+  a8w4_quant_tiles_kernel<MODE, CONV><<<grid, QT, 0, st>>>(qa, R);
+  return launch_status();
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+bool a8w4_tc_supported(int64_t M, int N, int K) {
+  if (M < 2 || N < 1 || K < KS || K % KS) return false;
+  if (K > QCH * 8 * QT) return false;  // one quantization CTA per row holds the row
+  return choose_splits((cdiv(M, TM)) * cdiv(N, TW), K, 1 << 30) > 0;
+}
+
+size_t a8w4_tc_workspace_bytes(int64_t M, int N, int K) {
+  return plan_tc(M, N, K, 1 << 30).bytes;
 }
 
 int a8w4_tc_setup() {
-  cudaError_t e = cudaFuncSetAttribute(a8w4_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)SMEM_BYTES);
-  return e == cudaSuccess ? QG_OK : QG_ERR_CUDA;
+  const void* fns[] = {(const void*)a8w4_tc_kernel<false, false>,
+                       (const void*)a8w4_tc_kernel<true, false>,
+                       (const void*)a8w4_tc_kernel<false, true>};
+  for (const void* f : fns)
+    if (cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES) !=
+        cudaSuccess)
+      return QG_ERR_CUDA;
+  return QG_OK;
 }
 
-int launch_a8w4_tc(int M, int N, int K, const float* x, int64_t ldx, const void* packed,
-                   const float* bias, float lo, float hi, float* y, int64_t ldy, int8_t* q_out,
-                   float* scale_out, int32_t* zp_out, void* ws, size_t ws_bytes, bool scale_bf16,
-                   cudaStream_t st) {
-  const int splits = a8w4_tc_splits(M, N, K, num_sms());
-  if (splits <= 0) return QG_ERR_UNSUPPORTED;
-  if (!ws || ws_bytes < a8w4_tc_workspace_bytes(M, N, K, splits)) return QG_ERR_WORKSPACE;
-  const int64_t mt = cdiv(M, BM), nt = cdiv(N, BN);
+int launch_a8w4_tc_call(const A8W4TcCall& c, void* ws, size_t ws_bytes, cudaStream_t st) {
+  const TcPlan p = plan_tc(c.M, c.N, c.K, num_sms());
+  if (p.splits <= 0) return QG_ERR_UNSUPPORTED;
+  if (!ws || ws_bytes < p.bytes) return QG_ERR_WORKSPACE;
+  if ((c.mode == kBlockAsym) && c.wzero) return QG_ERR_UNSUPPORTED;
   uint8_t* w = (uint8_t*)ws;
-  uint16_t* qc = (uint16_t*)w;
-  w += round_up((int64_t)M * K * 2, 256);
-  float* sA = (float*)w;
-  w += round_up((int64_t)M * 4, 256);
-  int32_t* zA = (int32_t*)w;
-  quantize_rows_centered_kernel<<<M, 256, 0, st>>>(K, x, ldx, qc, q_out, sA, zA);
-  int rc = launch_status();
+  QuantArgs qa{};
+  qa.M = (int)c.M;
+  qa.K = c.K;
+  qa.Mpad = (int)p.Mpad;
+  qa.src.x = c.x;
+  qa.src.ldx = c.ldx;
+  qa.src.H = c.H; qa.src.W = c.W; qa.src.Cin = c.Cin; qa.src.KH = c.KH; qa.src.KW = c.KW;
+  qa.src.sh = c.sh; qa.src.sw = c.sw; qa.src.ph = c.ph; qa.src.pw = c.pw;
+  qa.src.OH = c.OH; qa.src.OW = c.OW;
+  const bool x16 = ((uintptr_t)c.x & 15) == 0;
+  qa.vec4 = c.conv ? (x16 && c.Cin % 8 == 0) : (x16 && c.ldx % 4 == 0);
+  qa.atile = (uint16_t*)w;
+  qa.sA = (float*)(w + p.off_sA);
+  qa.Sg = c.wzero ? (float*)(w + p.off_Sg) : nullptr;
+  qa.q_out = c.q_out;
+  qa.q_vec = ((uintptr_t)c.q_out & 7) == 0;
+  qa.scale_out = c.scale_out;
+  qa.zp_out = c.zp_out;
+  const int qgrid = (int)cdiv(p.Mpad, p.R);
+  int rc;
+  if (c.conv) {
+    if (c.mode == kRowAsym) rc = launch_quant<kRowAsym, true>(qa, qgrid, p.R, st);
+    else if (c.mode == kRowSym) rc = launch_quant<kRowSym, true>(qa, qgrid, p.R, st);
+    else return QG_ERR_UNSUPPORTED;
+  } else {
+    if (c.mode == kRowAsym) rc = launch_quant<kRowAsym, false>(qa, qgrid, p.R, st);
+    else if (c.mode == kBlockAsym) rc = launch_quant<kBlockAsym, false>(qa, qgrid, p.R, st);
+    else rc = launch_quant<kRowSym, false>(qa, qgrid, p.R, st);
+  }
   if (rc != QG_OK) return rc;
-  if (scale_out && cudaMemcpyAsync(scale_out, sA, (size_t)M * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
-    return QG_ERR_CUDA;
-  if (zp_out && cudaMemcpyAsync(zp_out, zA, (size_t)M * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
-    return QG_ERR_CUDA;
-  const uint8_t* wq = (const uint8_t*)packed;
-  const void* wsc = wq + (size_t)N * (K / 2);
-  const int Kr = K / splits;
-  CUtensorMap tmA, tmW;
-  rc = make_tmap_generic(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, qc, (uint64_t)K, (uint64_t)M,
-                         (uint64_t)K * 2, KS, BM, CU_TENSOR_MAP_SWIZZLE_128B);
+
+  const uint8_t* wq = (const uint8_t*)c.packed;
+  CUtensorMap tmW;
+  rc = make_tmap_generic(&tmW, CU_TENSOR_MAP_DATA_TYPE_UINT32, wq, (uint64_t)c.K / 8,
+                         (uint64_t)c.N, (uint64_t)c.K / 2, KS / 8, TW, CU_TENSOR_MAP_SWIZZLE_NONE);
   if (rc != QG_OK) return rc;
-  rc = make_tmap_generic(&tmW, CU_TENSOR_MAP_DATA_TYPE_UINT32, wq, (uint64_t)K / 8, (uint64_t)N,
-                         (uint64_t)K / 2, (uint32_t)(Kr / 8), BN, CU_TENSOR_MAP_SWIZZLE_NONE);
-  if (rc != QG_OK) return rc;
-  Args a;
-  a.M = M; a.N = N; a.K = K; a.Kr = Kr; a.splits = splits; a.n_tiles = (int)nt;
-  a.wscale = wsc;
-  a.scale_bf16 = scale_bf16 ? 1 : 0;
-  a.sA = sA; a.bias = bias; a.lo = lo; a.hi = hi; a.y = y; a.ldy = ldy;
+  GemmArgs ga{};
+  ga.M = (int)c.M; ga.N = c.N; ga.K = c.K;
+  ga.Kr = c.K / p.splits; ga.splits = p.splits; ga.n_tiles = p.n_tiles; ga.nkb = c.K / KS;
+  ga.atile = qa.atile;
+  ga.wscale = wq + (size_t)c.N * (c.K / 2);
+  ga.scale_bf16 = c.scale_bf16 ? 1 : 0;
+  ga.wzero = c.wzero;
+  ga.sA = qa.sA;
+  ga.Sg = qa.Sg;
+  ga.bias = c.bias; ga.lo = c.lo; ga.hi = c.hi; ga.y = c.y; ga.ldy = c.ldy;
+  ga.stall = take_stall(kStallA8W4TC) ? 1 : 0;
+  ga.spin = ga.stall ? kStallSpinLimit : kSpinLimit;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(mt * nt * splits));
+  cfg.gridDim = dim3((unsigned)((int64_t)p.m_tiles * p.n_tiles * p.splits));
   cfg.blockDim = dim3(THREADS);
   cfg.dynamicSmemBytes = SMEM_BYTES;
   cfg.stream = st;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = (unsigned)splits;
+  attr[0].val.clusterDim.x = (unsigned)p.splits;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
-  // programmatic dependent launch: the prologue (barriers, TMEM, the weight
-  // nibbles and scales) overlaps the quantization grid
+  // programmatic dependent launch: barriers, TMEM, the weight nibbles and
+  // scales overlap the quantization grid
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, a8w4_tc_kernel, tmA, tmW, a, status_word());
+  cudaError_t e;
+  if (c.mode == kBlockAsym)
+    e = cudaLaunchKernelEx(&cfg, a8w4_tc_kernel<true, false>, tmW, ga, status_word());
+  else if (c.wzero)
+    e = cudaLaunchKernelEx(&cfg, a8w4_tc_kernel<false, true>, tmW, ga, status_word());
+  else
+    e = cudaLaunchKernelEx(&cfg, a8w4_tc_kernel<false, false>, tmW, ga, status_word());
   return e == cudaSuccess ? QG_OK : QG_ERR_CUDA;
 }
 

@@ -38,13 +38,6 @@ int setup_a8w4_gemv();
 int setup_a8w4_gemm_simt();
 int i8gemm_setup();
 int a8w4_tc_setup();
-bool a8w4_tc_supported(int M, int N, int K);
-int a8w4_tc_splits(int M, int N, int K, int sms);
-size_t a8w4_tc_workspace_bytes(int M, int N, int K, int splits);
-int launch_a8w4_tc(int M, int N, int K, const float* x, int64_t ldx, const void* packed,
-                   const float* bias, float lo, float hi, float* y, int64_t ldy, int8_t* q_out,
-                   float* scale_out, int32_t* zp_out, void* ws, size_t ws_bytes, bool scale_bf16,
-                   cudaStream_t st);
 
 int i8gemm_pack_b(int K, int N, const int8_t* B, int64_t ldb, void* packed, cudaStream_t st);
 size_t i8gemm_pack_b_bytes(int K, int N);
@@ -387,12 +380,25 @@ static size_t a8w4_ws_layout(int M, int K, size_t* off_scale, size_t* off_zp) {
   return q + s + round_up((int64_t)M * 4, 256);
 }
 
+// Workspace of an M > 1 A8W4 call, for every variant (per-row or per-block
+// activations, symmetric or asymmetric weights): the tensor-core layout
+// where that path applies, else the CUDA-core one.
 extern "C" size_t qgemm_a8w4_workspace_bytes(int M, int N, int K) {
   if (M <= 0 || N <= 0 || K <= 0) return 0;
   if (M == 1 && K <= kFusedGemvMaxK) return 0;
-  if (a8w4_tc_supported(M, N, K))
-    return a8w4_tc_workspace_bytes(M, N, K, a8w4_tc_splits(M, N, K, num_sms()));
+  if (a8w4_tc_supported(M, N, K)) return a8w4_tc_workspace_bytes(M, N, K);
   return a8w4_ws_layout(M, K, nullptr, nullptr);
+}
+
+// Fields of the tensor-core call shared by the plain-row entry points.
+static A8W4TcCall tc_rows(int M, int N, int K, const float* x, int64_t ldx, const void* packed_w,
+                          const float* bias, float lo, float hi, float* y, int64_t ldy,
+                          int8_t* q_out, float* scale_out, int32_t* zp_out) {
+  A8W4TcCall c{};
+  c.M = M; c.N = N; c.K = K; c.x = x; c.ldx = ldx; c.conv = false;
+  c.packed = packed_w; c.bias = bias; c.lo = lo; c.hi = hi; c.y = y; c.ldy = ldy;
+  c.q_out = q_out; c.scale_out = scale_out; c.zp_out = zp_out;
+  return c;
 }
 
 static int a8w4_linear(int M, int N, int K, const float* x, int64_t ldx, const void* packed_w,
@@ -417,8 +423,11 @@ static int a8w4_linear(int M, int N, int K, const float* x, int64_t ldx, const v
   if (a8w4_tc_supported(M, N, K)) {
     if (!workspace) return QG_ERR_WORKSPACE;
     if (!aligned(workspace, 256)) return QG_ERR_MISALIGNED;
-    return launch_a8w4_tc(M, N, K, x, ldx, packed_w, bias, clamp_min, clamp_max, y, ldy, q_out,
-                          scale_out, zp_out, workspace, workspace_bytes, sbf, st);
+    A8W4TcCall c = tc_rows(M, N, K, x, ldx, packed_w, bias, clamp_min, clamp_max, y, ldy, q_out,
+                           scale_out, zp_out);
+    c.mode = 0;
+    c.scale_bf16 = sbf;
+    return launch_a8w4_tc_call(c, workspace, workspace_bytes, st);
   }
   if (K > kSimtMaxK) return QG_ERR_UNSUPPORTED;
   size_t off_s = 0, off_z = 0;
@@ -459,25 +468,47 @@ extern "C" int qgemm_a8w4_f32_bf16s(int M, int N, int K, const float* x, int64_t
                      scale_out, zp_out, workspace, workspace_bytes, true, stream);
 }
 
-extern "C" int qgemm_a8w4_f32_actblock(int M, int N, int K, const float* x, int64_t ldx,
-                                       const void* packed_w, const float* bias,
-                                       float clamp_min, float clamp_max, float* y,
-                                       int64_t ldy, int8_t* q_out, float* scale_out,
-                                       int32_t* zp_out, void* stream) {
+// Checks shared by the per-block-activation and asymmetric-weight variants,
+// all made on the host before any device work: QG_OK when the call can run.
+static int a8w4_variant_args(int M, int N, int K, const float* x, int64_t ldx,
+                             const void* packed_w, const float* bias, float clamp_min,
+                             float clamp_max, float* y, int64_t ldy, float* scale_out,
+                             int32_t* zp_out, void* workspace, size_t workspace_bytes) {
   if (M < 0 || N <= 0 || K <= 0 || ldx < K || ldy < N) return QG_ERR_INVALID_ARG;
   if (K % 32) return QG_ERR_UNSUPPORTED;
   if (!(clamp_min <= clamp_max)) return QG_ERR_INVALID_ARG;  // also rejects NaN
   if (M == 0) return QG_OK;
-  if (M != 1) return QG_ERR_UNSUPPORTED;
   if (!x || !packed_w || !y) return QG_ERR_INVALID_ARG;
   if (!aligned(packed_w, 16)) return QG_ERR_MISALIGNED;
   if (!aligned(x, 4) || !aligned(y, 4) || (bias && !aligned(bias, 4))) return QG_ERR_MISALIGNED;
   if ((scale_out && !aligned(scale_out, 4)) || (zp_out && !aligned(zp_out, 4)))
     return QG_ERR_MISALIGNED;
-  int rc = device_ready();
-  if (rc != QG_OK) return rc;
-  return launch_a8w4_gemv_actblock(N, K, x, packed_w, bias, clamp_min, clamp_max, y, q_out,
-                                   scale_out, zp_out, (cudaStream_t)stream);
+  if (M == 1) {  // the fused GEMV: no workspace
+    if (K % 128 || K > 8192 || !aligned(x, 16)) return QG_ERR_UNSUPPORTED;
+  } else {       // the tensor-core path
+    if (!a8w4_tc_supported(M, N, K)) return QG_ERR_UNSUPPORTED;
+    if (!workspace || workspace_bytes < a8w4_tc_workspace_bytes(M, N, K)) return QG_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return QG_ERR_MISALIGNED;
+  }
+  return device_ready();
+}
+
+extern "C" int qgemm_a8w4_f32_actblock(int M, int N, int K, const float* x, int64_t ldx,
+                                       const void* packed_w, const float* bias,
+                                       float clamp_min, float clamp_max, float* y,
+                                       int64_t ldy, int8_t* q_out, float* scale_out,
+                                       int32_t* zp_out, void* workspace, size_t workspace_bytes,
+                                       void* stream) {
+  int rc = a8w4_variant_args(M, N, K, x, ldx, packed_w, bias, clamp_min, clamp_max, y, ldy,
+                             scale_out, zp_out, workspace, workspace_bytes);
+  if (rc != QG_OK || M == 0) return rc;
+  if (M == 1)
+    return launch_a8w4_gemv_actblock(N, K, x, packed_w, bias, clamp_min, clamp_max, y, q_out,
+                                     scale_out, zp_out, (cudaStream_t)stream);
+  A8W4TcCall c = tc_rows(M, N, K, x, ldx, packed_w, bias, clamp_min, clamp_max, y, ldy, q_out,
+                         scale_out, zp_out);
+  c.mode = 1;
+  return launch_a8w4_tc_call(c, workspace, workspace_bytes, (cudaStream_t)stream);
 }
 
 extern "C" size_t pack_w4_g32_asym_bytes(int N, int K) {
@@ -507,21 +538,19 @@ extern "C" int pack_w4_g32_asym(int N, int K, const int8_t* w, int64_t ldw,
 extern "C" int qgemm_a8w4_f32_asym(int M, int N, int K, const float* x, int64_t ldx,
                                    const void* packed_w, const float* bias, float clamp_min,
                                    float clamp_max, float* y, int64_t ldy, int8_t* q_out,
-                                   float* scale_out, int32_t* zp_out, void* stream) {
-  if (M < 0 || N <= 0 || K <= 0 || ldx < K || ldy < N) return QG_ERR_INVALID_ARG;
-  if (K % 32) return QG_ERR_UNSUPPORTED;
-  if (!(clamp_min <= clamp_max)) return QG_ERR_INVALID_ARG;  // also rejects NaN
-  if (M == 0) return QG_OK;
-  if (M != 1) return QG_ERR_UNSUPPORTED;
-  if (!x || !packed_w || !y) return QG_ERR_INVALID_ARG;
-  if (!aligned(packed_w, 16)) return QG_ERR_MISALIGNED;
-  if (!aligned(x, 4) || !aligned(y, 4) || (bias && !aligned(bias, 4))) return QG_ERR_MISALIGNED;
-  if ((scale_out && !aligned(scale_out, 4)) || (zp_out && !aligned(zp_out, 4)))
-    return QG_ERR_MISALIGNED;
-  int rc = device_ready();
-  if (rc != QG_OK) return rc;
-  return launch_a8w4_gemv_asym(N, K, x, packed_w, bias, clamp_min, clamp_max, y, q_out,
-                               scale_out, zp_out, (cudaStream_t)stream);
+                                   float* scale_out, int32_t* zp_out, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
+  int rc = a8w4_variant_args(M, N, K, x, ldx, packed_w, bias, clamp_min, clamp_max, y, ldy,
+                             scale_out, zp_out, workspace, workspace_bytes);
+  if (rc != QG_OK || M == 0) return rc;
+  if (M == 1)
+    return launch_a8w4_gemv_asym(N, K, x, packed_w, bias, clamp_min, clamp_max, y, q_out,
+                                 scale_out, zp_out, (cudaStream_t)stream);
+  A8W4TcCall c = tc_rows(M, N, K, x, ldx, packed_w, bias, clamp_min, clamp_max, y, ldy, q_out,
+                         scale_out, zp_out);
+  c.mode = 0;
+  c.wzero = (const float*)((const uint8_t*)packed_w + pack_w4_g32_bytes(N, K));
+  return launch_a8w4_tc_call(c, workspace, workspace_bytes, (cudaStream_t)stream);
 }
 
 // ---------------------------------------------------------------------------
@@ -539,26 +568,29 @@ extern "C" int quantize_rows_a8_sym(int M, int K, const float* x, int64_t ldx, i
   return launch_quantize_rows_sym(M, K, x, ldx, q, ldq, scale, nullptr, (cudaStream_t)stream);
 }
 
-// The conv's GEMM runs on the CUDA-core A8W4 kernel: 8 unrolled rows per CTA
-// row of the grid (at most 65535 of them) and 8*K bytes of shared memory.
+// The conv's contraction runs on the tensor-core A8W4 kernel when K % 64 == 0
+// (and K <= 8192); otherwise on the CUDA-core A8W4 kernel: 8 unrolled rows
+// per CTA row of the grid (at most 65535 of them) and 8*K bytes of shared
+// memory.
 static const int64_t kDynConvMaxRows = 65535 * 8;
+static const int64_t kDynConvMaxRowsTc = (int64_t)1 << 30;
 
 // Unrolled-matrix shape of a float-input conv: QG_OK with P rows of K, or
-// the status the call returns.
+// the status the call returns; *tc tells which kernel takes it.
 static int dynconv_shape(int Nb, int H, int W, int Cin, int Cout, int KH, int KW, int sh, int sw,
-                         int ph, int pw, int64_t* P, int* K) {
+                         int ph, int pw, int64_t* P, int* K, bool* tc) {
   if (Nb <= 0 || H <= 0 || W <= 0 || Cin <= 0 || Cout <= 0 || KH <= 0 || KW <= 0 || sh <= 0 ||
       sw <= 0 || ph < 0 || pw < 0)
     return QG_ERR_INVALID_ARG;
   if ((int64_t)H + 2 * (int64_t)ph < KH || (int64_t)W + 2 * (int64_t)pw < KW)
     return QG_ERR_INVALID_ARG;
   const int64_t k = (int64_t)KH * KW * Cin;
-  if (k % 32) return QG_ERR_UNSUPPORTED;
-  if (k > kSimtMaxK) return QG_ERR_UNSUPPORTED;
+  if (k % 32 || k > INT32_MAX) return QG_ERR_UNSUPPORTED;
   const int64_t OH = ((int64_t)H + 2 * (int64_t)ph - KH) / sh + 1;
   const int64_t OW = ((int64_t)W + 2 * (int64_t)pw - KW) / sw + 1;
   const int64_t p = (int64_t)Nb * OH * OW;
-  if (p > kDynConvMaxRows) return QG_ERR_UNSUPPORTED;
+  *tc = p >= 2 && p <= kDynConvMaxRowsTc && a8w4_tc_supported(p, Cout, (int)k);
+  if (!*tc && (k > kSimtMaxK || p > kDynConvMaxRows)) return QG_ERR_UNSUPPORTED;
   *P = p;
   *K = (int)k;
   return QG_OK;
@@ -569,10 +601,11 @@ extern "C" size_t qconv2d_f32_dyn_a8w4_workspace_bytes(int Nb, int H, int W, int
                                                        int stride_w, int pad_h, int pad_w) {
   int64_t P = 0;
   int K = 0;
-  if (dynconv_shape(Nb, H, W, Cin, Cout, KH, KW, stride_h, stride_w, pad_h, pad_w, &P, &K) !=
+  bool tc = false;
+  if (dynconv_shape(Nb, H, W, Cin, Cout, KH, KW, stride_h, stride_w, pad_h, pad_w, &P, &K, &tc) !=
       QG_OK)
     return 0;
-  return a8w4_ws_layout((int)P, K, nullptr, nullptr);
+  return tc ? a8w4_tc_workspace_bytes(P, Cout, K) : a8w4_ws_layout((int)P, K, nullptr, nullptr);
 }
 
 extern "C" int qconv2d_f32_dyn_a8w4(int Nb, int H, int W, int Cin, int Cout, int KH, int KW,
@@ -583,7 +616,9 @@ extern "C" int qconv2d_f32_dyn_a8w4(int Nb, int H, int W, int Cin, int Cout, int
                                     void* workspace, size_t workspace_bytes, void* stream) {
   int64_t P = 0;
   int K = 0;
-  int rc = dynconv_shape(Nb, H, W, Cin, Cout, KH, KW, stride_h, stride_w, pad_h, pad_w, &P, &K);
+  bool tc = false;
+  int rc = dynconv_shape(Nb, H, W, Cin, Cout, KH, KW, stride_h, stride_w, pad_h, pad_w, &P, &K,
+                         &tc);
   if (rc != QG_OK) return rc;
   if (symmetric != 0 && symmetric != 1) return QG_ERR_INVALID_ARG;
   if (!(clamp_min <= clamp_max)) return QG_ERR_INVALID_ARG;  // also rejects NaN
@@ -592,6 +627,22 @@ extern "C" int qconv2d_f32_dyn_a8w4(int Nb, int H, int W, int Cin, int Cout, int
   if (!aligned(x, 4) || !aligned(y, 4) || (bias && !aligned(bias, 4))) return QG_ERR_MISALIGNED;
   if ((scale_out && !aligned(scale_out, 4)) || (zp_out && !aligned(zp_out, 4)))
     return QG_ERR_MISALIGNED;
+  if (tc) {
+    if (!workspace) return QG_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return QG_ERR_MISALIGNED;
+    rc = device_ready();
+    if (rc != QG_OK) return rc;
+    const int OH = (int)(((int64_t)H + 2 * (int64_t)pad_h - KH) / stride_h + 1);
+    const int OW = (int)(((int64_t)W + 2 * (int64_t)pad_w - KW) / stride_w + 1);
+    A8W4TcCall c{};
+    c.M = P; c.N = Cout; c.K = K; c.x = x; c.ldx = 0; c.conv = true;
+    c.H = H; c.W = W; c.Cin = Cin; c.KH = KH; c.KW = KW; c.sh = stride_h; c.sw = stride_w;
+    c.ph = pad_h; c.pw = pad_w; c.OH = OH; c.OW = OW;
+    c.mode = symmetric ? 2 : 0;
+    c.packed = packed_w; c.bias = bias; c.lo = clamp_min; c.hi = clamp_max;
+    c.y = y; c.ldy = Cout; c.q_out = q_out; c.scale_out = scale_out; c.zp_out = zp_out;
+    return launch_a8w4_tc_call(c, workspace, workspace_bytes, (cudaStream_t)stream);
+  }
   size_t off_s = 0, off_z = 0;
   const size_t need = a8w4_ws_layout((int)P, K, &off_s, &off_z);
   if (!workspace || workspace_bytes < need) return QG_ERR_WORKSPACE;

@@ -159,6 +159,79 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 }
 
 // ---------------------------------------------------------------------------
+// Dynamic activation quantization (MNN BatchAsyDynamicQuant / BatchSym-
+// DynamicQuant; ONNX QuantizeLinear rounding, half to even).  All float32,
+// one IEEE rounding per operation, no contraction.
+//   asymmetric: rmin = min(0, min x), rmax = max(0, max x),
+//     scale = (rmax-rmin)/255 (1 if 0), inv = 1/scale,
+//     zp = clamp(rne(-128 - rmin*inv), -128, 127), q = clamp(rne(x*inv)+zp)
+//   symmetric: amax = max|x|, scale = amax/127, inv = 127/amax (both 1 when
+//     amax is 0), zp = 0, q = clamp(rne(x*inv), -127, 127)
+// ---------------------------------------------------------------------------
+struct RowQuant {
+  float scale, inv;
+  int zp;
+};
+
+__device__ __forceinline__ RowQuant row_quant_params(float rmin, float rmax) {
+  RowQuant r;
+  float s = __fdiv_rn(__fsub_rn(rmax, rmin), 255.0f);
+  if (s == 0.0f) s = 1.0f;
+  r.scale = s;
+  r.inv = __fdiv_rn(1.0f, s);
+  float t = __fsub_rn(-128.0f, __fmul_rn(rmin, r.inv));
+  int z = __float2int_rn(t);
+  r.zp = min(max(z, -128), 127);
+  return r;
+}
+
+__device__ __forceinline__ int quant_one(float x, const RowQuant& r) {
+  int v = __float2int_rn(__fmul_rn(x, r.inv)) + r.zp;
+  return min(max(v, -128), 127);
+}
+
+__device__ __forceinline__ RowQuant row_quant_params_sym(float amax) {
+  RowQuant r;
+  r.scale = amax == 0.0f ? 1.0f : __fdiv_rn(amax, 127.0f);
+  r.inv = amax == 0.0f ? 1.0f : __fdiv_rn(127.0f, amax);
+  r.zp = 0;
+  return r;
+}
+
+__device__ __forceinline__ int quant_one_sym(float x, const RowQuant& r) {
+  return min(max(__float2int_rn(__fmul_rn(x, r.inv)), -127), 127);
+}
+
+// ---------------------------------------------------------------------------
+// One call of the tensor-core A8W4 path (a8w4_tc.cu).  Activation rows are
+// plain rows x[M][ldx], or (conv) the unrolled rows of an NHWC image.  mode
+// 0: per-row asymmetric, 1: per-32-block asymmetric, 2: per-row symmetric
+// quantization; wzero selects asymmetric weights (f32 zeros [N][K/32]).
+// ---------------------------------------------------------------------------
+struct A8W4TcCall {
+  int64_t M;
+  int N, K;
+  const float* x;
+  int64_t ldx;
+  bool conv;
+  int H, W, Cin, KH, KW, sh, sw, ph, pw, OH, OW;
+  int mode;
+  const void* packed;
+  bool scale_bf16;
+  const float* wzero;
+  const float* bias;
+  float lo, hi;
+  float* y;
+  int64_t ldy;
+  int8_t* q_out;
+  float* scale_out;
+  int32_t* zp_out;
+};
+bool a8w4_tc_supported(int64_t M, int N, int K);
+size_t a8w4_tc_workspace_bytes(int64_t M, int N, int K);
+int launch_a8w4_tc_call(const A8W4TcCall& c, void* ws, size_t ws_bytes, cudaStream_t st);
+
+// ---------------------------------------------------------------------------
 // Integer dot products
 // ---------------------------------------------------------------------------
 // sum_b a.u8[b] * b.s8[b] + c  (a unsigned bytes, b signed bytes)

@@ -38,7 +38,7 @@
 extern "C" {
 #endif
 
-#define QG_API_VERSION 1
+#define QG_API_VERSION 2
 
 typedef enum {
   QG_OK = 0,
@@ -243,11 +243,13 @@ int pack_w4_g32(int N, int K, const int8_t* w, int64_t ldw,
  * so that it may start while the previous M == 1 call on the same stream is
  * still finishing: it reads packed_w (never x or bias) before that call has
  * completed.  So packed_w must not be written by the M == 1 call just before
- * it on the stream; every other ordering is kept as usual.  M > 1
- * quantizes into the workspace, then runs the tensor-core kernel (K % 128 == 0
- * and N % 4 == 0; exact per-group integer dots from bf16 MMAs, f32 group
- * combination, split-K partials reduced in a fixed order), otherwise a
- * CUDA-core kernel.
+ * it on the stream; every other ordering is kept as usual.  M > 1 with
+ * K % 64 == 0 and K <= 8192 runs two kernels: the rows are quantized into
+ * the workspace as bf16 tiles of qA - zA, then the tensor-core kernel forms
+ * the exact per-group integer dots with bf16 MMAs, combines the groups in
+ * float32 and reduces split-K partials in a fixed order.  Other M > 1 shapes
+ * (K <= 25600) run a CUDA-core kernel.  q_out must then be writable as bytes
+ * (any alignment).
  * ------------------------------------------------------------------------ */
 size_t qgemm_a8w4_workspace_bytes(int M, int N, int K);
 int qgemm_a8w4_f32(int M, int N, int K, const float* x, int64_t ldx,
@@ -282,43 +284,46 @@ int qgemm_a8w4_f32_bf16s(int M, int N, int K, const float* x, int64_t ldx,
                          void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
- * A8W4 GEMV with the activations quantized per K block.  [MNN]
+ * A8W4 linear with the activations quantized per K block.  [MNN]
  * ConvInt8TiledExecutor, dynamic-quant option 2: the input is quantized in as
  * many K blocks as the weights have quant blocks, each block with its own
  * scale and zero-point.  Here a block is one 32-wide weight group:
- *   y[n] = clamp(sum_g sw[n,g] * sA[g] * I[n,g] + bias[n])
- *   I[n,g] = sum_{k in g} (qA[k] - zA[g]) * w[n,k]      (exact integer)
- * with sA[g], zA[g] from the per-row rule of quantize_rows_a8 applied to the
- * 32 values of block g, and the group combination in float32.
- *   M must be 1 (else QG_ERR_UNSUPPORTED); K % 128 == 0, K <= 8192 and x
- *   16-byte aligned (else QG_ERR_UNSUPPORTED); packed_w from pack_w4_g32
- *   (f32 group scales).  q_out [K] int8, scale_out [K/32] f32 and
- *   zp_out [K/32] int32 are optional.  No workspace.  The same stream note
- *   as qgemm_a8w4_f32 (M == 1) applies: packed_w may be read before the
- *   previous M == 1 call on the stream has completed.
+ *   y[m,n] = clamp(sum_g sw[n,g] * sA[m,g] * I[m,n,g] + bias[n])
+ *   I[m,n,g] = sum_{k in g} (qA[m,k] - zA[m,g]) * w[n,k]   (exact integer)
+ * with sA[m,g], zA[m,g] from the per-row rule of quantize_rows_a8 applied to
+ * the 32 values of block g of row m, and the group combination in float32.
+ *   packed_w from pack_w4_g32 (f32 group scales).  q_out [M][K] int8,
+ *   scale_out [M][K/32] f32 and zp_out [M][K/32] int32 are optional.
+ *   M == 1: K % 128 == 0, K <= 8192 and x 16-byte aligned (else
+ *   QG_ERR_UNSUPPORTED); no workspace; the stream note of qgemm_a8w4_f32
+ *   (M == 1) applies.  M > 1: K % 64 == 0 and K <= 8192 (else
+ *   QG_ERR_UNSUPPORTED), the tensor-core path of qgemm_a8w4_f32 with a
+ *   workspace of qgemm_a8w4_workspace_bytes(M, N, K) bytes, 256-byte aligned.
  * ------------------------------------------------------------------------ */
 int qgemm_a8w4_f32_actblock(int M, int N, int K, const float* x, int64_t ldx,
                             const void* packed_w, const float* bias,
                             float clamp_min, float clamp_max,
                             float* y, int64_t ldy,
                             int8_t* q_out, float* scale_out, int32_t* zp_out,
-                            void* stream);
+                            void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
- * A8W4 GEMV with asymmetric int4 weights.  [MNN] ConvInt8TiledExecutor,
+ * A8W4 linear with asymmetric int4 weights.  [MNN] ConvInt8TiledExecutor,
  * asymmetric quant info: every (output channel, block) carries a zero and an
  * alpha, and a weight is alpha * code + zero.  Here:
  *   w_real[n,k] = sw[n,g] * w[n,k] + zw[n,g]     (w in [-8,7], g = k/32)
- *   y[n] = clamp(sA * sum_g (sw[n,g]*I[n,g] + zw[n,g]*S[g]) + bias[n])
- *   I[n,g] = sum_{k in g} (qA[k] - zA) * w[n,k],  S[g] = sum_{k in g} (qA[k] - zA)
+ *   y[m,n] = clamp(sA[m] * sum_g (sw[n,g]*I[m,n,g] + zw[n,g]*S[m,g]) + bias[n])
+ *   I[m,n,g] = sum_{k in g} (qA[m,k] - zA[m]) * w[n,k],
+ *   S[m,g] = sum_{k in g} (qA[m,k] - zA[m])
  * (I and S exact integers, the combination in float32).
  *   pack_w4_g32_asym: pack_w4_g32's layout followed by the f32 zeros
  *   zw[N][K/32] (row-major, contiguous), copied as given; size from
  *   pack_w4_g32_asym_bytes (0 when K % 32 != 0).  Checks as pack_w4_g32,
  *   plus group_zeros non-NULL and 4-byte aligned.
- *   qgemm_a8w4_f32_asym: M must be 1, K % 128 == 0, K <= 8192 and x 16-byte
- *   aligned (else QG_ERR_UNSUPPORTED); arguments and outputs as
- *   qgemm_a8w4_f32 for M == 1, no workspace, and the same stream note.
+ *   qgemm_a8w4_f32_asym: arguments and outputs as qgemm_a8w4_f32.  M == 1:
+ *   K % 128 == 0, K <= 8192 and x 16-byte aligned (else QG_ERR_UNSUPPORTED),
+ *   no workspace, the same stream note.  M > 1: K % 64 == 0 and K <= 8192
+ *   (else QG_ERR_UNSUPPORTED), a workspace of qgemm_a8w4_workspace_bytes.
  * ------------------------------------------------------------------------ */
 size_t pack_w4_g32_asym_bytes(int N, int K);
 int pack_w4_g32_asym(int N, int K, const int8_t* w, int64_t ldw, const float* group_scales,
@@ -328,7 +333,7 @@ int qgemm_a8w4_f32_asym(int M, int N, int K, const float* x, int64_t ldx,
                         float clamp_min, float clamp_max,
                         float* y, int64_t ldy,
                         int8_t* q_out, float* scale_out, int32_t* zp_out,
-                        void* stream);
+                        void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
  * Dynamic per-row symmetric int8 activation quantization.  [MNN]
@@ -367,7 +372,10 @@ int quantize_rows_a8_sym(int M, int K, const float* x, int64_t ldx,
  * as qgemm_a8w4_f32.  q_out [P][K] int8 / scale_out [P] / zp_out [P] int32
  * (P = Nb*OH*OW): optional, receive the unrolled row quantization.
  * Workspace: qconv2d_f32_dyn_a8w4_workspace_bytes (256-byte aligned).
- * Limits: K <= 25600 and P <= 524280 (else QG_ERR_UNSUPPORTED).
+ * With K % 64 == 0, K <= 8192 and P >= 2 the rows are unrolled and quantized
+ * straight into the tensor-core tiles of qgemm_a8w4_f32 (two kernels);
+ * otherwise they are unrolled into the workspace for the CUDA-core kernel,
+ * with the limits K <= 25600 and P <= 524280 (else QG_ERR_UNSUPPORTED).
  * ------------------------------------------------------------------------ */
 size_t qconv2d_f32_dyn_a8w4_workspace_bytes(int Nb, int H, int W, int Cin, int Cout,
                                             int KH, int KW, int stride_h, int stride_w,

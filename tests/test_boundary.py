@@ -29,7 +29,7 @@ def test_exports_every_declared_symbol():
 
 
 def test_status_strings_and_version():
-    assert lib.qg_version() == 1
+    assert lib.qg_version() == 2
     for code, name in qg.STATUS.items():
         assert lib.qg_status_string(code).decode().startswith(name)
     assert lib.qg_status_string(12345).decode() == "QG_ERR_UNKNOWN"
@@ -145,11 +145,19 @@ def test_bf16_scale_entry_points_validate_like_f32_ones():
 
 def test_actblock_gemv_validation():
     f = lib.qgemm_a8w4_f32_actblock
-    assert f(2, 8, 128, FAKE, 128, FAKE, NULL, -1.0, 1.0, FAKE, 8, NULL, NULL, NULL, NULL) == -4  # M != 1
-    assert f(1, 8, 48, FAKE, 48, FAKE, NULL, -1.0, 1.0, FAKE, 8, NULL, NULL, NULL, NULL) == -4    # K % 32
-    assert f(1, 8, 128, FAKE, 128, FAKE, NULL, 1.0, -1.0, FAKE, 8, NULL, NULL, NULL, NULL) == -1  # lo > hi
-    assert f(1, 8, 128, FAKE, 127, FAKE, NULL, -1.0, 1.0, FAKE, 8, NULL, NULL, NULL, NULL) == -1  # ldx < K
-    assert f(0, 8, 128, FAKE, 128, FAKE, NULL, -1.0, 1.0, FAKE, 8, NULL, NULL, NULL, NULL) == 0   # empty
+    args = (FAKE, NULL, -1.0, 1.0, FAKE, 8, NULL, NULL, NULL)
+    assert f(2, 8, 96, FAKE, 96, *args, FAKE, 1 << 20, NULL) == -4      # M > 1, K % 64 != 0
+    assert f(2, 8, 16384, FAKE, 16384, *args, FAKE, 1 << 30, NULL) == -4  # M > 1, K > 8192
+    assert f(2, 8, 128, FAKE, 128, *args, NULL, 0, NULL) == -7         # M > 1 needs a workspace
+    need = lib.qgemm_a8w4_workspace_bytes(2, 8, 128)
+    assert need > 0
+    assert f(2, 8, 128, FAKE, 128, *args, FAKE, need - 1, NULL) == -7  # too small
+    assert f(2, 8, 128, FAKE, 128, *args, ctypes.c_void_p(0x10010), need, NULL) == -2
+    assert f(1, 8, 96, FAKE, 96, *args, NULL, 0, NULL) == -4           # M == 1, K % 128
+    assert f(1, 8, 48, FAKE, 48, *args, NULL, 0, NULL) == -4           # K % 32
+    assert f(1, 8, 128, FAKE, 128, FAKE, NULL, 1.0, -1.0, FAKE, 8, NULL, NULL, NULL, NULL, 0, NULL) == -1
+    assert f(1, 8, 128, FAKE, 127, *args, NULL, 0, NULL) == -1         # ldx < K
+    assert f(0, 8, 128, FAKE, 128, *args, NULL, 0, NULL) == 0          # empty
 
 
 def test_asym_entry_points_validation():
@@ -161,9 +169,12 @@ def test_asym_entry_points_validation():
     assert p(4, 64, FAKE, 64, FAKE, ctypes.c_void_p(0x10002), FAKE, 1 << 20, NULL) == -2
     assert p(4, 64, FAKE, 64, FAKE, FAKE, FAKE, 4 * 32 + 2 * 4 * 2 * 4 - 1, NULL) == -7
     f = lib.qgemm_a8w4_f32_asym
-    assert f(2, 8, 128, FAKE, 128, FAKE, NULL, -1.0, 1.0, FAKE, 8, NULL, NULL, NULL, NULL) == -4
-    assert f(1, 8, 128, FAKE, 128, FAKE, NULL, 1.0, -1.0, FAKE, 8, NULL, NULL, NULL, NULL) == -1
-    assert f(0, 8, 128, FAKE, 128, FAKE, NULL, -1.0, 1.0, FAKE, 8, NULL, NULL, NULL, NULL) == 0
+    args = (FAKE, NULL, -1.0, 1.0, FAKE, 8, NULL, NULL, NULL)
+    assert f(2, 8, 96, FAKE, 96, *args, FAKE, 1 << 20, NULL) == -4      # M > 1, K % 64 != 0
+    assert f(2, 8, 128, FAKE, 128, *args, NULL, 0, NULL) == -7         # M > 1 needs a workspace
+    assert f(1, 8, 96, FAKE, 96, *args, NULL, 0, NULL) == -4           # M == 1, K % 128
+    assert f(1, 8, 128, FAKE, 128, FAKE, NULL, 1.0, -1.0, FAKE, 8, NULL, NULL, NULL, NULL, 0, NULL) == -1
+    assert f(0, 8, 128, FAKE, 128, *args, NULL, 0, NULL) == 0
 
 
 def test_symmetric_quantization_validation():

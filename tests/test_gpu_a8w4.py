@@ -121,7 +121,7 @@ def _check_a8w4(lib, w, bf16=False, **kw):
     np.testing.assert_array_equal(s.view(np.int32), s_ref.view(np.int32))
     np.testing.assert_array_equal(z, z_ref)
     M, N, K = w["M"], w["N"], w["K"]
-    kind = "gemv" if M == 1 else ("tc" if K % 128 == 0 and N % 4 == 0 else "simt")
+    kind = "gemv" if M == 1 else ("tc" if K % 64 == 0 and K <= 8192 else "simt")
     assert_a8w4_close(y, y_ref, f"a8w4{'_bf16s' if bf16 else ''} {kind} {M}x{N}x{K}")
     return y, y_ref
 
@@ -220,13 +220,13 @@ def test_a8w4_bf16_scales_full_size_128x4096x4096(lib):
 # A8W4 GEMV with the activations quantized per 32-wide K block
 # ---------------------------------------------------------------------------
 def _check_actblock(lib, w):
-    N, K = w["N"], w["K"]
+    M, N, K = w["M"], w["N"], w["K"]
     packed = lib.pack_w4_g32(_dev(w["qw"]), _dev(w["sw"]))
     x = _dev(w["x"])[:, :K]
-    y = torch.full((1, N + 1), 7.0, dtype=torch.float32, device="cuda")
-    q = torch.empty((1, K), dtype=torch.int8, device="cuda")
-    s = torch.empty(K // 32, dtype=torch.float32, device="cuda")
-    z = torch.empty(K // 32, dtype=torch.int32, device="cuda")
+    y = torch.full((M, N + 1), 7.0, dtype=torch.float32, device="cuda")
+    q = torch.empty((M, K), dtype=torch.int8, device="cuda")
+    s = torch.empty((M, K // 32), dtype=torch.float32, device="cuda")
+    z = torch.empty((M, K // 32), dtype=torch.int32, device="cuda")
     bias = None if w["bias"] is None else _dev(w["bias"])
     lib.qgemm_a8w4_f32_actblock(x, packed, N, bias, w["clamp_min"], w["clamp_max"], y[:, :N],
                                 q, s, z)
@@ -234,11 +234,11 @@ def _check_actblock(lib, w):
     y_ref, q_ref, s_ref, z_ref = oracle.qgemm_a8w4_f32_actblock(
         w["x"][:, :K], w["qw"], w["sw"], w["bias"], w["clamp_min"], w["clamp_max"])
     np.testing.assert_array_equal(q.cpu().numpy(), q_ref)
-    np.testing.assert_array_equal(s.cpu().numpy().view(np.int32), s_ref[0].view(np.int32))
-    np.testing.assert_array_equal(z.cpu().numpy(), z_ref[0])
+    np.testing.assert_array_equal(s.cpu().numpy().view(np.int32), s_ref.view(np.int32))
+    np.testing.assert_array_equal(z.cpu().numpy(), z_ref)
     y_np = y.cpu().numpy()
     assert (y_np[:, N:] == 7.0).all()
-    assert_a8w4_close(y_np[:, :N], y_ref, f"actblock 1x{N}x{K}")
+    assert_a8w4_close(y_np[:, :N], y_ref, f"actblock {'gemv' if M == 1 else 'tc'} {M}x{N}x{K}")
 
 
 def test_gemv_actblock_full_size_1x14336x4096(lib):
@@ -255,15 +255,32 @@ def test_gemv_actblock_shapes(lib, N, K):
     _check_actblock(lib, w)
 
 
+def test_a8w4_actblock_full_size_128x4096x4096(lib):
+    _check_actblock(lib, workloads.a8w4_gemm_128x4096x4096())
+
+
+@pytest.mark.parametrize("M,N,K", [(2, 64, 64), (9, 300, 1024), (17, 1000, 4096),
+                                   (129, 520, 384), (200, 132, 128), (3, 4096, 8192)])
+def test_a8w4_actblock_gemm_shapes(lib, M, N, K):
+    w = workloads.a8w4(M, N, K, seed=M * 17 + N + K, clamp=(-np.inf, np.inf), ldx=K + 1)
+    # blocks of magnitudes 10^-2 .. 10^0 (a 1000x spread); with a 10^5 spread
+    # the float32 group sum of y near 0 cancels terms of size 10^3 and its
+    # absolute error reaches ~1e-4 on any float32 path
+    scale = np.float32(10.0) ** np.random.default_rng(M + N).integers(-2, 1, (M, K // 32))
+    w["x"][:, :K] *= np.repeat(scale, 32, axis=1)
+    w["x"][0, 32:64] = 0.0                                 # a zero block
+    _check_actblock(lib, w)
+
+
 def test_gemv_actblock_rejects_what_it_does_not_cover(lib):
-    w = workloads.a8w4(2, 64, 256, seed=1)
-    packed = lib.pack_w4_g32(_dev(w["qw"]), _dev(w["sw"]))
     y = torch.empty((2, 64), dtype=torch.float32, device="cuda")
-    with pytest.raises(lib.QGError):                       # M != 1
-        lib.qgemm_a8w4_f32_actblock(_dev(w["x"])[:, :256], packed, 64, None, -1.0, 1.0, y)
+    w = workloads.a8w4(2, 64, 96, seed=1)
+    packed = lib.pack_w4_g32(_dev(w["qw"]), _dev(w["sw"]))
+    with pytest.raises(lib.QGError):                       # M > 1 with K % 64 != 0
+        lib.qgemm_a8w4_f32_actblock(_dev(w["x"])[:, :96], packed, 64, None, -1.0, 1.0, y)
     w = workloads.a8w4(1, 64, 96, seed=2)
     packed = lib.pack_w4_g32(_dev(w["qw"]), _dev(w["sw"]))
-    with pytest.raises(lib.QGError):                       # K % 128 != 0
+    with pytest.raises(lib.QGError):                       # M == 1 with K % 128 != 0
         lib.qgemm_a8w4_f32_actblock(_dev(w["x"])[:, :96], packed, 64, None, -1.0, 1.0, y[:1])
 
 
@@ -276,16 +293,16 @@ def _asym_zeros(w, seed):
 
 
 def _check_asym(lib, w, zw):
-    N, K = w["N"], w["K"]
+    M, N, K = w["M"], w["N"], w["K"]
     packed = lib.pack_w4_g32_asym(_dev(w["qw"]), _dev(w["sw"]), _dev(zw))
     torch.cuda.synchronize()
     np.testing.assert_array_equal(packed.cpu().numpy(),
                                   oracle.pack_w4_g32_asym(w["qw"], w["sw"], zw))
     x = _dev(w["x"])[:, :K]
-    y = torch.full((1, N + 1), 7.0, dtype=torch.float32, device="cuda")
-    q = torch.empty((1, K), dtype=torch.int8, device="cuda")
-    s = torch.empty(1, dtype=torch.float32, device="cuda")
-    z = torch.empty(1, dtype=torch.int32, device="cuda")
+    y = torch.full((M, N + 1), 7.0, dtype=torch.float32, device="cuda")
+    q = torch.empty((M, K), dtype=torch.int8, device="cuda")
+    s = torch.empty(M, dtype=torch.float32, device="cuda")
+    z = torch.empty(M, dtype=torch.int32, device="cuda")
     bias = None if w["bias"] is None else _dev(w["bias"])
     lib.qgemm_a8w4_f32_asym(x, packed, N, bias, w["clamp_min"], w["clamp_max"], y[:, :N], q, s, z)
     torch.cuda.synchronize()
@@ -296,7 +313,7 @@ def _check_asym(lib, w, zw):
     np.testing.assert_array_equal(z.cpu().numpy(), z_ref)
     y_np = y.cpu().numpy()
     assert (y_np[:, N:] == 7.0).all()
-    assert_a8w4_close(y_np[:, :N], y_ref, f"asym 1x{N}x{K}")
+    assert_a8w4_close(y_np[:, :N], y_ref, f"asym {'gemv' if M == 1 else 'tc'} {M}x{N}x{K}")
 
 
 def test_gemv_asym_full_size_1x14336x4096(lib):
@@ -308,6 +325,18 @@ def test_gemv_asym_full_size_1x14336x4096(lib):
 def test_gemv_asym_shapes(lib, N, K):
     w = workloads.a8w4(1, N, K, seed=N * 5 + K, clamp=(-np.inf, np.inf), ldx=K + 3)
     _check_asym(lib, w, _asym_zeros(w, N + K))
+
+
+def test_a8w4_asym_full_size_128x4096x4096(lib):
+    w = workloads.a8w4_gemm_128x4096x4096()
+    _check_asym(lib, w, _asym_zeros(w, 33))
+
+
+@pytest.mark.parametrize("M,N,K", [(2, 64, 64), (9, 300, 1024), (17, 1000, 4096),
+                                   (129, 520, 384), (200, 132, 128), (3, 4096, 8192)])
+def test_a8w4_asym_gemm_shapes(lib, M, N, K):
+    w = workloads.a8w4(M, N, K, seed=M * 19 + N + K, clamp=(-np.inf, np.inf), ldx=K + 1)
+    _check_asym(lib, w, _asym_zeros(w, M + N + K))
 
 
 def test_gemv_asym_with_zero_zeros_matches_symmetric_entry(lib):

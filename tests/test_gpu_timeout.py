@@ -14,6 +14,7 @@ import pytest
 
 import oracle
 import workloads
+from a8w4_tol import assert_a8w4_close
 
 pytestmark = pytest.mark.gpu
 torch = pytest.importorskip("torch")
@@ -66,3 +67,21 @@ def test_stall_hook_is_one_shot_and_disarmable(lib, cuda):
     assert lib.qg_device_status(True) == 0
     with pytest.raises(lib.QGError):
         lib.qg_test_arm_stall(7)
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 512, 4096), (20, 300, 1024)])
+def test_a8w4_tc_stalled_pipeline_times_out_then_recovers(lib, cuda, M, N, K):
+    lib.qg_device_status(True)
+    w = workloads.a8w4(M, N, K, seed=M + N, clamp=(-np.inf, np.inf))
+    packed = lib.pack_w4_g32(_dev(w["qw"]), _dev(w["sw"]))
+    x = _dev(w["x"])
+    bias = _dev(w["bias"])
+    y = torch.zeros((M, N), dtype=torch.float32, device="cuda")
+    lib.qg_test_arm_stall(2)
+    lib.qgemm_a8w4_f32(x, packed, N, bias, -np.inf, np.inf, y)
+    assert lib.qg_device_status(True) == QG_ERR_TIMEOUT
+    lib.qgemm_a8w4_f32(x, packed, N, bias, -np.inf, np.inf, y)
+    torch.cuda.synchronize()
+    y_ref = oracle.qgemm_a8w4_f32(w["x"], w["qw"], w["sw"], w["bias"], -np.inf, np.inf)[0]
+    assert_a8w4_close(y.cpu().numpy(), y_ref, f"a8w4 tc after a stall {M}x{N}x{K}")
+    assert lib.qg_device_status(True) == 0
