@@ -84,6 +84,10 @@ _sig("qgemm_s8s8_requant_packed", _i32, [_i32, _i32, _i32, _vp, _i64, _vp, _vp, 
 _sig("qconv2d_s8_workspace_bytes", _sz, [_i32] * 11)
 _sig("qconv2d_s8_im2col", _i32, [_i32] * 11 + [_vp, _vp, _vp, ctypes.POINTER(RequantParams),
                                                _vp, _vp, _sz, _vp])
+_sig("qconv2d_s8_pack_w_bytes", _sz, [_i32] * 4)
+_sig("qconv2d_s8_pack_w", _i32, [_i32] * 4 + [_vp, _vp, _sz, _vp])
+_sig("qconv2d_s8_im2col_packed", _i32, [_i32] * 11 + [_vp, _vp, _vp, ctypes.POINTER(RequantParams),
+                                                      _vp, _vp])
 _sig("quantize_rows_a8", _i32, [_i32, _i32, _vp, _i64, _vp, _i64, _vp, _vp, _vp])
 _sig("pack_w4_g32_bytes", _sz, [_i32, _i32])
 _sig("pack_w4_g32", _i32, [_i32, _i32, _vp, _i64, _vp, _vp, _sz, _vp])
@@ -350,6 +354,29 @@ def qconv2d_s8_im2col(x, w, y, rq, stride, pad, acc_out=None, workspace=None, st
                                  pad[1], _p(x), _p(w), _p(y), ctypes.byref(rq), _p(acc_out),
                                  _p(workspace), workspace.numel(), _stream(stream)),
            "qconv2d_s8_im2col")
+
+
+def qconv2d_s8_pack_w(w, packed=None, stream=None):
+    """Pack conv weights [Cout][KH][KW][Cin] once (weights-stationary)."""
+    Cout, KH, KW, Cin = w.shape
+    assert w.is_contiguous()
+    if packed is None:
+        packed = _empty_bytes(lib.qconv2d_s8_pack_w_bytes(Cout, KH, KW, Cin), w.device)
+    _check(lib.qconv2d_s8_pack_w(Cout, KH, KW, Cin, _p(w), _p(packed), packed.numel(),
+                                 _stream(stream)), "qconv2d_s8_pack_w")
+    return packed
+
+
+def qconv2d_s8_im2col_packed(x, packed_w, w_shape, y, rq, stride, pad, acc_out=None,
+                             stream=None):
+    """INT8 conv from weights packed by qconv2d_s8_pack_w (one launch)."""
+    Nb, H, W, Cin = x.shape
+    Cout, KH, KW, Cin2 = w_shape
+    assert Cin == Cin2 and x.is_contiguous() and y.is_contiguous()
+    _check(lib.qconv2d_s8_im2col_packed(Nb, H, W, Cin, Cout, KH, KW, stride[0], stride[1], pad[0],
+                                        pad[1], _p(x), _p(packed_w), _p(y), ctypes.byref(rq),
+                                        _p(acc_out), _stream(stream)),
+           "qconv2d_s8_im2col_packed")
 
 
 def quantize_rows_a8_sym(x, q, scale, stream=None):

@@ -617,28 +617,43 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int q = warp & 3;                         // TMEM lane quarter
     const int cb = (warp - EPI_WARP0) >> 2;         // 64-column half
     const int nl = 32 * q + lane;                   // weight row within the tile
-    // group scales (and zeros) of this CTA's rows and K range, as [g][n]
-    for (int i = etid; i < Gr * TW; i += NEPI) {
-      const int g = i / TW, n = i - g * TW;
-      const int64_t idx = (int64_t)(n0 + n) * G + g0 + g;
-      float v = 0.0f, z = 0.0f;
-      if (n0 + n < a.N) {
-        v = a.scale_bf16
-                ? __uint_as_float((uint32_t)__ldg(reinterpret_cast<const unsigned short*>(a.wscale) + idx) << 16)
-                : __ldg(reinterpret_cast<const float*>(a.wscale) + idx);
-        if (WZP) z = __ldg(a.wzero + idx);
+    // Group scales (and zeros) of this CTA's rows and K range, as [g][n]:
+    // thread (row r, half h) reads groups [16h, 16h + 16) of row r, all its
+    // loads issued before any is used (one memory round trip, not sixteen).
+    {
+      const int r = etid & (TW - 1), h = etid >> 7;
+      const int64_t base = (int64_t)(n0 + r) * G + g0 + 16 * h;
+      const bool row_ok = n0 + r < a.N;
+      float v[16], z[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const bool in = row_ok && 16 * h + j < Gr;
+        v[j] = !in ? 0.0f
+                   : a.scale_bf16
+                         ? __uint_as_float((uint32_t)__ldg(reinterpret_cast<const unsigned short*>(a.wscale) + base + j) << 16)
+                         : __ldg(reinterpret_cast<const float*>(a.wscale) + base + j);
+        z[j] = (WZP && in) ? __ldg(a.wzero + base + j) : 0.0f;
       }
-      scl[i] = v;
-      if (WZP) zws[i] = z;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        if (16 * h + j < Gr) {
+          scl[(16 * h + j) * TW + r] = v[j];
+          if (WZP) zws[(16 * h + j) * TW + r] = z[j];
+        }
+      }
     }
     // activation scales per block / group sums come from the quantization grid
     asm volatile("griddepcontrol.wait;" ::: "memory");
     if (ABLK || WZP) {
       const float* src = ABLK ? a.sA : a.Sg;
-      for (int i = etid; i < Gr * TM; i += NEPI) {
-        const int g = i / TM, mm = i - g * TM;
-        actp[i] = src[(int64_t)(m0 + mm) * G + g0 + g];
-      }
+      const int r = etid & (TM - 1), h = etid >> 7;
+      const float* p = src + (int64_t)(m0 + r) * G + g0 + 16 * h;
+      float v[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) v[j] = 16 * h + j < Gr ? p[j] : 0.0f;
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        if (16 * h + j < Gr) actp[(16 * h + j) * TM + r] = v[j];
     }
     bar_sync<1, NEPI>();
     f32x2 acc[32];
@@ -714,15 +729,22 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int m = m0 + mm, n = n0 + 4 * c;
       if (m >= a.M || n >= a.N) continue;
       const uint32_t off = (uint32_t)((mm * PST + 4 * c) * 4);
-      float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int j = 0; j < a.splits; ++j) {
-        const float4 t = ld_dsmem_f4(mapa(part_s + off, (uint32_t)j));
-        sum.x = __fadd_rn(sum.x, t.x);
-        sum.y = __fadd_rn(sum.y, t.y);
-        sum.z = __fadd_rn(sum.z, t.z);
-        sum.w = __fadd_rn(sum.w, t.w);
-      }
+      // every rank's partial requested before the first is added
+      float4 t[MAX_SPLITS];
+#pragma unroll
+      for (int j = 0; j < MAX_SPLITS; ++j)
+        if (j < a.splits) t[j] = ld_dsmem_f4(mapa(part_s + off, (uint32_t)j));
       const float s = ABLK ? 1.0f : a.sA[m];
+      float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int j = 0; j < MAX_SPLITS; ++j) {
+        if (j < a.splits) {
+          sum.x = __fadd_rn(sum.x, t[j].x);
+          sum.y = __fadd_rn(sum.y, t[j].y);
+          sum.z = __fadd_rn(sum.z, t[j].z);
+          sum.w = __fadd_rn(sum.w, t[j].w);
+        }
+      }
       float t4[4] = {sum.x, sum.y, sum.z, sum.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {

@@ -45,6 +45,11 @@ size_t i8gemm_packed_workspace_bytes(int M, int K);
 int i8gemm_run_packed(int M, int N, int K, const int8_t* A, int64_t lda, const void* packed_b,
                       int8_t* C, int64_t ldc, const qg_requant_t& rq, int32_t* acc_out,
                       int64_t ld_acc, void* ws, size_t ws_bytes, cudaStream_t st);
+size_t conv_pack_w_bytes(int Cout, int K);
+int conv_pack_w(int Cout, int K, const int8_t* w, void* packed, cudaStream_t st);
+int conv_run_packed(int Nb, int H, int W, int Cin, int Cout, int KH, int KW, int sh, int sw,
+                    int ph, int pw, const int8_t* x, const void* packed_w, int8_t* y,
+                    const qg_requant_t& rq, int32_t* acc_out, cudaStream_t st);
 size_t conv_workspace_bytes(int Nb, int H, int W, int Cin, int Cout, int KH, int KW, int sh,
                             int sw, int ph, int pw);
 int conv_run(int Nb, int H, int W, int Cin, int Cout, int KH, int KW, int sh, int sw, int ph,
@@ -295,23 +300,71 @@ extern "C" size_t qconv2d_s8_workspace_bytes(int Nb, int H, int W, int Cin, int 
   return conv_workspace_bytes(Nb, H, W, Cin, Cout, KH, KW, stride_h, stride_w, pad_h, pad_w);
 }
 
+// Checks shared by both conv entry points (everything but the weights).
+static int conv_args(int Nb, int H, int W, int Cin, int Cout, int KH, int KW, int stride_h,
+                     int stride_w, int pad_h, int pad_w, const int8_t* x, const int8_t* y,
+                     const qg_requant_t* rq, int32_t* acc_out) {
+  if (Nb <= 0 || H <= 0 || W <= 0 || Cin <= 0 || Cout <= 0 || KH <= 0 || KW <= 0 ||
+      stride_h <= 0 || stride_w <= 0 || pad_h < 0 || pad_w < 0)
+    return QG_ERR_INVALID_ARG;
+  if (!x || !y) return QG_ERR_INVALID_ARG;
+  if (H + 2 * pad_h < KH || W + 2 * pad_w < KW) return QG_ERR_INVALID_ARG;
+  if (pad_h >= KH || pad_w >= KW) return QG_ERR_UNSUPPORTED;
+  const int64_t K = (int64_t)KH * KW * Cin;
+  if (K > INT32_MAX) return QG_ERR_INVALID_ARG;
+  const int64_t M = (int64_t)Nb * ((H + 2 * pad_h - KH) / stride_h + 1) *
+                    ((W + 2 * pad_w - KW) / stride_w + 1);
+  if (M > INT32_MAX) return QG_ERR_UNSUPPORTED;
+  int rc = check_requant(rq, (int)K);
+  if (rc != QG_OK) return rc;
+  if (rq->b_zero_point != 0) return QG_ERR_UNSUPPORTED;
+  if (acc_out && !aligned(acc_out, 4)) return QG_ERR_MISALIGNED;
+  return QG_OK;
+}
+
+extern "C" size_t qconv2d_s8_pack_w_bytes(int Cout, int KH, int KW, int Cin) {
+  if (Cout <= 0 || KH <= 0 || KW <= 0 || Cin <= 0) return 0;
+  const int64_t K = (int64_t)KH * KW * Cin;
+  if (K > INT32_MAX) return 0;
+  return conv_pack_w_bytes(Cout, (int)K);
+}
+
+extern "C" int qconv2d_s8_pack_w(int Cout, int KH, int KW, int Cin, const int8_t* w,
+                                 void* packed_w, size_t packed_bytes, void* stream) {
+  if (Cout <= 0 || KH <= 0 || KW <= 0 || Cin <= 0 || !w || !packed_w) return QG_ERR_INVALID_ARG;
+  const int64_t K = (int64_t)KH * KW * Cin;
+  if (K > INT32_MAX) return QG_ERR_INVALID_ARG;
+  if (!aligned(packed_w, 128)) return QG_ERR_MISALIGNED;
+  if (packed_bytes < conv_pack_w_bytes(Cout, (int)K)) return QG_ERR_WORKSPACE;
+  int rc = device_ready();
+  if (rc != QG_OK) return rc;
+  return conv_pack_w(Cout, (int)K, w, packed_w, (cudaStream_t)stream);
+}
+
+extern "C" int qconv2d_s8_im2col_packed(int Nb, int H, int W, int Cin, int Cout, int KH, int KW,
+                                        int stride_h, int stride_w, int pad_h, int pad_w,
+                                        const int8_t* x, const void* packed_w, int8_t* y,
+                                        const qg_requant_t* rq, int32_t* acc_out, void* stream) {
+  int rc = conv_args(Nb, H, W, Cin, Cout, KH, KW, stride_h, stride_w, pad_h, pad_w, x, y, rq,
+                     acc_out);
+  if (rc != QG_OK) return rc;
+  if (!packed_w) return QG_ERR_INVALID_ARG;
+  if (!aligned(packed_w, 128)) return QG_ERR_MISALIGNED;
+  rc = device_ready();
+  if (rc != QG_OK) return rc;
+  return conv_run_packed(Nb, H, W, Cin, Cout, KH, KW, stride_h, stride_w, pad_h, pad_w, x,
+                         packed_w, y, *rq, acc_out, (cudaStream_t)stream);
+}
+
 extern "C" int qconv2d_s8_im2col(int Nb, int H, int W, int Cin, int Cout, int KH, int KW,
                                  int stride_h, int stride_w, int pad_h, int pad_w,
                                  const int8_t* x, const int8_t* w, int8_t* y,
                                  const qg_requant_t* rq, int32_t* acc_out, void* workspace,
                                  size_t workspace_bytes, void* stream) {
-  if (Nb <= 0 || H <= 0 || W <= 0 || Cin <= 0 || Cout <= 0 || KH <= 0 || KW <= 0 ||
-      stride_h <= 0 || stride_w <= 0 || pad_h < 0 || pad_w < 0)
-    return QG_ERR_INVALID_ARG;
-  if (!x || !w || !y) return QG_ERR_INVALID_ARG;
-  if (H + 2 * pad_h < KH || W + 2 * pad_w < KW) return QG_ERR_INVALID_ARG;
-  if (pad_h >= KH || pad_w >= KW) return QG_ERR_UNSUPPORTED;
-  const int64_t K = (int64_t)KH * KW * Cin;
-  if (K > INT32_MAX) return QG_ERR_INVALID_ARG;
-  int rc = check_requant(rq, (int)K);
+  if (!w) return QG_ERR_INVALID_ARG;
+  int rc = conv_args(Nb, H, W, Cin, Cout, KH, KW, stride_h, stride_w, pad_h, pad_w, x, y, rq,
+                     acc_out);
   if (rc != QG_OK) return rc;
-  if (rq->b_zero_point != 0) return QG_ERR_UNSUPPORTED;
-  if (acc_out && !aligned(acc_out, 4)) return QG_ERR_MISALIGNED;
   if (workspace && !aligned(workspace, 256)) return QG_ERR_MISALIGNED;
   const size_t need =
       conv_workspace_bytes(Nb, H, W, Cin, Cout, KH, KW, stride_h, stride_w, pad_h, pad_w);

@@ -146,9 +146,107 @@ struct EpiArgs {
   uint32_t spin;    // poll limit of the pipeline waits
 };
 
+// ---------------------------------------------------------------------------
+// Implicit im2col for the convolution (MNN tileSplitFunction: the unrolled
+// input, with the input zero-point in padded taps; [QG] section 2).  Row m
+// of the virtual A matrix is output pixel (n, oh, ow); byte k = (kh*KW +
+// kw)*Cin + ci holds x[n, oh*sh+kh-ph, ow*sw+kw-pw, ci], or za outside the
+// image.  The producer warp writes each stage's 128 rows x 128 bytes straight
+// into the swizzled shared-memory tile: 16-byte cp.async copies when every
+// 16-byte chunk of a row is one contiguous run of channels (Cin % 16 == 0,
+// x 16-byte aligned), byte loads otherwise.  Bytes past K and rows past M are
+// left as they are: the packed weights are zero past K, and rows past M are
+// never stored.
+// ---------------------------------------------------------------------------
+struct ConvGather {
+  const int8_t* x;
+  int H, W, Cin, KH, KW, sh, sw, ph, pw, OH, OW;
+  int M, K;
+  int za;
+  int vec16;
+};
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ int conv_byte(const ConvGather& g, int n, int oh, int ow, int k) {
+  const int tap = k / g.Cin, ci = k - tap * g.Cin;
+  const int kh = tap / g.KW, kw = tap - kh * g.KW;
+  const int ih = oh * g.sh + kh - g.ph, iw = ow * g.sw + kw - g.pw;
+  if (ih < 0 || ih >= g.H || iw < 0 || iw >= g.W) return g.za;
+  return g.x[(((int64_t)n * g.H + ih) * g.W + iw) * g.Cin + ci];
+}
+
+// Rows lane, lane+32, lane+64, lane+96 of tile tm, K block kb.
+__device__ __forceinline__ void conv_gather_stage(const ConvGather& g, uint8_t* dst_stage, int tm,
+                                                  int kb, int lane) {
+  const uint32_t za4 = (uint32_t)(uint8_t)g.za * 0x01010101u;
+#pragma unroll 1
+  for (int i = 0; i < 4; ++i) {
+    const int r = lane + 32 * i;
+    const int m = tm * BM + r;
+    if (m >= g.M) continue;
+    const int ow = m % g.OW;
+    const int t = m / g.OW;
+    const int oh = t % g.OH, n = t / g.OH;
+    uint8_t* drow = dst_stage + r * 128;
+    if (g.vec16) {
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const int k = kb * BK + 16 * c;
+        if (k >= g.K) break;
+        uint8_t* d = drow + ((c ^ (r & 7)) << 4);
+        const int tap = k / g.Cin, ci = k - tap * g.Cin;
+        const int kh = tap / g.KW, kw = tap - kh * g.KW;
+        const int ih = oh * g.sh + kh - g.ph, iw = ow * g.sw + kw - g.pw;
+        if (ih >= 0 && ih < g.H && iw >= 0 && iw < g.W)
+          cp_async16(smem_u32(d), g.x + (((int64_t)n * g.H + ih) * g.W + iw) * g.Cin + ci);
+        else
+          *reinterpret_cast<uint4*>(d) = make_uint4(za4, za4, za4, za4);
+      }
+    } else {
+#pragma unroll 1
+      for (int c = 0; c < 8; ++c) {
+        const int k0 = kb * BK + 16 * c;
+        if (k0 >= g.K) break;
+        uint32_t wv[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t word = 0;
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            const int k = k0 + 4 * q + b;
+            const int v = k < g.K ? conv_byte(g, n, oh, ow, k) : 0;
+            word |= ((uint32_t)v & 0xFFu) << (8 * b);
+          }
+          wv[q] = word;
+        }
+        *reinterpret_cast<uint4*>(drow + ((c ^ (r & 7)) << 4)) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+      }
+    }
+  }
+}
+
+// CONV = false: A is a row-major matrix read by the tensor-copy engine.
+// CONV = true: A is the implicit im2col of `cg`, gathered by the whole
+// producer warp (see conv_gather_stage); B still comes by tensor copies.
+template <bool CONV>
 __global__ void __launch_bounds__(THREADS, 1)
     i8gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                     int num_kb, int tiles_m, int tiles_n, EpiArgs ep, int* status) {
+                     int num_kb, int tiles_m, int tiles_n, EpiArgs ep, ConvGather cg, int* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sA = smem;
@@ -168,7 +266,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], 1);
+      mbar_init(&full[s], CONV ? 32 : 1);  // conv: every producer lane arrives
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -177,7 +275,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     mbar_init(drain, 1);
     fence_mbar_init();
-    prefetch_tmap(&tmA);
+    if (!CONV) prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
   }
   if (warp == 1) {
@@ -189,7 +287,48 @@ __global__ void __launch_bounds__(THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  if (warp == 0) {
+  if (CONV && warp == 0) {
+    // ---------------- implicit-im2col producer (whole warp) ----------------
+    // Stage s is signalled one stage late: after the copies of stage s+1 are
+    // issued, each lane waits for its own copies of stage s, makes them and
+    // its zero-point fills visible to the tensor cores, and arrives.
+    int stage = 0, prev = -1;
+    uint32_t phase = 0;
+    uint32_t issued = 0, last_ph = 0;  // B tensor copies (lane 0)
+    for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
+      const int tm = t % tiles_m, tn = t / tiles_m;
+      for (int kb = 0; kb < num_kb; ++kb) {
+        bool got = true;
+        if (lane == 0) got = mbar_poll(&empty[stage], phase ^ 1, status, ep.spin);
+        if (!__shfl_sync(0xffffffffu, (int)got, 0)) goto conv_done;
+        if (lane == 0) {
+          mbar_expect_tx(&full[stage], B_STAGE);
+          tma_load_2d(sB + stage * B_STAGE, &tmB, kb * BK, tn * BN, &full[stage]);
+          issued |= 1u << stage;
+          last_ph = (last_ph & ~(1u << stage)) | (phase << stage);
+        }
+        conv_gather_stage(cg, sA + stage * A_STAGE, tm, kb, lane);
+        cp_async_commit();
+        if (prev >= 0) {
+          cp_async_wait<1>();
+          fence_proxy_async_smem();
+          mbar_arrive(&full[prev]);
+        }
+        prev = stage;
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+    }
+  conv_done:
+    cp_async_wait<0>();
+    fence_proxy_async_smem();
+    if (prev >= 0) mbar_arrive(&full[prev]);
+    if (lane == 0)
+      for (int st = 0; st < STAGES; ++st)
+        if ((issued >> st) & 1u) mbar_poll(&full[st], (last_ph >> st) & 1u, status);
+  } else if (warp == 0) {
     // ------------------------- TMA producer -------------------------
     if (lane == 0) {
       int stage = 0;
@@ -703,29 +842,6 @@ __global__ void __launch_bounds__(256) stage_a_kernel(int K, const int8_t* __res
   }
 }
 
-// Explicit im2col with the input zero-point in padded taps (conv).
-__global__ void im2col_zp_kernel(int Nb, int H, int W, int Cin, int KH, int KW, int sh, int sw,
-                                 int ph, int pw, int OH, int OW, const int8_t* __restrict__ x,
-                                 int8_t za, int8_t* __restrict__ A, int64_t lda) {
-  const int64_t K = (int64_t)KH * KW * Cin;
-  const int64_t total = (int64_t)Nb * OH * OW * K;
-  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t m = i / K;
-    const int k = (int)(i % K);
-    const int ci = k % Cin, tap = k / Cin;
-    const int kw = tap % KW, kh = tap / KW;
-    const int ow = (int)(m % OW);
-    const int64_t t = m / OW;
-    const int oh = (int)(t % OH);
-    const int n = (int)(t / OH);
-    const int ih = oh * sh + kh - ph, iw = ow * sw + kw - pw;
-    int8_t v = za;
-    if (ih >= 0 && ih < H && iw >= 0 && iw < W) v = x[(((int64_t)n * H + ih) * W + iw) * Cin + ci];
-    A[m * lda + k] = v;
-  }
-}
-
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
@@ -826,8 +942,11 @@ size_t i8gemm_packed_workspace_bytes(int M, int K) {
 }
 
 int i8gemm_setup() {
-  cudaError_t e = cudaFuncSetAttribute(i8gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)SMEM_BYTES);
+  cudaError_t e = cudaFuncSetAttribute(i8gemm_tc_kernel<false>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+  if (e != cudaSuccess) return QG_ERR_CUDA;
+  e = cudaFuncSetAttribute(i8gemm_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)SMEM_BYTES);
   if (e != cudaSuccess) return QG_ERR_CUDA;
   e = cudaFuncSetAttribute(i8gemm_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)P_SMEM_BYTES);
@@ -853,6 +972,26 @@ int i8gemm_setup() {
     return QG_ERR_CUDA;
   g_max_pairs[dev] = clusters;
   return get_encode();
+}
+
+static EpiArgs make_epi(int M, int N, int K, const void* packed_b, const qg_requant_t& rq,
+                        const int32_t* rowsum, int8_t* C, int64_t ldc, int32_t* acc_out,
+                        int64_t ld_acc) {
+  const PackDims d = pack_dims(K, N);
+  EpiArgs ep;
+  ep.M = M; ep.N = N; ep.K = K;
+  ep.za = rq.a_zero_point; ep.zb = rq.b_zero_point; ep.zo = rq.out_zero_point;
+  ep.lo = rq.clamp_min; ep.hi = rq.clamp_max;
+  ep.colsum = (const int32_t*)((const int8_t*)packed_b + d.Np * d.Kp);
+  ep.rowsum = rowsum;
+  ep.bias = rq.bias;
+  ep.per_channel = rq.per_channel;
+  ep.m0 = rq.multiplier0; ep.sh = rq.shift0;
+  ep.m0v = rq.multiplier; ep.shv = rq.shift;
+  ep.C = C; ep.ldc = ldc; ep.acc_out = acc_out; ep.ld_acc = ld_acc;
+  ep.stall = 0;
+  ep.spin = kSpinLimit;
+  return ep;
 }
 
 int i8gemm_run_packed(int M, int N, int K, const int8_t* A, int64_t lda, const void* packed_b,
@@ -885,17 +1024,7 @@ int i8gemm_run_packed(int M, int N, int K, const int8_t* A, int64_t lda, const v
   rc = make_tmap(&tmB, packed_b, (uint64_t)d.Kp, (uint64_t)d.Np, (uint64_t)d.Kp,
                  pair_path ? BM : BN);
   if (rc != QG_OK) return rc;
-  EpiArgs ep;
-  ep.M = M; ep.N = N; ep.K = K;
-  ep.za = rq.a_zero_point; ep.zb = rq.b_zero_point; ep.zo = rq.out_zero_point;
-  ep.lo = rq.clamp_min; ep.hi = rq.clamp_max;
-  ep.colsum = (const int32_t*)((const int8_t*)packed_b + d.Np * d.Kp);
-  ep.rowsum = rowsum;
-  ep.bias = rq.bias;
-  ep.per_channel = rq.per_channel;
-  ep.m0 = rq.multiplier0; ep.sh = rq.shift0;
-  ep.m0v = rq.multiplier; ep.shv = rq.shift;
-  ep.C = C; ep.ldc = ldc; ep.acc_out = acc_out; ep.ld_acc = ld_acc;
+  EpiArgs ep = make_epi(M, N, K, packed_b, rq, rowsum, C, ldc, acc_out, ld_acc);
   const int num_kb = (int)(d.Kp / BK);
   ep.stall = (M <= BM && num_kb > 1 && take_stall(kStallInt8Gemm)) ? 1 : 0;
   ep.spin = ep.stall ? kStallSpinLimit : kSpinLimit;
@@ -926,14 +1055,16 @@ int i8gemm_run_packed(int M, int N, int K, const int8_t* A, int64_t lda, const v
   const int tiles_m = (int)cdiv(M, BM), tiles_n = (int)cdiv(N, BN);
   const int tiles = tiles_m * tiles_n;
   const int grid = tiles < num_sms() ? tiles : num_sms();
-  i8gemm_tc_kernel<<<grid, THREADS, SMEM_BYTES, st>>>(tmA, tmB, num_kb, tiles_m, tiles_n, ep,
-                                                      status_word());
+  i8gemm_tc_kernel<false><<<grid, THREADS, SMEM_BYTES, st>>>(tmA, tmB, num_kb, tiles_m, tiles_n,
+                                                             ep, ConvGather{}, status_word());
   return launch_status();
 }
 
 // ---------------------------------------------------------------------------
-// INT8 convolution: weights packed (K-major already, padded, column sums),
-// zero-point-padded im2col of x, then the GEMM above.
+// INT8 convolution: the weights [Cout][KH][KW][Cin] are K-major already and
+// are packed like B (padded, column sums); the one-CTA tensor-core kernel
+// gathers the im2col rows itself (implicit GEMM), so a call is one launch
+// with packed weights, two with raw ones (pack, then the GEMM).
 // ---------------------------------------------------------------------------
 static void conv_geometry(int H, int W, int KH, int KW, int sh, int sw, int ph, int pw, int* OH,
                           int* OW) {
@@ -941,38 +1072,56 @@ static void conv_geometry(int H, int W, int KH, int KW, int sh, int sw, int ph, 
   *OW = (W + 2 * pw - KW) / sw + 1;
 }
 
-size_t conv_workspace_bytes(int Nb, int H, int W, int Cin, int Cout, int KH, int KW, int sh,
-                            int sw, int ph, int pw) {
-  int OH, OW;
-  conv_geometry(H, W, KH, KW, sh, sw, ph, pw, &OH, &OW);
-  const int64_t K = (int64_t)KH * KW * Cin;
-  const int64_t M = (int64_t)Nb * OH * OW;
-  return (size_t)(round_up((int64_t)i8gemm_pack_b_bytes((int)K, Cout), 256) +
-                  round_up(M * staged_lda((int)K), 256));
+size_t conv_pack_w_bytes(int Cout, int K) { return i8gemm_pack_b_bytes(K, Cout); }
+
+int conv_pack_w(int Cout, int K, const int8_t* w, void* packed, cudaStream_t st) {
+  return i8gemm_pack_b_kmajor(K, Cout, w, K, packed, st);
 }
 
-int conv_run(int Nb, int H, int W, int Cin, int Cout, int KH, int KW, int sh, int sw, int ph,
-             int pw, const int8_t* x, const int8_t* w, int8_t* y, const qg_requant_t& rq,
-             int32_t* acc_out, void* ws, size_t ws_bytes, cudaStream_t st) {
+size_t conv_workspace_bytes(int Nb, int H, int W, int Cin, int Cout, int KH, int KW, int sh,
+                            int sw, int ph, int pw) {
+  (void)Nb; (void)H; (void)W; (void)sh; (void)sw; (void)ph; (void)pw;
+  return (size_t)round_up((int64_t)i8gemm_pack_b_bytes(KH * KW * Cin, Cout), 256);
+}
+
+int conv_run_packed(int Nb, int H, int W, int Cin, int Cout, int KH, int KW, int sh, int sw,
+                    int ph, int pw, const int8_t* x, const void* packed_w, int8_t* y,
+                    const qg_requant_t& rq, int32_t* acc_out, cudaStream_t st) {
   int OH, OW;
   conv_geometry(H, W, KH, KW, sh, sw, ph, pw, &OH, &OW);
   const int K = KH * KW * Cin;
   const int64_t M = (int64_t)Nb * OH * OW;
   if (M > INT32_MAX) return QG_ERR_UNSUPPORTED;
-  const size_t pb = round_up((int64_t)i8gemm_pack_b_bytes(K, Cout), 256);
-  int8_t* packed = (int8_t*)ws;
-  int8_t* Aim = (int8_t*)ws + pb;
-  int rc = i8gemm_pack_b_kmajor(K, Cout, w, K, packed, st);
+  const PackDims d = pack_dims(K, Cout);
+  CUtensorMap tmB;
+  int rc = make_tmap(&tmB, packed_w, (uint64_t)d.Kp, (uint64_t)d.Np, (uint64_t)d.Kp, BN);
   if (rc != QG_OK) return rc;
-  const int64_t lda = staged_lda(K);
-  const int64_t total = M * K;
-  int blocks = (int)min64(cdiv(total, 256), (int64_t)num_sms() * 16);
-  im2col_zp_kernel<<<blocks, 256, 0, st>>>(Nb, H, W, Cin, KH, KW, sh, sw, ph, pw, OH, OW, x,
-                                           (int8_t)rq.a_zero_point, Aim, lda);
-  rc = launch_status();
+  EpiArgs ep = make_epi((int)M, Cout, K, packed_w, rq, nullptr, y, Cout, acc_out, Cout);
+  ConvGather cg;
+  cg.x = x;
+  cg.H = H; cg.W = W; cg.Cin = Cin; cg.KH = KH; cg.KW = KW;
+  cg.sh = sh; cg.sw = sw; cg.ph = ph; cg.pw = pw; cg.OH = OH; cg.OW = OW;
+  cg.M = (int)M; cg.K = K;
+  cg.za = rq.a_zero_point;
+  cg.vec16 = (Cin % 16 == 0) && (((uintptr_t)x & 15) == 0);
+  const int num_kb = (int)(d.Kp / BK);
+  const int tiles_m = (int)cdiv(M, BM), tiles_n = (int)cdiv(Cout, BN);
+  const int tiles = tiles_m * tiles_n;
+  const int grid = tiles < num_sms() ? tiles : num_sms();
+  i8gemm_tc_kernel<true><<<grid, THREADS, SMEM_BYTES, st>>>(tmB, tmB, num_kb, tiles_m, tiles_n,
+                                                            ep, cg, status_word());
+  return launch_status();
+}
+
+int conv_run(int Nb, int H, int W, int Cin, int Cout, int KH, int KW, int sh, int sw, int ph,
+             int pw, const int8_t* x, const int8_t* w, int8_t* y, const qg_requant_t& rq,
+             int32_t* acc_out, void* ws, size_t ws_bytes, cudaStream_t st) {
+  const int K = KH * KW * Cin;
+  if (!ws || ws_bytes < conv_workspace_bytes(Nb, H, W, Cin, Cout, KH, KW, sh, sw, ph, pw))
+    return QG_ERR_WORKSPACE;
+  int rc = conv_pack_w(Cout, K, w, ws, st);
   if (rc != QG_OK) return rc;
-  return i8gemm_run_packed((int)M, Cout, K, Aim, lda, packed, y, Cout, rq, acc_out, Cout, nullptr,
-                           0, st);
+  return conv_run_packed(Nb, H, W, Cin, Cout, KH, KW, sh, sw, ph, pw, x, ws, y, rq, acc_out, st);
 }
 
 }  // namespace qg

@@ -173,9 +173,11 @@ int qgemm_s8s8_requant_packed(int M, int N, int K,
                               void* stream);
 
 /* ------------------------------------------------------------------------
- * INT8 convolution as implicit-im2col GEMM.  [MNN] tileSplitFunction: the
- * im2col buffer is filled with the input zero-point where a tap falls in the
- * padding; [QG] section 2: padding must stand for real zero.
+ * INT8 convolution as an implicit-im2col GEMM.  [MNN] tileSplitFunction: the
+ * unrolled input holds the input zero-point where a tap falls in the
+ * padding; [QG] section 2: padding must stand for real zero.  No im2col
+ * buffer exists: the tensor-core kernel's producer gathers each row of the
+ * virtual unrolled matrix straight from x into its shared-memory tile.
  *
  *   x: int8 NHWC [Nb][H][W][Cin]      w: int8 [Cout][KH][KW][Cin] (zw = 0)
  *   y: int8 NHWC [Nb][OH][OW][Cout], OH = (H+2*pad_h-KH)/stride_h + 1 (same for W)
@@ -183,7 +185,23 @@ int qgemm_s8s8_requant_packed(int M, int N, int K,
  * GEMM view: M = Nb*OH*OW, N = Cout, K = KH*KW*Cin; pad value =
  * rq->a_zero_point; rq->b_zero_point must be 0.  Per-Cout requant via
  * rq->per_channel.  Fused ReLU: rq->clamp_min = rq->out_zero_point.
+ * pad_h < KH and pad_w < KW (else QG_ERR_UNSUPPORTED); M <= INT32_MAX.
+ *
+ * Weight-stationary form ([MNN] reorderWeight: weights reordered once at
+ * load, with their per-channel sums): qconv2d_s8_pack_w packs w once into an
+ * opaque buffer of qconv2d_s8_pack_w_bytes bytes (128-byte aligned), and
+ * qconv2d_s8_im2col_packed runs the convolution from it in one launch, with
+ * no workspace.  qconv2d_s8_im2col packs w into its workspace on every call
+ * (two launches).  The gather copies 16-byte runs when Cin % 16 == 0 and x
+ * is 16-byte aligned, single bytes otherwise (slower, same result).
  * ------------------------------------------------------------------------ */
+size_t qconv2d_s8_pack_w_bytes(int Cout, int KH, int KW, int Cin);
+int qconv2d_s8_pack_w(int Cout, int KH, int KW, int Cin, const int8_t* w,
+                      void* packed_w, size_t packed_bytes, void* stream);
+int qconv2d_s8_im2col_packed(int Nb, int H, int W, int Cin, int Cout, int KH, int KW,
+                             int stride_h, int stride_w, int pad_h, int pad_w,
+                             const int8_t* x, const void* packed_w, int8_t* y,
+                             const qg_requant_t* rq, int32_t* acc_out, void* stream);
 size_t qconv2d_s8_workspace_bytes(int Nb, int H, int W, int Cin, int Cout,
                                   int KH, int KW, int stride_h, int stride_w,
                                   int pad_h, int pad_w);

@@ -172,7 +172,7 @@ def test_gemm_8192x8192x8200_every_output(lib, packed):
 # ---------------------------------------------------------------------------
 # convolution
 # ---------------------------------------------------------------------------
-def run_conv(lib, w, with_acc=True):
+def run_conv(lib, w, with_acc=True, packed=False, x_offset=0):
     mult, shift, m0, sh = _params(lib, dict(ratio=w["ratio"], per_channel=True))
     bias = None if w["bias"] is None else _dev(w["bias"])
     rq = lib.make_requant(a_zero_point=w["za"], bias=bias, multiplier=mult, shift=shift,
@@ -181,7 +181,17 @@ def run_conv(lib, w, with_acc=True):
     OH, OW = lib.conv_out_hw(w["H"], w["W"], w["KH"], w["KW"], w["stride"], w["pad"])
     y = torch.empty((w["Nb"], OH, OW, w["Cout"]), dtype=torch.int8, device="cuda")
     acc = torch.empty((w["Nb"], OH, OW, w["Cout"]), dtype=torch.int32, device="cuda") if with_acc else None
-    lib.qconv2d_s8_im2col(_dev(w["x"]), _dev(w["w"]), y, rq, w["stride"], w["pad"], acc_out=acc)
+    x = _dev(w["x"])
+    if x_offset:  # the same image at an address that is not 16-byte aligned
+        buf = torch.empty(x.numel() + x_offset, dtype=torch.int8, device="cuda")
+        x = buf[x_offset:].view(x.shape)
+        x.copy_(_dev(w["x"]))
+    if packed:
+        pw = lib.qconv2d_s8_pack_w(_dev(w["w"]))
+        lib.qconv2d_s8_im2col_packed(x, pw, w["w"].shape, y, rq, w["stride"], w["pad"],
+                                     acc_out=acc)
+    else:
+        lib.qconv2d_s8_im2col(x, _dev(w["w"]), y, rq, w["stride"], w["pad"], acc_out=acc)
     torch.cuda.synchronize()
     y_ref, acc_ref = oracle.qconv2d_s8(w["x"], w["w"], w["stride"], w["pad"], w["za"], w["bias"],
                                        m0, sh, w["out_zp"], w["clamp_min"], w["clamp_max"])
@@ -194,6 +204,21 @@ def run_conv(lib, w, with_acc=True):
 def test_conv_56x56x64_bit_exact(lib):
     y_ref = run_conv(lib, workloads.int8_conv_56x56x64_3x3())
     assert (y_ref == -10).mean() > 0.05      # the ReLU floor at the out zero-point binds
+
+
+@pytest.mark.parametrize("x_offset", [0, 3])
+def test_conv_56x56x64_packed_weights_bit_exact(lib, x_offset):
+    # weights packed once; x_offset = 3 takes the byte-gather path
+    run_conv(lib, workloads.int8_conv_56x56x64_3x3(), packed=True, x_offset=x_offset)
+
+
+@pytest.mark.parametrize("Nb,H,W,Cin,Cout,KH,KW,s,p", [
+    (2, 17, 19, 32, 96, 3, 3, 1, 1), (1, 40, 33, 16, 300, 5, 5, 2, 2), (3, 9, 9, 48, 40, 1, 3, 1, 0),
+    (1, 12, 12, 3, 8, 7, 7, 2, 3), (1, 300, 3, 64, 64, 3, 1, 1, 1)])
+def test_conv_packed_shapes(lib, Nb, H, W, Cin, Cout, KH, KW, s, p):
+    w = workloads.int8_conv(Nb, H, W, Cin, Cout, KH, KW, (s, s), (p, p), seed=H * 3 + Cin + Cout,
+                            relu=(Cout % 2 == 0))
+    run_conv(lib, w, packed=True)
 
 
 @pytest.mark.parametrize("Nb,H,W,Cin,Cout,KH,KW,s,p", [
