@@ -715,26 +715,46 @@ __global__ void __launch_bounds__(THREADS, 1)
   // share of the rows over all ranks in rank order (deterministic) and
   // writes y; the second barrier keeps every CTA's shared memory alive until
   // its peers have read it.
+  // This CTA reduces rows [r0, r1) of the tile; epilogue thread etid takes
+  // the 4-column chunk c = etid % 32 of rows r0 + etid / 32 + 8j.  Its bias
+  // and row scales are fetched before the cluster barrier, so each output
+  // waits only for the partials.
+  const int rows_per = (TM + a.splits - 1) / a.splits;
+  const int r0 = split * rows_per, r1 = min(TM, r0 + rows_per);
+  constexpr int RJ = TM / 8;  // rows per thread at most (one split)
+  float bias4[4] = {0.f, 0.f, 0.f, 0.f};
+  float srow[RJ];
+  if (warp >= EPI_WARP0) {
+    const int etid = threadIdx.x - EPI_WARP0 * 32;
+    const int c = etid & 31;
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      if (a.bias && n0 + 4 * c + e < a.N) bias4[e] = __ldg(a.bias + n0 + 4 * c + e);
+#pragma unroll
+    for (int j = 0; j < RJ; ++j) {
+      const int m = m0 + r0 + (etid >> 5) + 8 * j;
+      srow[j] = (!ABLK && r0 + (etid >> 5) + 8 * j < r1 && m < a.M) ? a.sA[m] : 1.0f;
+    }
+  }
   __syncwarp();
   cluster_sync_all();
   if (warp >= EPI_WARP0) {
     const int etid = threadIdx.x - EPI_WARP0 * 32;
-    const int rows_per = (TM + a.splits - 1) / a.splits;
-    const int r0 = split * rows_per, r1 = min(TM, r0 + rows_per);
     const uint32_t part_s = smem_u32(part);
     const bool vec = ((a.ldy & 3) == 0) && ((reinterpret_cast<uintptr_t>(a.y) & 15) == 0);
-    for (int i = etid; i < (r1 - r0) * (TW / 4); i += NEPI) {
-      const int mm = r0 + i / (TW / 4);
-      const int c = i % (TW / 4);
+    const int c = etid & 31;
+#pragma unroll
+    for (int jr = 0; jr < RJ; ++jr) {
+      const int mm = r0 + (etid >> 5) + 8 * jr;
       const int m = m0 + mm, n = n0 + 4 * c;
-      if (m >= a.M || n >= a.N) continue;
+      if (mm >= r1 || m >= a.M || n >= a.N) continue;
       const uint32_t off = (uint32_t)((mm * PST + 4 * c) * 4);
       // every rank's partial requested before the first is added
       float4 t[MAX_SPLITS];
 #pragma unroll
       for (int j = 0; j < MAX_SPLITS; ++j)
         if (j < a.splits) t[j] = ld_dsmem_f4(mapa(part_s + off, (uint32_t)j));
-      const float s = ABLK ? 1.0f : a.sA[m];
+      const float s = srow[jr];
       float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
       for (int j = 0; j < MAX_SPLITS; ++j) {
@@ -749,7 +769,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         if (!ABLK) t4[e] = __fmul_rn(s, t4[e]);
-        if (a.bias && n + e < a.N) t4[e] = __fadd_rn(t4[e], a.bias[n + e]);
+        if (a.bias) t4[e] = __fadd_rn(t4[e], bias4[e]);
         t4[e] = fminf(fmaxf(t4[e], a.lo), a.hi);
       }
       float* yr = a.y + (int64_t)m * a.ldy + n;

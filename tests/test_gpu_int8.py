@@ -214,7 +214,7 @@ def test_conv_56x56x64_packed_weights_bit_exact(lib, x_offset):
 
 @pytest.mark.parametrize("Nb,H,W,Cin,Cout,KH,KW,s,p", [
     (2, 17, 19, 32, 96, 3, 3, 1, 1), (1, 40, 33, 16, 300, 5, 5, 2, 2), (3, 9, 9, 48, 40, 1, 3, 1, 0),
-    (1, 12, 12, 3, 8, 7, 7, 2, 3), (1, 300, 3, 64, 64, 3, 1, 1, 1)])
+    (1, 12, 12, 3, 8, 7, 7, 2, 3), (1, 300, 3, 64, 64, 3, 3, 1, 1)])
 def test_conv_packed_shapes(lib, Nb, H, W, Cin, Cout, KH, KW, s, p):
     w = workloads.int8_conv(Nb, H, W, Cin, Cout, KH, KW, (s, s), (p, p), seed=H * 3 + Cin + Cout,
                             relu=(Cout % 2 == 0))
