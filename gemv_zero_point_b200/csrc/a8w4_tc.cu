@@ -33,17 +33,23 @@
 //     and their partial tiles are reduced through distributed shared memory
 //     in a fixed order.
 //
-// Roles of a8w4_tc_kernel (448 threads, one CTA per SM):
-//   warp 0      bulk copies of the activation stages (after the grid
-//               dependency wait)
-//   warp 1      TMEM allocation; MMA issue: per 32-wide group two K = 16
-//               MMAs into one of 4 rotating 128-column TMEM buffers
+// Roles of a8w4_tc_kernel (704 threads, one CTA per SM):
+//   warp 0      tensor copies of the weight scale (and zero) tables before
+//               the grid dependency wait; after it the activation tables and
+//               the bulk copies of the activation stages
+//   warp 1      TMEM allocation; MMA issue: per 64-wide stage four K = 16
+//               MMAs (two per 32-wide group) into one of 2 TMEM stage
+//               buffers of 2 x 128 columns, one commit for the accumulators
 //   warps 2..5  weight nibbles: a ring of 64-wide K slices of the CTA's 128
 //               rows (tensor copies, issued before the grid dependency wait),
 //               expanded to bf16 w = u - 8 in the swizzled stage layout
-//   warps 6..13 per group: tcgen05.ld of the exact group dots, release of the
-//               buffer, acc += scale * I with packed f32x2 FMAs; then the
-//               partial tile, the cluster reduction and y
+//   warps 6..21 per stage: tcgen05.ld of the exact group dots (32 columns
+//               per warp), release of the buffer, acc += scale * I with
+//               packed f32x2 FMAs; then the partial tile, the cluster
+//               reduction and y
+// The single-thread roles poll their barriers (mbarrier.test_wait): a
+// suspending try_wait costs some hundred cycles even on a completed phase,
+// several times the issue cost of an MMA.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -67,27 +73,41 @@ constexpr int STAGE_BYTES = 128 * KS * 2;  // 16 KiB, both operands
 constexpr int STAGES = 4;
 constexpr int NRING = 8;                // weight nibble stages in flight
 constexpr int NIB_BYTES = TW * KS / 2;  // 4 KiB of nibbles per stage
-constexpr int NBUF = 4;                 // TMEM group buffers of TM columns
+constexpr int NSB = 2;                  // TMEM stage buffers: the 2 groups of a stage, 2*TM columns
 constexpr int KR_MAX = 1024;            // K range per CTA
 constexpr int GR_MAX = KR_MAX / 32;
 constexpr int MAX_SPLITS = 8;
-constexpr int THREADS = 14 * 32;
+constexpr int THREADS = 22 * 32;
 constexpr int CONV_WARP0 = 2;
 constexpr int NCONV = 128;              // converter threads
 constexpr int EPI_WARP0 = 6;
-constexpr int NEPI = 256;               // epilogue threads
+constexpr int NEPI = 512;               // epilogue threads: 4 lane quarters x 4 column blocks
 constexpr int PST = TW + 4;             // row stride (floats) of the partial tile [m][n]
 
 // shared-memory map (offsets from the 1024-byte aligned base)
 constexpr size_t OFF_A = 0;                                        // activation stages
 constexpr size_t OFF_W = OFF_A + (size_t)STAGES * STAGE_BYTES;     // weight stages
 constexpr size_t OFF_N = OFF_W + (size_t)STAGES * STAGE_BYTES;     // nibble ring
-constexpr size_t OFF_SCL = OFF_N + (size_t)NRING * NIB_BYTES;      // [GR][TW] weight scales
-constexpr size_t OFF_ZW = OFF_SCL + (size_t)GR_MAX * TW * 4;       // [GR][TW] weight zeros
-constexpr size_t OFF_ACT = OFF_ZW + (size_t)GR_MAX * TW * 4;       // [GR][TM] act scales / sums
+constexpr size_t OFF_SCL = OFF_N + (size_t)NRING * NIB_BYTES;      // [TW][Gr] weight scales
+constexpr size_t OFF_ZW = OFF_SCL + (size_t)GR_MAX * TW * 4;       // [TW][Gr] weight zeros
+constexpr size_t OFF_ACT = OFF_ZW + (size_t)GR_MAX * TW * 4;       // [TM][Gr] act scales / sums
 constexpr size_t OFF_BAR = OFF_ACT + (size_t)GR_MAX * TM * 4;
 constexpr size_t SMEM_BYTES = 1024 + OFF_BAR + 512;
 static_assert((size_t)TM * PST * 4 <= OFF_N, "partial tile reuses the stage buffers");
+static_assert(OFF_SCL % 1024 == 0 && OFF_ZW % 1024 == 0 && OFF_ACT % 1024 == 0,
+              "swizzled tables start on a swizzle atom");
+
+// The per-group tables (weight scales / zeros [row][Gr], activation block
+// scales / sums [row][Gr]) are kept as rows of Gr elements; when a row is
+// 32, 64 or 128 bytes they arrive by one tensor copy with the matching
+// swizzle (16-byte chunk c of the row at byte address a moves to
+// c ^ ((a >> 7) & (span/16 - 1))), which spreads a column of the table over
+// the banks; other sizes are loaded by threads into the same layout.
+__device__ __forceinline__ uint32_t tbl_off(int row, int g, int esz, int rowbytes) {
+  const uint32_t raw = (uint32_t)(row * rowbytes + g * esz);
+  const uint32_t mask = rowbytes == 128 ? 7u : rowbytes == 64 ? 3u : rowbytes == 32 ? 1u : 0u;
+  return raw ^ (((raw >> 7) & mask) << 4);
+}
 
 // kind::f16 instruction descriptor: D f32, A bf16, B bf16, both K-major,
 // N = TM, M = TW.
@@ -182,6 +202,19 @@ __device__ __forceinline__ bool bar_and(bool v) {
 template <int ID, int N>
 __device__ __forceinline__ void bar_sync() {
   asm volatile("bar.sync %0, %1;" ::"n"(ID), "n"(N) : "memory");
+}
+
+// Poll a barrier phase from one thread, sleeping briefly between polls so
+// the spinning warp does not take the issue slots of the warps doing the
+// arithmetic on its sub-partition; bounded like mbar_poll.
+__device__ __forceinline__ bool poll_yield(uint64_t* bar, uint32_t parity, int* status,
+                                           uint32_t limit) {
+  for (uint32_t i = 0; i < (limit << 4); ++i) {
+    if (mbar_test(bar, parity)) return true;
+    __nanosleep(32);
+  }
+  record_error(status, QG_ERR_TIMEOUT);
+  return false;
 }
 
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -440,28 +473,37 @@ struct GemmArgs {
   float lo, hi;
   float* y;
   int64_t ldy;
+  int tma_w, tma_act;      // the weight / activation tables come by tensor copy
   int stall;               // test hook: the activation stage 1 is never issued
   uint32_t spin;           // poll limit of the pipeline waits
 };
 
+// Tensor maps of one call: nibbles, and the per-group tables when they come
+// by tensor copy (otherwise unused copies of the nibble map).
+struct TcMaps {
+  CUtensorMap w, scl, zw, act;
+};
+
 template <bool ABLK, bool WZP>
 __global__ void __launch_bounds__(THREADS, 1)
-    a8w4_tc_kernel(const __grid_constant__ CUtensorMap tmW, GemmArgs a, int* status) {
+    a8w4_tc_kernel(const __grid_constant__ TcMaps tm_, GemmArgs a, int* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sA = smem + OFF_A;
   uint8_t* sW = smem + OFF_W;
   uint8_t* sN = smem + OFF_N;
-  float* scl = reinterpret_cast<float*>(smem + OFF_SCL);   // [g][n]
-  float* zws = reinterpret_cast<float*>(smem + OFF_ZW);    // [g][n]
-  float* actp = reinterpret_cast<float*>(smem + OFF_ACT);  // [g][m]
+  uint8_t* scl = smem + OFF_SCL;   // [n][Gr] weight scales (f32 or bf16), swizzled rows
+  uint8_t* zws = smem + OFF_ZW;    // [n][Gr] f32 weight zeros
+  uint8_t* actp = smem + OFF_ACT;  // [m][Gr] f32 activation block scales / group sums
   uint64_t* a_full = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
   uint64_t* w_full = a_full + STAGES;
   uint64_t* empty = w_full + STAGES;
   uint64_t* nib_full = empty + STAGES;
   uint64_t* tfull = nib_full + NRING;
-  uint64_t* tempty = tfull + NBUF;
-  uint64_t* drain = tempty + NBUF;
+  uint64_t* tempty = tfull + NSB;
+  uint64_t* prm_full = tempty + NSB;   // weight tables landed
+  uint64_t* act_full = prm_full + 1;   // activation tables landed
+  uint64_t* drain = act_full + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   float* part = reinterpret_cast<float*>(smem);  // [TM][PST], after the mainloop
 
@@ -474,6 +516,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int G = a.K >> 5, g0 = k0 >> 5;
   const int Gr = a.Kr >> 5;
   const int nst = a.Kr / KS;
+  const int sesz = a.scale_bf16 ? 2 : 4;  // bytes per stored weight scale
+  const int srow = Gr * sesz, frow = Gr * 4;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -482,18 +526,20 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&empty[s], 1);
     }
     for (int s = 0; s < NRING; ++s) mbar_init(&nib_full[s], 1);
-    for (int b = 0; b < NBUF; ++b) {
+    for (int b = 0; b < NSB; ++b) {
       mbar_init(&tfull[b], 1);
       mbar_init(&tempty[b], NEPI / 32);
     }
+    mbar_init(prm_full, 1);
+    mbar_init(act_full, 1);
     mbar_init(drain, 1);
     fence_mbar_init();
-    prefetch_tmap(&tmW);
+    prefetch_tmap(&tm_.w);
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_u32(tmem_slot)),
-                 "r"(NBUF * TM)
+                 "r"(NSB * 2 * TM)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
@@ -503,16 +549,28 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint32_t tmem_base = *tmem_slot;
 
   if (warp == 0) {
-    // ---------------- activation stages (bulk copies) ----------------
+    // ------------- tables and activation stages (tensor / bulk copies) -------------
     if (lane == 0) {
       uint32_t issued = 0, last_ph = 0;
-      // the activation tiles come from the quantization grid
+      bool prm = false, act = false;
+      if (a.tma_w) {  // inputs of the call: before the grid dependency wait
+        mbar_arrive_expect_tx(prm_full, (uint32_t)(TW * (srow + (WZP ? frow : 0))));
+        tma_load_2d(scl, &tm_.scl, g0, n0, prm_full);
+        if (WZP) tma_load_2d(zws, &tm_.zw, g0, n0, prm_full);
+        prm = true;
+      }
+      // the activation tiles and tables come from the quantization grid
       asm volatile("griddepcontrol.wait;" ::: "memory");
+      if ((ABLK || WZP) && a.tma_act) {
+        mbar_arrive_expect_tx(act_full, (uint32_t)(TM * frow));
+        tma_load_2d(actp, &tm_.act, g0, m0, act_full);
+        act = true;
+      }
       const uint8_t* src = reinterpret_cast<const uint8_t*>(a.atile) +
                            ((int64_t)tm * a.nkb + (k0 / KS)) * STAGE_BYTES;
       for (int s = 0; s < nst; ++s) {
         const int slot = s % STAGES;
-        if (s >= STAGES && !mbar_poll(&empty[slot], ((s / STAGES) - 1) & 1, status, a.spin)) break;
+        if (s >= STAGES && !poll_yield(&empty[slot], ((s / STAGES) - 1) & 1, status, a.spin)) break;
         if (a.stall && s == 1) continue;
         mbar_arrive_expect_tx(&a_full[slot], STAGE_BYTES);
         bulk_g2s(sA + slot * STAGE_BYTES, src + (int64_t)s * STAGE_BYTES, STAGE_BYTES,
@@ -523,37 +581,36 @@ __global__ void __launch_bounds__(THREADS, 1)
       // every copy issued here has landed before the CTA may exit
       for (int st = 0; st < STAGES; ++st)
         if ((issued >> st) & 1u) mbar_poll(&a_full[st], (last_ph >> st) & 1u, status);
+      if (prm) mbar_poll(prm_full, 0, status);
+      if (act) mbar_poll(act_full, 0, status);
     }
   } else if (warp == 1) {
     // ---------------- MMA issue ----------------
+    // Per stage: both groups (two K = 16 MMAs each) into one TMEM stage
+    // buffer, one commit for the accumulators and one for the stage.
     if (lane == 0) {
       bool failed = false;
-      for (int s = 0; s < nst && !failed; ++s) {
-        const int slot = s % STAGES;
+      for (int s = 0; s < nst; ++s) {
+        const int slot = s % STAGES, sb = s % NSB;
         const uint32_t par = (uint32_t)(s / STAGES) & 1;
-        if (!mbar_poll(&a_full[slot], par, status, a.spin) ||
-            !mbar_poll(&w_full[slot], par, status, a.spin)) {
+        if (!poll_yield(&a_full[slot], par, status, a.spin) ||
+            !poll_yield(&w_full[slot], par, status, a.spin) ||
+            !poll_yield(&tempty[sb], ((uint32_t)(s / NSB) & 1) ^ 1, status, a.spin)) {
           failed = true;
           break;
         }
         tc_fence_after();
-        const uint32_t wa = smem_u32(sW + slot * STAGE_BYTES);
-        const uint32_t xa = smem_u32(sA + slot * STAGE_BYTES);
+        // descriptor start addresses count 16-byte units: K = 16 more is +2
+        const uint64_t dw = sdesc_sw128(smem_u32(sW + slot * STAGE_BYTES));
+        const uint64_t dx = sdesc_sw128(smem_u32(sA + slot * STAGE_BYTES));
+        const uint32_t d = tmem_base + (uint32_t)(sb * 2 * TM);
 #pragma unroll
         for (int gi = 0; gi < 2; ++gi) {
-          const int g = 2 * s + gi;
-          const int buf = g % NBUF;
-          if (!mbar_poll(&tempty[buf], ((uint32_t)(g / NBUF) & 1) ^ 1, status, a.spin)) {
-            failed = true;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t d = tmem_base + (uint32_t)(buf * TM);
-          mma_bf16(d, sdesc_sw128(wa + 64 * gi), sdesc_sw128(xa + 64 * gi), 0);
-          mma_bf16(d, sdesc_sw128(wa + 64 * gi + 32), sdesc_sw128(xa + 64 * gi + 32), 1);
-          mma_commit(&tfull[buf]);
+          mma_bf16(d + gi * TM, dw + 4 * gi, dx + 4 * gi, 0);
+          mma_bf16(d + gi * TM, dw + 4 * gi + 2, dx + 4 * gi + 2, 1);
         }
-        if (!failed) mma_commit(&empty[slot]);
+        mma_commit(&tfull[sb]);
+        mma_commit(&empty[slot]);
       }
       if (failed) {
         // MMAs already issued finish before their operands or TMEM go away
@@ -568,41 +625,57 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (ctid == 0) {
       for (int s = 0; s < nst && s < NRING; ++s) {
         mbar_arrive_expect_tx(&nib_full[s], NIB_BYTES);
-        tma_load_2d(sN + s * NIB_BYTES, &tmW, (k0 + KS * s) / 8, n0, &nib_full[s]);
+        tma_load_2d(sN + s * NIB_BYTES, &tm_.w, (k0 + KS * s) / 8, n0, &nib_full[s]);
         issued |= 1u << s;
       }
     }
     bool ok = true;
+    // Converter thread r owns row r of every stage: its 8 nibble words (32
+    // bytes, two 128-bit loads issued before any use) become the row's 8
+    // swizzled 16-byte bf16 chunks.
+    const int r = ctid;
+    const uint32_t nib_row = smem_u32(sN) + (uint32_t)(r * 32);
+    const uint32_t dst_row = smem_u32(sW) + (uint32_t)(r * 128);
     for (int s = 0; s < nst; ++s) {
       const int slot = s % STAGES, ns = s % NRING;
+      // thread 0 polls both barriers; a hardware barrier releases the rest
       bool w = true;
-      if (s >= STAGES) w = mbar_wait(&empty[slot], ((s / STAGES) - 1) & 1, status, a.spin);
-      w = w && mbar_wait(&nib_full[ns], (s / NRING) & 1, status, a.spin);
-      ok = bar_and<2, NCONV>(w);
-      if (!ok) break;
-      const uint32_t* nib = reinterpret_cast<const uint32_t*>(sN + ns * NIB_BYTES);
-      uint8_t* dst = sW + slot * STAGE_BYTES;
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int idx = ctid + u * NCONV;  // row * 8 + word
-        const int r = idx >> 3, c = idx & 7;
-        const uint32_t wd = nib[idx];
-        const uint32_t L = wd & 0x0F0F0F0Fu, H = (wd >> 4) & 0x0F0F0F0Fu;
-        uint4 o;
-        o.x = bf16x2_minus136(prmt(L, 0x43434343u, 0x5140u));
-        o.y = bf16x2_minus136(prmt(L, 0x43434343u, 0x5342u));
-        o.z = bf16x2_minus136(prmt(H, 0x43434343u, 0x5140u));
-        o.w = bf16x2_minus136(prmt(H, 0x43434343u, 0x5342u));
-        *reinterpret_cast<uint4*>(dst + r * 128 + ((c ^ (r & 7)) << 4)) = o;
+      if (ctid == 0) {
+        if (s >= STAGES) w = poll_yield(&empty[slot], ((s / STAGES) - 1) & 1, status, a.spin);
+        w = w && poll_yield(&nib_full[ns], (s / NRING) & 1, status, a.spin);
       }
-      fence_proxy_async_smem();
+      w = bar_and<2, NCONV>(w);
+      if (w) {
+        uint32_t wd[8];
+        asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                     : "=r"(wd[0]), "=r"(wd[1]), "=r"(wd[2]), "=r"(wd[3])
+                     : "r"(nib_row + (uint32_t)(ns * NIB_BYTES)));
+        asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                     : "=r"(wd[4]), "=r"(wd[5]), "=r"(wd[6]), "=r"(wd[7])
+                     : "r"(nib_row + (uint32_t)(ns * NIB_BYTES) + 16));
+        const uint32_t dst = dst_row + (uint32_t)(slot * STAGE_BYTES);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint32_t L = wd[c] & 0x0F0F0F0Fu, H = (wd[c] >> 4) & 0x0F0F0F0Fu;
+          const uint32_t o0 = bf16x2_minus136(prmt(L, 0x43434343u, 0x5140u));
+          const uint32_t o1 = bf16x2_minus136(prmt(L, 0x43434343u, 0x5342u));
+          const uint32_t o2 = bf16x2_minus136(prmt(H, 0x43434343u, 0x5140u));
+          const uint32_t o3 = bf16x2_minus136(prmt(H, 0x43434343u, 0x5342u));
+          asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(dst + ((c ^ (r & 7)) << 4)),
+                       "r"(o0), "r"(o1), "r"(o2), "r"(o3)
+                       : "memory");
+        }
+        fence_proxy_async_smem();
+      }
+      ok = w;
+      if (!ok) break;
       bar_sync<2, NCONV>();  // every converter is done with this nibble stage
       if (ctid == 0) {
         mbar_arrive(&w_full[slot]);
         const int sn = s + NRING;
         if (sn < nst) {
           mbar_arrive_expect_tx(&nib_full[ns], NIB_BYTES);
-          tma_load_2d(sN + ns * NIB_BYTES, &tmW, (k0 + KS * sn) / 8, n0, &nib_full[ns]);
+          tma_load_2d(sN + ns * NIB_BYTES, &tm_.w, (k0 + KS * sn) / 8, n0, &nib_full[ns]);
           last_ph = (last_ph & ~(1u << ns)) | ((uint32_t)((sn / NRING) & 1) << ns);
         }
       }
@@ -613,99 +686,99 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else {
     // ---------------- epilogue ----------------
-    const int etid = threadIdx.x - EPI_WARP0 * 32;  // 0..255
+    const int etid = threadIdx.x - EPI_WARP0 * 32;  // 0..511
     const int q = warp & 3;                         // TMEM lane quarter
-    const int cb = (warp - EPI_WARP0) >> 2;         // 64-column half
+    const int cb = (warp - EPI_WARP0) >> 2;         // 32-column block of a group
     const int nl = 32 * q + lane;                   // weight row within the tile
-    // Group scales (and zeros) of this CTA's rows and K range, as [g][n]:
-    // thread (row r, half h) reads groups [16h, 16h + 16) of row r, all its
-    // loads issued before any is used (one memory round trip, not sixteen).
-    {
-      const int r = etid & (TW - 1), h = etid >> 7;
-      const int64_t base = (int64_t)(n0 + r) * G + g0 + 16 * h;
-      const bool row_ok = n0 + r < a.N;
-      float v[16], z[16];
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const bool in = row_ok && 16 * h + j < Gr;
-        v[j] = !in ? 0.0f
-                   : a.scale_bf16
-                         ? __uint_as_float((uint32_t)__ldg(reinterpret_cast<const unsigned short*>(a.wscale) + base + j) << 16)
-                         : __ldg(reinterpret_cast<const float*>(a.wscale) + base + j);
-        z[j] = (WZP && in) ? __ldg(a.wzero + base + j) : 0.0f;
-      }
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        if (16 * h + j < Gr) {
-          scl[(16 * h + j) * TW + r] = v[j];
-          if (WZP) zws[(16 * h + j) * TW + r] = z[j];
-        }
+    if (!a.tma_w) {
+      // tables by thread loads (row sizes the tensor copy cannot take)
+      for (int i = etid; i < Gr * TW; i += NEPI) {
+        const int n = i / Gr, g = i - n * Gr;
+        const int64_t idx = (int64_t)(n0 + n) * G + g0 + g;
+        const bool in = n0 + n < a.N;
+        if (a.scale_bf16)
+          *reinterpret_cast<unsigned short*>(scl + tbl_off(n, g, 2, srow)) =
+              in ? __ldg(reinterpret_cast<const unsigned short*>(a.wscale) + idx) : (unsigned short)0;
+        else
+          *reinterpret_cast<float*>(scl + tbl_off(n, g, 4, srow)) =
+              in ? __ldg(reinterpret_cast<const float*>(a.wscale) + idx) : 0.0f;
+        if (WZP) *reinterpret_cast<float*>(zws + tbl_off(n, g, 4, frow)) = in ? __ldg(a.wzero + idx) : 0.0f;
       }
     }
-    // activation scales per block / group sums come from the quantization grid
+    // activation tables come from the quantization grid
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    if (ABLK || WZP) {
+    if ((ABLK || WZP) && !a.tma_act) {
       const float* src = ABLK ? a.sA : a.Sg;
-      const int r = etid & (TM - 1), h = etid >> 7;
-      const float* p = src + (int64_t)(m0 + r) * G + g0 + 16 * h;
-      float v[16];
-#pragma unroll
-      for (int j = 0; j < 16; ++j) v[j] = 16 * h + j < Gr ? p[j] : 0.0f;
-#pragma unroll
-      for (int j = 0; j < 16; ++j)
-        if (16 * h + j < Gr) actp[(16 * h + j) * TM + r] = v[j];
+      for (int i = etid; i < Gr * TM; i += NEPI) {
+        const int mm = i / Gr, g = i - mm * Gr;
+        *reinterpret_cast<float*>(actp + tbl_off(mm, g, 4, frow)) = src[(int64_t)(m0 + mm) * G + g0 + g];
+      }
     }
-    bar_sync<1, NEPI>();
-    f32x2 acc[32];
-#pragma unroll
-    for (int j = 0; j < 32; ++j) acc[j] = 0ull;
     bool ok = true;
-    for (int g = 0; g < Gr && ok; ++g) {
-      const int buf = g % NBUF;
-      // warp-uniform decision: the TMEM loads below are .sync.aligned
-      ok = __all_sync(0xffffffffu, mbar_wait(&tfull[buf], (uint32_t)(g / NBUF) & 1, status, a.spin));
+    if (a.tma_w) ok = mbar_wait(prm_full, 0, status, a.spin);
+    if ((ABLK || WZP) && a.tma_act) ok = mbar_wait(act_full, 0, status, a.spin) && ok;
+    ok = bar_and<1, NEPI>(ok);  // also publishes the thread-loaded tables
+    f32x2 acc[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) acc[j] = 0ull;
+    for (int s = 0; s < nst && ok; ++s) {
+      const int sb = s % NSB;
+      // each warp waits on its own: lane 0 polls the accumulator barrier and
+      // the warp takes its decision together (the TMEM loads below are
+      // .sync.aligned); warps are not held in step with each other
+      bool w = true;
+      if (lane == 0) w = poll_yield(&tfull[sb], (uint32_t)(s / NSB) & 1, status, a.spin);
+      ok = __shfl_sync(0xffffffffu, (int)w, 0) != 0;
       if (!ok) break;
       tc_fence_after();
-      const float sw = scl[g * TW + nl];
-      const f32x2 s2 = pack2(sw, sw);
-      const f32x2* ap = reinterpret_cast<const f32x2*>(actp + g * TM + 64 * cb);
-      const uint32_t taddr = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * TM + 64 * cb);
-      // the two 32-column halves one after the other (32 staging registers)
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
+      for (int gi = 0; gi < 2; ++gi) {
+        const int g = 2 * s + gi;
         uint32_t p[32];
-        tmem_ld32(taddr + 32 * h, p);
+        tmem_ld32(tmem_base + ((uint32_t)(32 * q) << 16) +
+                      (uint32_t)(sb * 2 * TM + gi * TM + 32 * cb), p);
         tmem_wait_ld();
-        if (h == 1) {  // both halves read: hand the buffer back to the MMA warp
+        if (gi == 1) {  // both groups read: hand the stage buffer back
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&tempty[buf]);
+          if (lane == 0) mbar_arrive(&tempty[sb]);
         }
+        const float sw =
+            a.scale_bf16
+                ? __uint_as_float((uint32_t)*reinterpret_cast<const unsigned short*>(scl + tbl_off(nl, g, 2, srow)) << 16)
+                : *reinterpret_cast<const float*>(scl + tbl_off(nl, g, 4, srow));
+        const f32x2 s2 = pack2(sw, sw);
+        if (ABLK) {
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const f32x2 d = pack2u(p[2 * j], p[2 * j + 1]);
-          if (ABLK)
-            ffma2(acc[16 * h + j], d, fmul2(s2, ap[16 * h + j]));
-          else
-            ffma2(acc[16 * h + j], d, s2);
+          for (int j = 0; j < 16; ++j) {
+            const float a0 = *reinterpret_cast<const float*>(actp + tbl_off(32 * cb + 2 * j, g, 4, frow));
+            const float a1 = *reinterpret_cast<const float*>(actp + tbl_off(32 * cb + 2 * j + 1, g, 4, frow));
+            ffma2(acc[j], pack2u(p[2 * j], p[2 * j + 1]), fmul2(s2, pack2(a0, a1)));
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) ffma2(acc[j], pack2u(p[2 * j], p[2 * j + 1]), s2);
         }
-      }
-      if (WZP) {
-        const float zw = zws[g * TW + nl];
-        const f32x2 z2 = pack2(zw, zw);
-        const f32x2* sp = reinterpret_cast<const f32x2*>(actp + g * TM + 64 * cb);
+        if (WZP) {
+          const float zw = *reinterpret_cast<const float*>(zws + tbl_off(nl, g, 4, frow));
+          const f32x2 z2 = pack2(zw, zw);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) ffma2(acc[j], sp[j], z2);
+          for (int j = 0; j < 16; ++j) {
+            const float s0 = *reinterpret_cast<const float*>(actp + tbl_off(32 * cb + 2 * j, g, 4, frow));
+            const float s1 = *reinterpret_cast<const float*>(actp + tbl_off(32 * cb + 2 * j + 1, g, 4, frow));
+            ffma2(acc[j], pack2(s0, s1), z2);
+          }
+        }
       }
     }
     ok = bar_and<1, NEPI>(ok);
     // park the partial tile as [m][n]; every MMA has completed (the last
-    // group's accumulator was waited for), so the stage buffers are free
+    // stage's accumulators were waited for), so the stage buffers are free
     if (ok) {
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        part[(64 * cb + 2 * j) * PST + nl] = lo_f(acc[j]);
-        part[(64 * cb + 2 * j + 1) * PST + nl] = hi_f(acc[j]);
+      for (int j = 0; j < 16; ++j) {
+        part[(32 * cb + 2 * j) * PST + nl] = lo_f(acc[j]);
+        part[(32 * cb + 2 * j + 1) * PST + nl] = hi_f(acc[j]);
       }
     }
   }
@@ -714,16 +787,18 @@ __global__ void __launch_bounds__(THREADS, 1)
   // first cluster barrier every partial is visible; CTA `split` sums its
   // share of the rows over all ranks in rank order (deterministic) and
   // writes y; the second barrier keeps every CTA's shared memory alive until
-  // its peers have read it.
-  // This CTA reduces rows [r0, r1) of the tile; epilogue thread etid takes
-  // the 4-column chunk c = etid % 32 of rows r0 + etid / 32 + 8j.  Its bias
-  // and row scales are fetched before the cluster barrier, so each output
-  // waits only for the partials.
+  // its peers have read it.  This CTA reduces rows [r0, r1) of the tile;
+  // epilogue thread etid takes the 4-column chunk c = etid % 32 of rows
+  // r0 + etid / 32 + 16j.  Its bias and row scales are fetched before the
+  // cluster barrier, so each output waits only for the partials.
   const int rows_per = (TM + a.splits - 1) / a.splits;
   const int r0 = split * rows_per, r1 = min(TM, r0 + rows_per);
-  constexpr int RJ = TM / 8;  // rows per thread at most (one split)
+  constexpr int RSTEP = NEPI / 32;
+  constexpr int RJ = TM / RSTEP;  // rows per thread at most (one split)
   float bias4[4] = {0.f, 0.f, 0.f, 0.f};
-  float srow[RJ];
+  float srow_s[RJ];
+  __syncwarp();
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
   if (warp >= EPI_WARP0) {
     const int etid = threadIdx.x - EPI_WARP0 * 32;
     const int c = etid & 31;
@@ -732,12 +807,12 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (a.bias && n0 + 4 * c + e < a.N) bias4[e] = __ldg(a.bias + n0 + 4 * c + e);
 #pragma unroll
     for (int j = 0; j < RJ; ++j) {
-      const int m = m0 + r0 + (etid >> 5) + 8 * j;
-      srow[j] = (!ABLK && r0 + (etid >> 5) + 8 * j < r1 && m < a.M) ? a.sA[m] : 1.0f;
+      const int mm = r0 + (etid >> 5) + RSTEP * j;
+      srow_s[j] = (!ABLK && mm < r1 && m0 + mm < a.M) ? a.sA[m0 + mm] : 1.0f;
     }
   }
   __syncwarp();
-  cluster_sync_all();
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
   if (warp >= EPI_WARP0) {
     const int etid = threadIdx.x - EPI_WARP0 * 32;
     const uint32_t part_s = smem_u32(part);
@@ -745,7 +820,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int c = etid & 31;
 #pragma unroll
     for (int jr = 0; jr < RJ; ++jr) {
-      const int mm = r0 + (etid >> 5) + 8 * jr;
+      const int mm = r0 + (etid >> 5) + RSTEP * jr;
       const int m = m0 + mm, n = n0 + 4 * c;
       if (mm >= r1 || m >= a.M || n >= a.N) continue;
       const uint32_t off = (uint32_t)((mm * PST + 4 * c) * 4);
@@ -754,7 +829,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
       for (int j = 0; j < MAX_SPLITS; ++j)
         if (j < a.splits) t[j] = ld_dsmem_f4(mapa(part_s + off, (uint32_t)j));
-      const float s = srow[jr];
+      const float s = srow_s[jr];
       float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
       for (int j = 0; j < MAX_SPLITS; ++j) {
@@ -782,8 +857,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
     }
   }
+  // peers may still read this CTA's partial tile: leave only after all have
+  // finished (no memory ordering is needed for that)
   __syncwarp();
-  cluster_sync_all();
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;\n\tbarrier.cluster.wait.aligned;" ::: "memory");
 
   // Reconverge every warp (single lanes ran the copy and MMA loops) so the
   // CTA barrier below counts complete warps, then free TMEM.
@@ -793,7 +870,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (warp == 1) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
-                 "r"(NBUF * TM)
+                 "r"(NSB * 2 * TM)
                  : "memory");
   }
 }
@@ -904,10 +981,11 @@ int launch_a8w4_tc_call(const A8W4TcCall& c, void* ws, size_t ws_bytes, cudaStre
   if (rc != QG_OK) return rc;
 
   const uint8_t* wq = (const uint8_t*)c.packed;
-  CUtensorMap tmW;
-  rc = make_tmap_generic(&tmW, CU_TENSOR_MAP_DATA_TYPE_UINT32, wq, (uint64_t)c.K / 8,
+  TcMaps maps;
+  rc = make_tmap_generic(&maps.w, CU_TENSOR_MAP_DATA_TYPE_UINT32, wq, (uint64_t)c.K / 8,
                          (uint64_t)c.N, (uint64_t)c.K / 2, KS / 8, TW, CU_TENSOR_MAP_SWIZZLE_NONE);
   if (rc != QG_OK) return rc;
+  maps.scl = maps.zw = maps.act = maps.w;
   GemmArgs ga{};
   ga.M = (int)c.M; ga.N = c.N; ga.K = c.K;
   ga.Kr = c.K / p.splits; ga.splits = p.splits; ga.n_tiles = p.n_tiles; ga.nkb = c.K / KS;
@@ -918,6 +996,39 @@ int launch_a8w4_tc_call(const A8W4TcCall& c, void* ws, size_t ws_bytes, cudaStre
   ga.sA = qa.sA;
   ga.Sg = qa.Sg;
   ga.bias = c.bias; ga.lo = c.lo; ga.hi = c.hi; ga.y = c.y; ga.ldy = c.ldy;
+  // The per-group tables by tensor copy when a CTA's row of them is 32, 64
+  // or 128 bytes and the global rows are 16-byte multiples (else thread loads).
+  const int G = c.K / 32, Gr = ga.Kr / 32;
+  auto swz_for = [](int rowbytes) {
+    return rowbytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                           : rowbytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
+  };
+  auto tma_ok = [](int rowbytes, int64_t pitch, const void* base) {
+    return (rowbytes == 32 || rowbytes == 64 || rowbytes == 128) && pitch % 16 == 0 &&
+           ((uintptr_t)base & 15) == 0;
+  };
+  const int sesz = c.scale_bf16 ? 2 : 4;
+  ga.tma_w = tma_ok(Gr * sesz, (int64_t)G * sesz, ga.wscale) &&
+             (!c.wzero || tma_ok(Gr * 4, (int64_t)G * 4, c.wzero));
+  if (ga.tma_w) {
+    rc = make_tmap_generic(&maps.scl,
+                           c.scale_bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                           ga.wscale, (uint64_t)G, (uint64_t)c.N, (uint64_t)G * sesz, (uint32_t)Gr,
+                           TW, swz_for(Gr * sesz));
+    if (rc != QG_OK) return rc;
+    if (c.wzero) {
+      rc = make_tmap_generic(&maps.zw, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, c.wzero, (uint64_t)G,
+                             (uint64_t)c.N, (uint64_t)G * 4, (uint32_t)Gr, TW, swz_for(Gr * 4));
+      if (rc != QG_OK) return rc;
+    }
+  }
+  const float* act_src = c.mode == kBlockAsym ? qa.sA : qa.Sg;
+  ga.tma_act = act_src && tma_ok(Gr * 4, (int64_t)G * 4, act_src);
+  if (ga.tma_act) {
+    rc = make_tmap_generic(&maps.act, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, act_src, (uint64_t)G,
+                           (uint64_t)p.Mpad, (uint64_t)G * 4, (uint32_t)Gr, TM, swz_for(Gr * 4));
+    if (rc != QG_OK) return rc;
+  }
   ga.stall = take_stall(kStallA8W4TC) ? 1 : 0;
   ga.spin = ga.stall ? kStallSpinLimit : kSpinLimit;
   cudaLaunchConfig_t cfg = {};
@@ -931,18 +1042,18 @@ int launch_a8w4_tc_call(const A8W4TcCall& c, void* ws, size_t ws_bytes, cudaStre
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   // programmatic dependent launch: barriers, TMEM, the weight nibbles and
-  // scales overlap the quantization grid
+  // tables overlap the quantization grid
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
   cudaError_t e;
   if (c.mode == kBlockAsym)
-    e = cudaLaunchKernelEx(&cfg, a8w4_tc_kernel<true, false>, tmW, ga, status_word());
+    e = cudaLaunchKernelEx(&cfg, a8w4_tc_kernel<true, false>, maps, ga, status_word());
   else if (c.wzero)
-    e = cudaLaunchKernelEx(&cfg, a8w4_tc_kernel<false, true>, tmW, ga, status_word());
+    e = cudaLaunchKernelEx(&cfg, a8w4_tc_kernel<false, true>, maps, ga, status_word());
   else
-    e = cudaLaunchKernelEx(&cfg, a8w4_tc_kernel<false, false>, tmW, ga, status_word());
+    e = cudaLaunchKernelEx(&cfg, a8w4_tc_kernel<false, false>, maps, ga, status_word());
   return e == cudaSuccess ? QG_OK : QG_ERR_CUDA;
 }
 
