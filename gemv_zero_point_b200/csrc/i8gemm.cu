@@ -38,6 +38,8 @@ constexpr int A_STAGE = BM * BK;  // 16 KiB
 constexpr int B_STAGE = BN * BK;  // 32 KiB
 constexpr int TMEM_COLS = 2 * BN; // double-buffered accumulator
 constexpr int THREADS = 192;      // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
+constexpr int CONV_PW = 4;        // implicit-im2col gather warps: one A row per thread
+constexpr int THREADS_CONV = (CONV_PW + 5) * 32;  // + MMA warp + 4 epilogue warps
 constexpr size_t SMEM_BYTES = 1024 /*align slack*/ + STAGES * (A_STAGE + B_STAGE) + 4096;
 
 // Instruction descriptor for kind::i8: D s32, A s8, B s8, both K-major,
@@ -182,69 +184,103 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
                : "memory");
 }
 
-__device__ __forceinline__ int conv_byte(const ConvGather& g, int n, int oh, int ow, int k) {
-  const int tap = k / g.Cin, ci = k - tap * g.Cin;
-  const int kh = tap / g.KW, kw = tap - kh * g.KW;
-  const int ih = oh * g.sh + kh - g.ph, iw = ow * g.sw + kw - g.pw;
-  if (ih < 0 || ih >= g.H || iw < 0 || iw >= g.W) return g.za;
-  return g.x[(((int64_t)n * g.H + ih) * g.W + iw) * g.Cin + ci];
+// The output pixel of im2col row m, decoded once per tile: its image and
+// the input coordinates of tap (0, 0).
+struct ConvRow {
+  const int8_t* img;
+  int ihb, iwb;
+  bool ok;
+};
+__device__ __forceinline__ ConvRow conv_row(const ConvGather& g, int m) {
+  ConvRow cr;
+  cr.ok = m < g.M;
+  const int mm = cr.ok ? m : 0;
+  const int ow = mm % g.OW, t = mm / g.OW;
+  const int oh = t % g.OH, n = t / g.OH;
+  cr.ihb = oh * g.sh - g.ph;
+  cr.iwb = ow * g.sw - g.pw;
+  cr.img = g.x + (int64_t)n * g.H * g.W * g.Cin;
+  return cr;
 }
 
-// Rows lane, lane+32, lane+64, lane+96 of tile tm, K block kb.
-__device__ __forceinline__ void conv_gather_stage(const ConvGather& g, uint8_t* dst_stage, int tm,
-                                                  int kb, int lane) {
+// Row r of K block kb into the swizzled stage (row r at byte r*128, 16-byte
+// chunk c at position c ^ (r & 7)).  With Cin % 16 == 0 and a 16-byte
+// aligned input, a 16-byte chunk of K lies inside one tap: lane c of the
+// warp decodes chunk c of the block (tap, channel) and the warp shares it,
+// then each thread copies its row's chunk with cp.async, or writes the
+// input zero-point where the tap falls in the padding.  Otherwise the bytes
+// are read one by one (first layers with few channels), stepping
+// (kh, kw, ci) along K without divisions.  K positions at or beyond K are
+// left as they are: the packed weights are zero there.
+__device__ __forceinline__ void conv_gather_row(const ConvGather& g, const ConvRow& cr,
+                                                uint8_t* drow, int r, int kb, int lane) {
   const uint32_t za4 = (uint32_t)(uint8_t)g.za * 0x01010101u;
-#pragma unroll 1
-  for (int i = 0; i < 4; ++i) {
-    const int r = lane + 32 * i;
-    const int m = tm * BM + r;
-    if (m >= g.M) continue;
-    const int ow = m % g.OW;
-    const int t = m / g.OW;
-    const int oh = t % g.OH, n = t / g.OH;
-    uint8_t* drow = dst_stage + r * 128;
-    if (g.vec16) {
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const int k = kb * BK + 16 * c;
-        if (k >= g.K) break;
-        uint8_t* d = drow + ((c ^ (r & 7)) << 4);
-        const int tap = k / g.Cin, ci = k - tap * g.Cin;
-        const int kh = tap / g.KW, kw = tap - kh * g.KW;
-        const int ih = oh * g.sh + kh - g.ph, iw = ow * g.sw + kw - g.pw;
-        if (ih >= 0 && ih < g.H && iw >= 0 && iw < g.W)
-          cp_async16(smem_u32(d), g.x + (((int64_t)n * g.H + ih) * g.W + iw) * g.Cin + ci);
-        else
-          *reinterpret_cast<uint4*>(d) = make_uint4(za4, za4, za4, za4);
+  const int k0 = kb * BK;
+  if (g.vec16) {
+    int ckh = -1, ckw = 0, cci = 0;
+    if (lane < 8) {
+      const int k = k0 + 16 * lane;
+      if (k < g.K) {
+        const int tap = k / g.Cin;
+        cci = k - tap * g.Cin;
+        ckh = tap / g.KW;
+        ckw = tap - ckh * g.KW;
       }
-    } else {
+    }
+    int kh[8], kw[8], ci[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      kh[c] = __shfl_sync(0xffffffffu, ckh, c);
+      kw[c] = __shfl_sync(0xffffffffu, ckw, c);
+      ci[c] = __shfl_sync(0xffffffffu, cci, c);
+    }
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      if (kh[c] < 0) break;
+      uint8_t* d = drow + ((c ^ (r & 7)) << 4);
+      const int ih = cr.ihb + kh[c], iw = cr.iwb + kw[c];
+      if (cr.ok && (unsigned)ih < (unsigned)g.H && (unsigned)iw < (unsigned)g.W)
+        cp_async16(smem_u32(d), cr.img + ((int64_t)ih * g.W + iw) * g.Cin + ci[c]);
+      else
+        *reinterpret_cast<uint4*>(d) = make_uint4(za4, za4, za4, za4);
+    }
+  } else {
+    if (k0 >= g.K) return;
+    int tap = k0 / g.Cin;
+    int ci = k0 - tap * g.Cin;
+    int kh = tap / g.KW;
+    int kw = tap - kh * g.KW;
 #pragma unroll 1
-      for (int c = 0; c < 8; ++c) {
-        const int k0 = kb * BK + 16 * c;
-        if (k0 >= g.K) break;
-        uint32_t wv[4];
+    for (int c = 0; c < 8; ++c) {
+      if (k0 + 16 * c >= g.K) break;
+      uint32_t wv[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint32_t word = 0;
-#pragma unroll
-          for (int b = 0; b < 4; ++b) {
-            const int k = k0 + 4 * q + b;
-            const int v = k < g.K ? conv_byte(g, n, oh, ow, k) : 0;
-            word |= ((uint32_t)v & 0xFFu) << (8 * b);
+      for (int b = 0; b < 16; ++b) {
+        const int k = k0 + 16 * c + b;
+        const int ih = cr.ihb + kh, iw = cr.iwb + kw;
+        int v = g.za;
+        if (k < g.K && cr.ok && (unsigned)ih < (unsigned)g.H && (unsigned)iw < (unsigned)g.W)
+          v = cr.img[((int64_t)ih * g.W + iw) * g.Cin + ci];
+        wv[b >> 2] |= ((uint32_t)v & 0xFFu) << (8 * (b & 3));
+        if (++ci == g.Cin) {
+          ci = 0;
+          if (++kw == g.KW) {
+            kw = 0;
+            ++kh;
           }
-          wv[q] = word;
         }
-        *reinterpret_cast<uint4*>(drow + ((c ^ (r & 7)) << 4)) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
       }
+      *reinterpret_cast<uint4*>(drow + ((c ^ (r & 7)) << 4)) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
     }
   }
 }
 
 // CONV = false: A is a row-major matrix read by the tensor-copy engine.
-// CONV = true: A is the implicit im2col of `cg`, gathered by the whole
-// producer warp (see conv_gather_stage); B still comes by tensor copies.
+// CONV = true: A is the implicit im2col of `cg`, gathered by CONV_PW warps
+// (one tile row per thread, see conv_gather_row); B still comes by tensor
+// copies.  Warp roles: producers, then the MMA warp, then 4 epilogue warps.
 template <bool CONV>
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __launch_bounds__(CONV ? THREADS_CONV : THREADS, 1)
     i8gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      int num_kb, int tiles_m, int tiles_n, EpiArgs ep, ConvGather cg, int* status) {
   extern __shared__ uint8_t smem_raw[];
@@ -261,12 +297,14 @@ __global__ void __launch_bounds__(THREADS, 1)
   int32_t* c_m0 = c_term + BN;                   // [BN]
   int32_t* c_sh = c_m0 + BN;                     // [BN]
 
+  constexpr int PW = CONV ? CONV_PW : 1;  // producer warps
+  constexpr int MMA_WARP = PW, EPI_WARP0 = PW + 1;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tiles = tiles_m * tiles_n;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], CONV ? 32 : 1);  // conv: every producer lane arrives
+      mbar_init(&full[s], CONV ? 32 * PW : 1);  // conv: every producer thread arrives
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -278,7 +316,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (!CONV) prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
   }
-  if (warp == 1) {
+  if (warp == MMA_WARP) {
     tmem_alloc(tmem_slot, TMEM_COLS);
     tmem_relinquish();
   }
@@ -287,27 +325,31 @@ __global__ void __launch_bounds__(THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  if (CONV && warp == 0) {
-    // ---------------- implicit-im2col producer (whole warp) ----------------
-    // Stage s is signalled one stage late: after the copies of stage s+1 are
-    // issued, each lane waits for its own copies of stage s, makes them and
-    // its zero-point fills visible to the tensor cores, and arrives.
+  if (CONV && warp < PW) {
+    // ---------------- implicit-im2col producers ----------------
+    // Thread ptid gathers row ptid of every tile.  Stage s is signalled one
+    // stage late: after the copies of stage s+1 are issued, each thread
+    // waits for its own copies of stage s, makes them and its zero-point
+    // fills visible to the tensor cores, and arrives.  Warp 0 lane 0 also
+    // issues the weight tensor copies.
+    const int ptid = threadIdx.x;  // 0 .. 32*PW-1
     int stage = 0, prev = -1;
     uint32_t phase = 0;
-    uint32_t issued = 0, last_ph = 0;  // B tensor copies (lane 0)
+    uint32_t issued = 0, last_ph = 0;  // B tensor copies (thread 0)
     for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
       const int tm = t % tiles_m, tn = t / tiles_m;
+      const ConvRow cr = conv_row(cg, tm * BM + ptid);
       for (int kb = 0; kb < num_kb; ++kb) {
         bool got = true;
         if (lane == 0) got = mbar_poll(&empty[stage], phase ^ 1, status, ep.spin);
         if (!__shfl_sync(0xffffffffu, (int)got, 0)) goto conv_done;
-        if (lane == 0) {
+        if (ptid == 0) {
           mbar_expect_tx(&full[stage], B_STAGE);
           tma_load_2d(sB + stage * B_STAGE, &tmB, kb * BK, tn * BN, &full[stage]);
           issued |= 1u << stage;
           last_ph = (last_ph & ~(1u << stage)) | (phase << stage);
         }
-        conv_gather_stage(cg, sA + stage * A_STAGE, tm, kb, lane);
+        conv_gather_row(cg, cr, sA + stage * A_STAGE + ptid * BK, ptid, kb, lane);
         cp_async_commit();
         if (prev >= 0) {
           cp_async_wait<1>();
@@ -325,7 +367,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     cp_async_wait<0>();
     fence_proxy_async_smem();
     if (prev >= 0) mbar_arrive(&full[prev]);
-    if (lane == 0)
+    if (ptid == 0)
       for (int st = 0; st < STAGES; ++st)
         if ((issued >> st) & 1u) mbar_poll(&full[st], (last_ph >> st) & 1u, status);
   } else if (warp == 0) {
@@ -357,7 +399,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int st = 0; st < STAGES; ++st)
         if ((issued >> st) & 1u) mbar_poll(&full[st], (last_ph >> st) & 1u, status);
     }
-  } else if (warp == 1) {
+  } else if (warp == MMA_WARP) {
     // ------------------------- MMA issuer -------------------------
     if (lane == 0) {
       int stage = 0;
@@ -402,7 +444,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else {
     // ------------------------- epilogue -------------------------
     const int q = warp & 3;                 // TMEM lane quarter of this warp
-    const int etid = threadIdx.x - 64;      // 0..127
+    const int etid = threadIdx.x - 32 * EPI_WARP0;  // 0..127
     const int row_in_tile = 32 * q + lane;
     const int64_t Kza_zb = (int64_t)ep.K * ep.za * ep.zb;
     int local = 0;
@@ -481,7 +523,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncwarp();
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem_base, TMEM_COLS);
   }
@@ -1108,7 +1150,7 @@ int conv_run_packed(int Nb, int H, int W, int Cin, int Cout, int KH, int KW, int
   const int tiles_m = (int)cdiv(M, BM), tiles_n = (int)cdiv(Cout, BN);
   const int tiles = tiles_m * tiles_n;
   const int grid = tiles < num_sms() ? tiles : num_sms();
-  i8gemm_tc_kernel<true><<<grid, THREADS, SMEM_BYTES, st>>>(tmB, tmB, num_kb, tiles_m, tiles_n,
+  i8gemm_tc_kernel<true><<<grid, THREADS_CONV, SMEM_BYTES, st>>>(tmB, tmB, num_kb, tiles_m, tiles_n,
                                                             ep, cg, status_word());
   return launch_status();
 }
