@@ -99,6 +99,45 @@ def test_gemm_shapes(lib, M, N, K, per_channel, zb):
     check_gemm(lib, w)
 
 
+# M > 128 runs on CTA pairs.  Rows the tensor-copy engine cannot address
+# (pitch or base not a multiple of 16 bytes) are first copied to a 16-byte
+# pitch.  Cases: pitches 8, 4 and 1 (mod 16), a base offset into the
+# allocation, b_zero_point != 0 (row sums), ragged M / N / K, and more tiles
+# than resident CTA pairs (the stage ring wraps across tiles).
+PAIR_UNALIGNED = [
+    # M,   N,    K,   lda, a_off, zb
+    (300, 300, 264, 264, 0, 0),       # pitch = 8 (mod 16)
+    (257, 520, 1000, 1004, 0, 0),     # pitch = 4 (mod 8)
+    (384, 256, 1000, 1000, 8, 0),     # base 8 bytes into the allocation
+    (300, 300, 264, 264, 4, 5),       # base 4 bytes in, b zero-point (row sums)
+    (260, 130, 131, 131, 0, 0),       # odd pitch
+    (4096, 2560, 136, 136, 0, 0),     # 160 pair tiles
+]
+
+
+@pytest.mark.parametrize("M,N,K,lda,a_off,zb", PAIR_UNALIGNED)
+def test_gemm_pair_unaligned_rows(lib, M, N, K, lda, a_off, zb):
+    w = workloads.int8_gemm(M, N, K, 7000 + M + lda, zb=zb, per_channel=True, lda=lda,
+                            ratio_range=(1e-5, 1e-3))
+    flat = torch.full((M * lda + a_off + 16,), 99, dtype=torch.int8, device="cuda")
+    flat[a_off:a_off + M * lda].copy_(_dev(w["A"]).reshape(-1))
+    A = torch.as_strided(flat, (M, K), (lda, 1), a_off)
+    B = _dev(w["B"])[:, :N]
+    mult, shift, m0, sh = _params(lib, w)
+    rq = lib.make_requant(a_zero_point=w["za"], b_zero_point=w["zb"], bias=_dev(w["bias"]),
+                          multiplier=mult, shift=shift, out_zero_point=w["out_zp"],
+                          clamp_min=w["clamp_min"], clamp_max=w["clamp_max"])
+    C = torch.full((M, N), 55, dtype=torch.int8, device="cuda")
+    acc = torch.full((M, N), 7, dtype=torch.int32, device="cuda")
+    lib.qgemm_s8s8_requant_packed(A, lib.qgemm_pack_b_s8(B), N, C, rq, K=K, acc_out=acc)
+    torch.cuda.synchronize()
+    C_ref, acc_ref = oracle.qgemm_s8s8_requant(w["A"][:, :K], w["B"][:, :N], w["za"], w["zb"],
+                                               w["bias"], m0, sh, w["out_zp"], w["clamp_min"],
+                                               w["clamp_max"])
+    np.testing.assert_array_equal(acc.cpu().numpy(), acc_ref)
+    np.testing.assert_array_equal(C.cpu().numpy(), C_ref)
+
+
 def test_gemm_relu_clamp_and_no_bias(lib):
     w = workloads.int8_gemm(200, 96, 200, seed=77, with_bias=False, out_zp=-10,
                             clamp=(-10, 127))
