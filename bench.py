@@ -485,16 +485,16 @@ def build_cases(workload, qg, torch):
     if workload == "a8w4_gemv_1x14336x4096":
         return [("a8w4_gemv_1x14336x4096", A8W4Case(qg, torch, W.a8w4_gemv_1x14336x4096(), 8), "hbm")]
     if workload == "a8w4_gemm_128x4096x4096":
-        return [("a8w4_gemm_128x4096x4096", A8W4Case(qg, torch, W.a8w4_gemm_128x4096x4096(), 16), "hbm")]
+        return [("a8w4_gemm_128x4096x4096", A8W4Case(qg, torch, W.a8w4_gemm_128x4096x4096(), 16), "tensor_bf16")]
     if workload == "a8w4_gemv_asym_1x14336x4096":   # asymmetric int4 weights (44 MB per set)
         return [("a8w4_gemv_asym_1x14336x4096",
                  A8W4Case(qg, torch, W.a8w4_gemv_1x14336x4096(), 7, asym=True), "hbm")]
     if workload == "a8w4_gemm_actblock_128x4096x4096":
         return [("a8w4_gemm_actblock_128x4096x4096",
-                 A8W4Case(qg, torch, W.a8w4_gemm_128x4096x4096(), 16, actblock=True), "hbm")]
+                 A8W4Case(qg, torch, W.a8w4_gemm_128x4096x4096(), 16, actblock=True), "tensor_bf16")]
     if workload == "a8w4_gemm_asym_128x4096x4096":
         return [("a8w4_gemm_asym_128x4096x4096",
-                 A8W4Case(qg, torch, W.a8w4_gemm_128x4096x4096(), 12, asym=True), "hbm")]
+                 A8W4Case(qg, torch, W.a8w4_gemm_128x4096x4096(), 12, asym=True), "tensor_bf16")]
     if workload == "a8w4_gemv_actblock_1x14336x4096":   # activations quantized per K block
         return [("a8w4_gemv_actblock_1x14336x4096",
                  A8W4Case(qg, torch, W.a8w4_gemv_1x14336x4096(), 8, actblock=True), "hbm")]
@@ -976,6 +976,21 @@ def main():
                                "frac_of_nominal_int8": kt / NOMINAL_INT8_TOPS,
                                "traffic": traffic_for(name),
                                "peak_source": f"{peak_src} bf16 {'sustained' if k_sust else 'burst'} x {INT8_OVER_BF16:g} (int8/bf16 nominal)"}
+        elif bound == "tensor_bf16":
+            # int8 x int4 work done as exact bf16 MMAs: the bf16 tensor rate
+            # bounds it (at M = 128 its time at that rate exceeds the time to
+            # stream the weights at the copy bandwidth)
+            kt = c.ops() / tk / 1e12
+            k_clk = (part_timing[j] or {}).get("clocks") or {}
+            k_sust = "sw_power_cap" in k_clk.get("reasons", [])
+            k_peak = peaks["bf16_tflops_sustained"] if k_sust else peaks["bf16_tflops"]
+            kb = c.bytes() / tk / 1e9
+            part["frac_of_hbm"] = part["GB/s"] / peaks["hbm_gbs"]
+            rooflines[name] = {"bound": "tensor", "achieved": kt, "peak": k_peak,
+                               "unit": "TFLOP/s", "frac": kt / k_peak,
+                               "hbm_frac": kb / peaks["hbm_gbs"],
+                               "traffic": traffic_for(name),
+                               "peak_source": f"{peak_src} bf16 {'sustained' if k_sust else 'burst'} (the MMAs are bf16)"}
         else:
             kb = c.bytes() / tk / 1e9
             part["frac_of_hbm"] = part["GB/s"] / peaks["hbm_gbs"]

@@ -315,6 +315,12 @@ __device__ __forceinline__ float4 ld_cg_f4(const float* p) {
   return v;
 }
 
+__device__ __forceinline__ uint32_t ld_stream_u32(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
+  return v;
+}
+
 __device__ __forceinline__ float ld_stream_f32(const float* p) {
   float v;
   asm volatile("ld.global.nc.L1::no_allocate.f32 %0, [%1];" : "=f"(v) : "l"(p));
@@ -577,7 +583,12 @@ __global__ void __launch_bounds__(W * 32, 1) a8w4_gemv_stream_kernel(
   static_assert(W % GPL == 0, "split rows need W to be a multiple of GPL");
 
   uint4 wbuf[D][GPL];
-  float sbuf[D][GPL];
+  float sbuf[SBF ? 1 : D][GPL];
+  // SBF: the row's bf16 scales as 32-bit words, read whole (lane l holds
+  // words l, l + 32, ...: 128 contiguous bytes per load) and handed to the
+  // lanes of their groups by shuffles when the row is used
+  constexpr int SW = (GPL + 1) / 2;
+  uint32_t swd[SBF ? D : 1][SW];
   float zbuf[WZP ? D : 1][GPL];  // WZP: f32 weight zero of each group
   // loads of this warp's row j into buffer u (nothing past the last row)
   const uint32_t ssel = (lane & 1) ? 0x3244u : 0x1044u;  // bf16 half of the scale word
@@ -589,8 +600,16 @@ __global__ void __launch_bounds__(W * 32, 1) a8w4_gemv_stream_kernel(
         const int g = lane + 32 * i;
         if (g < G) {
           wbuf[u][i] = ld_stream_u4(wq + (int64_t)r * rowbytes + 16 * g);
-          sbuf[u][i] = ld_row_scale<SBF>(wscale, r, G, lane, i, ssel);
+          if constexpr (!SBF) sbuf[u][i] = ld_row_scale<false>(wscale, r, G, lane, i, ssel);
           if constexpr (WZP) zbuf[u][i] = ld_stream_f32(wzero + (int64_t)r * G + g);
+        }
+      }
+      if constexpr (SBF) {
+        const uint32_t* rw = reinterpret_cast<const uint32_t*>(wscale) + (int64_t)r * (G >> 1);
+#pragma unroll
+        for (int jj = 0; jj < SW; ++jj) {
+          const int w = lane + 32 * jj;
+          swd[u][jj] = w < (G >> 1) ? ld_stream_u32(rw + w) : 0u;
         }
       }
     }
@@ -768,11 +787,25 @@ __global__ void __launch_bounds__(W * 32, 1) a8w4_gemv_stream_kernel(
       const int j = j0 + u;
       if (j < nrows) {
         float acc = 0.0f;
+        float scv[GPL];
+#pragma unroll
+        for (int i = 0; i < GPL; ++i) {
+          if constexpr (SBF) {
+            // group g = lane + 32i: word g / 2 = lane / 2 + 16i of the row
+            const uint32_t wv =
+                __shfl_sync(0xffffffffu, swd[u][i >> 1], (lane >> 1) + 16 * (i & 1));
+            uint32_t d;
+            asm("prmt.b32 %0, %1, 0, %2;" : "=r"(d) : "r"(wv), "r"(ssel));
+            scv[i] = __uint_as_float(d);
+          } else {
+            scv[i] = sbuf[u][i];
+          }
+        }
 #pragma unroll
         for (int i = 0; i < GPL; ++i) {
           const int g = lane + 32 * i;
           if (g < G) {
-            const float sc = ABLK ? __fmul_rn(sbuf[u][i], sag[i]) : sbuf[u][i];
+            const float sc = ABLK ? __fmul_rn(scv[i], sag[i]) : scv[i];
             acc = fmaf(sc, (float)group_dot(wbuf[u][i], a[i], cseed[i], zag[i]), acc);
             if constexpr (WZP) acc = fmaf(zbuf[u][i], asum[i], acc);
           }
