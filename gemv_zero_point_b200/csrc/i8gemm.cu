@@ -652,17 +652,35 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (warp == 0) {
     // ------------------------- TMA producer (both CTAs) -------------------------
     if (lane == 0) {
-      int stage = 0;
+      // B never comes from the grid this one may overlap (the A staging
+      // pass, launched as its programmatic primary): the first ring's worth
+      // of B tiles is requested before the grid dependency wait, A after it.
+      int pre = 0;
+      for (int t = pair, kb = 0; pre < P_STAGES && t < tiles; ++pre) {
+        int tm, tn;
+        pair_tile_coords(t, tiles_m, tiles_n, tm, tn);
+        const uint32_t fb = mapa_u32(smem_u32(&full[pre]), 0);
+        if (leader) mbar_arrive_expect_tx(&full[pre], 2u * 2u * P_STAGE);
+        tma_load_2d_pair(sB + pre * P_STAGE, &tmB, kb * BK, tn * 256 + (int)rank * BM, fb);
+        if (++kb == num_kb) {
+          kb = 0;
+          t += npairs;
+        }
+      }
+      asm volatile("griddepcontrol.wait;" ::: "memory");
+      int stage = 0, it = 0;
       uint32_t phase = 0;
       for (int t = pair; t < tiles; t += npairs) {
         int tm, tn;
         pair_tile_coords(t, tiles_m, tiles_n, tm, tn);
-        for (int kb = 0; kb < num_kb; ++kb) {
-          if (!mbar_poll(&empty[stage], phase ^ 1, status)) goto producer_done;
+        for (int kb = 0; kb < num_kb; ++kb, ++it) {
           const uint32_t fb = mapa_u32(smem_u32(&full[stage]), 0);
-          if (leader) mbar_arrive_expect_tx(&full[stage], 2u * 2u * P_STAGE);
+          if (it >= pre) {  // slots of the first ring pass were set up above
+            if (!mbar_poll(&empty[stage], phase ^ 1, status)) goto producer_done;
+            if (leader) mbar_arrive_expect_tx(&full[stage], 2u * 2u * P_STAGE);
+            tma_load_2d_pair(sB + stage * P_STAGE, &tmB, kb * BK, tn * 256 + (int)rank * BM, fb);
+          }
           tma_load_2d_pair(sA + stage * P_STAGE, &tmA, kb * BK, tm * 256 + (int)rank * BM, fb);
-          tma_load_2d_pair(sB + stage * P_STAGE, &tmB, kb * BK, tn * 256 + (int)rank * BM, fb);
           if (++stage == P_STAGES) {
             stage = 0;
             phase ^= 1;
@@ -729,6 +747,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       epi_bar_sync();
       const int m = tm * 256 + (int)rank * BM + row_in_tile;
       const bool row_ok = m < ep.M;
+      if (local == 0) asm volatile("griddepcontrol.wait;" ::: "memory");  // row sums
       const int32_t r_term = (ep.rowsum && row_ok) ? -ep.zb * ep.rowsum[m] : 0;
       const bool ok = epi_bar_and(mbar_wait(&tfull[buf], use & 1, status, ep.spin));
       tc_fence_after();
@@ -854,6 +873,9 @@ __global__ void pack_b_kmajor_kernel(int K, int N, const int8_t* __restrict__ W,
 __global__ void __launch_bounds__(256) stage_a_kernel(int K, const int8_t* __restrict__ A,
                                                       int64_t lda, int8_t* __restrict__ Aw,
                                                       int64_t ldw, int32_t* __restrict__ rowsum) {
+  // the GEMM grid may start its prologue and its B copies now; it waits for
+  // this grid before it reads the staged rows or the row sums
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   __shared__ int red[8];
   const int64_t m = blockIdx.x;
   const int8_t* src = A + m * lda;
@@ -1083,13 +1105,18 @@ int i8gemm_run_packed(int M, int N, int K, const int8_t* A, int64_t lda, const v
     cfg.blockDim = dim3(THREADS);
     cfg.dynamicSmemBytes = P_SMEM_BYTES;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    // after this call's staging pass: programmatic dependent launch (the
+    // staging grid started only once all earlier work had finished, so
+    // everything but its own output is complete when this grid starts)
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = (need_copy || need_rowsum) ? 2 : 1;
     cudaError_t e = cudaLaunchKernelEx(&cfg, i8gemm_tc2_kernel, tmA, tmB, num_kb, tiles_m, tiles_n,
                                        ep, status_word());
     return e == cudaSuccess ? QG_OK : QG_ERR_CUDA;
