@@ -90,7 +90,7 @@ constexpr size_t OFF_W = OFF_A + (size_t)STAGES * STAGE_BYTES;     // weight sta
 constexpr size_t OFF_N = OFF_W + (size_t)STAGES * STAGE_BYTES;     // nibble ring
 constexpr size_t OFF_SCL = OFF_N + (size_t)NRING * NIB_BYTES;      // [TW][Gr] weight scales
 constexpr size_t OFF_ZW = OFF_SCL + (size_t)GR_MAX * TW * 4;       // [TW][Gr] weight zeros
-constexpr size_t OFF_ACT = OFF_ZW + (size_t)GR_MAX * TW * 4;       // [TM][Gr] act scales / sums
+constexpr size_t OFF_ACT = OFF_ZW + (size_t)GR_MAX * TW * 4;       // [Gr][TM] act scales / sums
 constexpr size_t OFF_BAR = OFF_ACT + (size_t)GR_MAX * TM * 4;
 constexpr size_t SMEM_BYTES = 1024 + OFF_BAR + 512;
 static_assert((size_t)TM * PST * 4 <= OFF_N, "partial tile reuses the stage buffers");
@@ -257,8 +257,8 @@ struct QuantArgs {
   RowSource src;
   int vec4;             // the 8 floats of a chunk can be read as two aligned float4
   uint16_t* atile;      // [Mpad/128][K/64][128][64] bf16 (qA - zA), swizzled
-  float* sA;            // per-row scale [Mpad], or per-block [Mpad][K/32]
-  float* Sg;            // per-block sums of qA - zA [Mpad][K/32] (weight zeros), or NULL
+  float* sA;            // per-row scale [Mpad], or per-block [K/32][Mpad] (transposed)
+  float* Sg;            // per-block sums of qA - zA [K/32][Mpad] (weight zeros), or NULL
   int8_t* q_out;        // optional [M][K] codes
   int q_vec;            // q_out is 8-byte aligned
   float* scale_out;     // optional [M] (per row) or [M][K/32] (per block)
@@ -443,13 +443,15 @@ __global__ void __launch_bounds__(QT) a8w4_quant_tiles_kernel(QuantArgs a, int R
         for (int e = 0; e < 8; ++e) qo[e] = (int8_t)code[e];
       }
     }
+    // per-group tables for the GEMM transposed, [G][Mpad]; the caller's
+    // outputs stay [M][G]
     if (MODE == kBlockAsym && (t & 3) == 0) {
       const int64_t b = m * G + (c >> 2);
-      a.sA[b] = q.scale;
+      a.sA[(int64_t)(c >> 2) * a.Mpad + m] = q.scale;
       if (a.scale_out) a.scale_out[b] = q.scale;
       if (a.zp_out) a.zp_out[b] = q.zp;
     }
-    if (a.Sg && (t & 3) == 0) a.Sg[m * G + (c >> 2)] = (float)csum;
+    if (a.Sg && (t & 3) == 0) a.Sg[(int64_t)(c >> 2) * a.Mpad + m] = (float)csum;
   }
   if (MODE != kBlockAsym && t == 0 && m < a.Mpad) {
     a.sA[m] = live ? rowq.scale : 0.0f;
@@ -467,8 +469,9 @@ struct GemmArgs {
   const void* wscale;      // [N][K/32] f32, or bf16 when scale_bf16
   int scale_bf16;
   const float* wzero;      // [N][K/32] f32 weight zeros (WZP)
-  const float* sA;         // [Mpad] or [Mpad][K/32] (ABLK)
-  const float* Sg;         // [Mpad][K/32] (WZP)
+  const float* sA;         // [Mpad] or [K/32][Mpad] (ABLK)
+  const float* Sg;         // [K/32][Mpad] (WZP)
+  int Mpad;
   const float* bias;
   float lo, hi;
   float* y;
@@ -494,7 +497,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint8_t* sN = smem + OFF_N;
   uint8_t* scl = smem + OFF_SCL;   // [n][Gr] weight scales (f32 or bf16), swizzled rows
   uint8_t* zws = smem + OFF_ZW;    // [n][Gr] f32 weight zeros
-  uint8_t* actp = smem + OFF_ACT;  // [m][Gr] f32 activation block scales / group sums
+  // [g][m] f32 activation block scales / group sums: the 32 rows of a
+  // warp's column block for one group are 128 contiguous bytes
+  float* actp = reinterpret_cast<float*>(smem + OFF_ACT);
   uint64_t* a_full = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
   uint64_t* w_full = a_full + STAGES;
   uint64_t* empty = w_full + STAGES;
@@ -563,7 +568,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       asm volatile("griddepcontrol.wait;" ::: "memory");
       if ((ABLK || WZP) && a.tma_act) {
         mbar_arrive_expect_tx(act_full, (uint32_t)(TM * frow));
-        tma_load_2d(actp, &tm_.act, g0, m0, act_full);
+        tma_load_2d(actp, &tm_.act, m0, g0, act_full);
         act = true;
       }
       const uint8_t* src = reinterpret_cast<const uint8_t*>(a.atile) +
@@ -708,10 +713,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     // activation tables come from the quantization grid
     asm volatile("griddepcontrol.wait;" ::: "memory");
     if ((ABLK || WZP) && !a.tma_act) {
-      const float* src = ABLK ? a.sA : a.Sg;
+      const float* src = ABLK ? a.sA : a.Sg;  // [G][Mpad]
       for (int i = etid; i < Gr * TM; i += NEPI) {
-        const int mm = i / Gr, g = i - mm * Gr;
-        *reinterpret_cast<float*>(actp + tbl_off(mm, g, 4, frow)) = src[(int64_t)(m0 + mm) * G + g0 + g];
+        const int g = i / TM, mm = i - g * TM;
+        actp[i] = src[(int64_t)(g0 + g) * a.Mpad + m0 + mm];
       }
     }
     bool ok = true;
@@ -749,11 +754,12 @@ __global__ void __launch_bounds__(THREADS, 1)
                 : *reinterpret_cast<const float*>(scl + tbl_off(nl, g, 4, srow));
         const f32x2 s2 = pack2(sw, sw);
         if (ABLK) {
+          const float4* av = reinterpret_cast<const float4*>(actp + g * TM + 32 * cb);
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const float a0 = *reinterpret_cast<const float*>(actp + tbl_off(32 * cb + 2 * j, g, 4, frow));
-            const float a1 = *reinterpret_cast<const float*>(actp + tbl_off(32 * cb + 2 * j + 1, g, 4, frow));
-            ffma2(acc[j], pack2u(p[2 * j], p[2 * j + 1]), fmul2(s2, pack2(a0, a1)));
+          for (int j = 0; j < 16; j += 2) {
+            const float4 a4 = av[j >> 1];  // same address in every lane: a broadcast
+            ffma2(acc[j], pack2u(p[2 * j], p[2 * j + 1]), fmul2(s2, pack2(a4.x, a4.y)));
+            ffma2(acc[j + 1], pack2u(p[2 * j + 2], p[2 * j + 3]), fmul2(s2, pack2(a4.z, a4.w)));
           }
         } else {
 #pragma unroll
@@ -762,11 +768,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (WZP) {
           const float zw = *reinterpret_cast<const float*>(zws + tbl_off(nl, g, 4, frow));
           const f32x2 z2 = pack2(zw, zw);
+          const float4* sv = reinterpret_cast<const float4*>(actp + g * TM + 32 * cb);
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const float s0 = *reinterpret_cast<const float*>(actp + tbl_off(32 * cb + 2 * j, g, 4, frow));
-            const float s1 = *reinterpret_cast<const float*>(actp + tbl_off(32 * cb + 2 * j + 1, g, 4, frow));
-            ffma2(acc[j], pack2(s0, s1), z2);
+          for (int j = 0; j < 16; j += 2) {
+            const float4 s4 = sv[j >> 1];
+            ffma2(acc[j], pack2(s4.x, s4.y), z2);
+            ffma2(acc[j + 1], pack2(s4.z, s4.w), z2);
           }
         }
       }
@@ -995,6 +1002,7 @@ int launch_a8w4_tc_call(const A8W4TcCall& c, void* ws, size_t ws_bytes, cudaStre
   ga.wzero = c.wzero;
   ga.sA = qa.sA;
   ga.Sg = qa.Sg;
+  ga.Mpad = (int)p.Mpad;
   ga.bias = c.bias; ga.lo = c.lo; ga.hi = c.hi; ga.y = c.y; ga.ldy = c.ldy;
   // The per-group tables by tensor copy when a CTA's row of them is 32, 64
   // or 128 bytes and the global rows are 16-byte multiples (else thread loads).
@@ -1022,11 +1030,14 @@ int launch_a8w4_tc_call(const A8W4TcCall& c, void* ws, size_t ws_bytes, cudaStre
       if (rc != QG_OK) return rc;
     }
   }
+  // activation tables [G][Mpad] (transposed by the quantization grid): a
+  // box of TM rows of Gr groups, unswizzled
   const float* act_src = c.mode == kBlockAsym ? qa.sA : qa.Sg;
-  ga.tma_act = act_src && tma_ok(Gr * 4, (int64_t)G * 4, act_src);
+  ga.tma_act = act_src && ((uintptr_t)act_src & 15) == 0 && p.Mpad % 4 == 0;
   if (ga.tma_act) {
-    rc = make_tmap_generic(&maps.act, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, act_src, (uint64_t)G,
-                           (uint64_t)p.Mpad, (uint64_t)G * 4, (uint32_t)Gr, TM, swz_for(Gr * 4));
+    rc = make_tmap_generic(&maps.act, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, act_src, (uint64_t)p.Mpad,
+                           (uint64_t)G, (uint64_t)p.Mpad * 4, TM, (uint32_t)Gr,
+                           CU_TENSOR_MAP_SWIZZLE_NONE);
     if (rc != QG_OK) return rc;
   }
   ga.stall = take_stall(kStallA8W4TC) ? 1 : 0;
