@@ -122,13 +122,14 @@ __device__ __forceinline__ bool epi_bar_and(bool v) {
 
 // y = clamp(zo + rne(acc*M0 / 2^(31+sh)), lo, hi).  With p = acc*M0 and
 // s = 31+sh: rne(p/2^s) = (p + 2^(s-1) - 1 + ((p >> s) & 1)) >> s.
+// |acc| <= 2^31 - 1 (the overflow bound) and M0 < 2^31 give |p| < 2^62, so
+// the rounded quotient fits int32 and the clamp runs in 32 bits:
+// clamp(q + zo, lo, hi) = clamp(q, lo - zo, hi - zo) + zo.
 __device__ __forceinline__ int requant1(int acc, int m0, int sh, int zo, int lo, int hi) {
   const int s = 31 + sh;
   const long long p = (long long)acc * (long long)m0;
-  const long long q = (p + ((1LL << (s - 1)) - 1) + ((p >> s) & 1)) >> s;
-  long long v = q + zo;
-  v = v < lo ? lo : (v > hi ? hi : v);
-  return (int)v;
+  const int q = (int)((p + ((1LL << (s - 1)) - 1) + ((p >> s) & 1)) >> s);
+  return min(max(q, lo - zo), hi - zo) + zo;
 }
 
 struct EpiArgs {
