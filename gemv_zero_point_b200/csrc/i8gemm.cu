@@ -294,7 +294,8 @@ __global__ void __launch_bounds__(CONV ? THREADS_CONV : THREADS, 1)
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;                 // MMA completion after a failed wait
   uint32_t* tmem_slot = (uint32_t*)(drain + 1);
-  int32_t* c_term = (int32_t*)(tmem_slot + 4);  // [BN] per-column constant
+  // [BN] per-column constants, 16-byte aligned (read four at a time)
+  int32_t* c_term = (int32_t*)(((uintptr_t)(tmem_slot + 4) + 15) & ~(uintptr_t)15);
   int32_t* c_m0 = c_term + BN;                   // [BN]
   int32_t* c_sh = c_m0 + BN;                     // [BN]
 
@@ -481,12 +482,20 @@ __global__ void __launch_bounds__(CONV ? THREADS_CONV : THREADS, 1)
           int accv[32];
           uint32_t packed[8] = {0, 0, 0, 0, 0, 0, 0, 0};
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int c = ch * 32 + j;
-            const int a = (int)((uint32_t)r[j] + (uint32_t)c_term[c] + (uint32_t)r_term);
-            accv[j] = a;
-            const int yv = requant1(a, c_m0[c], c_sh[c], ep.zo, ep.lo, ep.hi);
-            packed[j >> 2] |= ((uint32_t)yv & 0xFFu) << (8 * (j & 3));
+          for (int jj = 0; jj < 8; ++jj) {  // four columns' constants per load
+            const int4 t4 = reinterpret_cast<const int4*>(c_term + ch * 32)[jj];
+            const int4 m4 = reinterpret_cast<const int4*>(c_m0 + ch * 32)[jj];
+            const int4 s4 = reinterpret_cast<const int4*>(c_sh + ch * 32)[jj];
+            const int tt[4] = {t4.x, t4.y, t4.z, t4.w}, mv[4] = {m4.x, m4.y, m4.z, m4.w},
+                      sv[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int j = 4 * jj + e;
+              const int a = (int)((uint32_t)r[j] + (uint32_t)tt[e] + (uint32_t)r_term);
+              accv[j] = a;
+              const int yv = requant1(a, mv[e], sv[e], ep.zo, ep.lo, ep.hi);
+              packed[j >> 2] |= ((uint32_t)yv & 0xFFu) << (8 * (j & 3));
+            }
           }
           int8_t* cp = ep.C + (int64_t)m * ep.ldc + nb;
           if (full_chunk && (((uintptr_t)cp & 15) == 0)) {
@@ -615,7 +624,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint64_t* tfull = empty + P_STAGES;
   uint64_t* tempty = tfull + 2;
   uint32_t* tmem_slot = (uint32_t*)(tempty + 2);
-  int32_t* c_term = (int32_t*)(tmem_slot + 4);
+  int32_t* c_term = (int32_t*)(((uintptr_t)(tmem_slot + 4) + 15) & ~(uintptr_t)15);
   int32_t* c_m0 = c_term + 256;
   int32_t* c_sh = c_m0 + 256;
 
@@ -763,12 +772,20 @@ __global__ void __launch_bounds__(THREADS, 1)
           int accv[32];
           uint32_t packed[8] = {0, 0, 0, 0, 0, 0, 0, 0};
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int c = ch * 32 + j;
-            const int a = (int)((uint32_t)r[j] + (uint32_t)c_term[c] + (uint32_t)r_term);
-            accv[j] = a;
-            const int yv = requant1(a, c_m0[c], c_sh[c], ep.zo, ep.lo, ep.hi);
-            packed[j >> 2] |= ((uint32_t)yv & 0xFFu) << (8 * (j & 3));
+          for (int jj = 0; jj < 8; ++jj) {  // four columns' constants per load
+            const int4 t4 = reinterpret_cast<const int4*>(c_term + ch * 32)[jj];
+            const int4 m4 = reinterpret_cast<const int4*>(c_m0 + ch * 32)[jj];
+            const int4 s4 = reinterpret_cast<const int4*>(c_sh + ch * 32)[jj];
+            const int tt[4] = {t4.x, t4.y, t4.z, t4.w}, mv[4] = {m4.x, m4.y, m4.z, m4.w},
+                      sv[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int j = 4 * jj + e;
+              const int a = (int)((uint32_t)r[j] + (uint32_t)tt[e] + (uint32_t)r_term);
+              accv[j] = a;
+              const int yv = requant1(a, mv[e], sv[e], ep.zo, ep.lo, ep.hi);
+              packed[j >> 2] |= ((uint32_t)yv & 0xFFu) << (8 * (j & 3));
+            }
           }
           int8_t* cp = ep.C + (int64_t)m * ep.ldc + nb;
           if (full_chunk && (((uintptr_t)cp & 15) == 0)) {
