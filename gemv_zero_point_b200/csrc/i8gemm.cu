@@ -40,7 +40,7 @@ constexpr int TMEM_COLS = 2 * BN; // double-buffered accumulator
 constexpr int THREADS = 192;      // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
 constexpr int CONV_PW = 4;        // implicit-im2col gather warps: one A row per thread
 constexpr int THREADS_CONV = (CONV_PW + 5) * 32;  // + MMA warp + 4 epilogue warps
-constexpr size_t SMEM_BYTES = 1024 /*align slack*/ + STAGES * (A_STAGE + B_STAGE) + 4096;
+constexpr size_t SMEM_BYTES = 1024 /*align slack*/ + STAGES * (A_STAGE + B_STAGE) + 6144;
 
 // Instruction descriptor for kind::i8: D s32, A s8, B s8, both K-major,
 // N = BN, M = BM.
@@ -124,12 +124,14 @@ __device__ __forceinline__ bool epi_bar_and(bool v) {
 // s = 31+sh: rne(p/2^s) = (p + 2^(s-1) - 1 + ((p >> s) & 1)) >> s.
 // |acc| <= 2^31 - 1 (the overflow bound) and M0 < 2^31 give |p| < 2^62, so
 // the rounded quotient fits int32 and the clamp runs in 32 bits:
-// clamp(q + zo, lo, hi) = clamp(q, lo - zo, hi - zo) + zo.
-__device__ __forceinline__ int requant1(int acc, int m0, int sh, int zo, int lo, int hi) {
-  const int s = 31 + sh;
+// clamp(q + zo, lo, hi) = clamp(q, lo - zo, hi - zo) + zo.  The epilogue
+// passes s = 31 + shift and rnd = 2^(s-1) - 1 precomputed per column, and
+// the clamp bounds lo - zo, hi - zo.
+__device__ __forceinline__ int requant_s(int acc, int m0, int s, long long rnd, int zo, int lo_z,
+                                         int hi_z) {
   const long long p = (long long)acc * (long long)m0;
-  const int q = (int)((p + ((1LL << (s - 1)) - 1) + ((p >> s) & 1)) >> s);
-  return min(max(q, lo - zo), hi - zo) + zo;
+  const int q = (int)((p + rnd + ((p >> s) & 1)) >> s);
+  return min(max(q, lo_z), hi_z) + zo;
 }
 
 struct EpiArgs {
@@ -297,7 +299,8 @@ __global__ void __launch_bounds__(CONV ? THREADS_CONV : THREADS, 1)
   // [BN] per-column constants, 16-byte aligned (read four at a time)
   int32_t* c_term = (int32_t*)(((uintptr_t)(tmem_slot + 4) + 15) & ~(uintptr_t)15);
   int32_t* c_m0 = c_term + BN;                   // [BN]
-  int32_t* c_sh = c_m0 + BN;                     // [BN]
+  int32_t* c_sh = c_m0 + BN;                     // [BN] 31 + shift
+  long long* c_rnd = (long long*)(c_sh + BN);    // [BN] 2^(30 + shift) - 1
 
   constexpr int PW = CONV ? CONV_PW : 1;  // producer warps
   constexpr int MMA_WARP = PW, EPI_WARP0 = PW + 1;
@@ -449,6 +452,7 @@ __global__ void __launch_bounds__(CONV ? THREADS_CONV : THREADS, 1)
     const int etid = threadIdx.x - 32 * EPI_WARP0;  // 0..127
     const int row_in_tile = 32 * q + lane;
     const int64_t Kza_zb = (int64_t)ep.K * ep.za * ep.zb;
+    const int lo_z = ep.lo - ep.zo, hi_z = ep.hi - ep.zo;
     int local = 0;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++local) {
       const int tm = t % tiles_m, tn = t / tiles_m;
@@ -462,7 +466,9 @@ __global__ void __launch_bounds__(CONV ? THREADS_CONV : THREADS, 1)
                             (int64_t)ep.za * ep.colsum[n] + Kza_zb;
           c_term[c] = (int32_t)v;  // wraps mod 2^32; the final sum is in range
           c_m0[c] = ep.per_channel ? ep.m0v[n] : ep.m0;
-          c_sh[c] = ep.per_channel ? ep.shv[n] : ep.sh;
+          const int sft = 31 + (ep.per_channel ? ep.shv[n] : ep.sh);
+          c_sh[c] = sft;
+          c_rnd[c] = (1LL << (sft - 1)) - 1;
         }
       }
       epi_bar_sync();
@@ -486,14 +492,17 @@ __global__ void __launch_bounds__(CONV ? THREADS_CONV : THREADS, 1)
             const int4 t4 = reinterpret_cast<const int4*>(c_term + ch * 32)[jj];
             const int4 m4 = reinterpret_cast<const int4*>(c_m0 + ch * 32)[jj];
             const int4 s4 = reinterpret_cast<const int4*>(c_sh + ch * 32)[jj];
+            const longlong2 r01 = reinterpret_cast<const longlong2*>(c_rnd + ch * 32)[2 * jj];
+            const longlong2 r23 = reinterpret_cast<const longlong2*>(c_rnd + ch * 32)[2 * jj + 1];
             const int tt[4] = {t4.x, t4.y, t4.z, t4.w}, mv[4] = {m4.x, m4.y, m4.z, m4.w},
                       sv[4] = {s4.x, s4.y, s4.z, s4.w};
+            const long long rv[4] = {r01.x, r01.y, r23.x, r23.y};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const int j = 4 * jj + e;
               const int a = (int)((uint32_t)r[j] + (uint32_t)tt[e] + (uint32_t)r_term);
               accv[j] = a;
-              const int yv = requant1(a, mv[e], sv[e], ep.zo, ep.lo, ep.hi);
+              const int yv = requant_s(a, mv[e], sv[e], rv[e], ep.zo, lo_z, hi_z);
               packed[j >> 2] |= ((uint32_t)yv & 0xFFu) << (8 * (j & 3));
             }
           }
@@ -552,7 +561,7 @@ __global__ void __launch_bounds__(CONV ? THREADS_CONV : THREADS, 1)
 // ---------------------------------------------------------------------------
 constexpr int P_STAGES = 6;
 constexpr int P_STAGE = BM * BK;  // 16 KiB for the A half, same for the B half
-constexpr size_t P_SMEM_BYTES = 1024 + (size_t)P_STAGES * 2 * P_STAGE + 4096;
+constexpr size_t P_SMEM_BYTES = 1024 + (size_t)P_STAGES * 2 * P_STAGE + 6144;
 constexpr int P_GROUP_M = 16;     // pair-tile rows per raster group (A slice stays in L2)
 // kind::i8, D s32, A/B s8 K-major, N = 256, M = 256 (the pair)
 constexpr uint32_t IDESC2 = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(256 >> 3) << 17) |
@@ -626,7 +635,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint32_t* tmem_slot = (uint32_t*)(tempty + 2);
   int32_t* c_term = (int32_t*)(((uintptr_t)(tmem_slot + 4) + 15) & ~(uintptr_t)15);
   int32_t* c_m0 = c_term + 256;
-  int32_t* c_sh = c_m0 + 256;
+  int32_t* c_sh = c_m0 + 256;                    // 31 + shift
+  long long* c_rnd = (long long*)(c_sh + 256);   // 2^(30 + shift) - 1
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_rank_u32();
@@ -735,6 +745,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int etid = threadIdx.x - 64;
     const int row_in_tile = 32 * q + lane;
     const int64_t Kza_zb = (int64_t)ep.K * ep.za * ep.zb;
+    const int lo_z = ep.lo - ep.zo, hi_z = ep.hi - ep.zo;
     const uint32_t tempty_leader0 = mapa_u32(smem_u32(&tempty[0]), 0);
     const uint32_t tempty_leader1 = mapa_u32(smem_u32(&tempty[1]), 0);
     int local = 0;
@@ -751,7 +762,9 @@ __global__ void __launch_bounds__(THREADS, 1)
                             (int64_t)ep.za * ep.colsum[n] + Kza_zb;
           c_term[c] = (int32_t)v;
           c_m0[c] = ep.per_channel ? ep.m0v[n] : ep.m0;
-          c_sh[c] = ep.per_channel ? ep.shv[n] : ep.sh;
+          const int sft = 31 + (ep.per_channel ? ep.shv[n] : ep.sh);
+          c_sh[c] = sft;
+          c_rnd[c] = (1LL << (sft - 1)) - 1;
         }
       }
       epi_bar_sync();
@@ -776,14 +789,17 @@ __global__ void __launch_bounds__(THREADS, 1)
             const int4 t4 = reinterpret_cast<const int4*>(c_term + ch * 32)[jj];
             const int4 m4 = reinterpret_cast<const int4*>(c_m0 + ch * 32)[jj];
             const int4 s4 = reinterpret_cast<const int4*>(c_sh + ch * 32)[jj];
+            const longlong2 r01 = reinterpret_cast<const longlong2*>(c_rnd + ch * 32)[2 * jj];
+            const longlong2 r23 = reinterpret_cast<const longlong2*>(c_rnd + ch * 32)[2 * jj + 1];
             const int tt[4] = {t4.x, t4.y, t4.z, t4.w}, mv[4] = {m4.x, m4.y, m4.z, m4.w},
                       sv[4] = {s4.x, s4.y, s4.z, s4.w};
+            const long long rv[4] = {r01.x, r01.y, r23.x, r23.y};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const int j = 4 * jj + e;
               const int a = (int)((uint32_t)r[j] + (uint32_t)tt[e] + (uint32_t)r_term);
               accv[j] = a;
-              const int yv = requant1(a, mv[e], sv[e], ep.zo, ep.lo, ep.hi);
+              const int yv = requant_s(a, mv[e], sv[e], rv[e], ep.zo, lo_z, hi_z);
               packed[j >> 2] |= ((uint32_t)yv & 0xFFu) << (8 * (j & 3));
             }
           }
