@@ -151,6 +151,32 @@ def test_a8w4_gemm_shapes(lib, M, N, K):
     _check_a8w4(lib, w, ldy_pad=1)
 
 
+# Degenerate activation rows through every A8W4 path (the GEMV for M = 1,
+# the quantization tiles + tensor-core kernel for M > 1 with K % 64 == 0,
+# the CUDA-core kernel otherwise): an all-zero row (scale 1, zero-point
+# -128), constant positive and negative rows (the range includes 0), a
+# single spike among zeros, values near the f32 subnormal range, and a row
+# whose extremes are the clamp bounds of the codes.
+def _degenerate_rows(M, K, seed):
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((M, K), dtype=np.float32)
+    specials = [np.zeros(K, np.float32), np.full(K, 3.25, np.float32),
+                np.full(K, -0.75, np.float32), np.zeros(K, np.float32),
+                rng.standard_normal(K).astype(np.float32) * np.float32(1e-30),
+                np.linspace(-1e4, 1e4, K).astype(np.float32)]
+    specials[3][K // 3] = 1e3
+    for i, row in enumerate(specials[:M]):
+        x[i] = row
+    return x
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 300, 1024), (6, 200, 1024), (6, 200, 96), (130, 64, 512)])
+def test_a8w4_degenerate_rows(lib, M, N, K):
+    w = workloads.a8w4(M, N, K, seed=900 + M + K, clamp=(-np.inf, np.inf))
+    w["x"] = _degenerate_rows(M, K, 901 + M)
+    _check_a8w4(lib, w)
+
+
 def test_a8w4_gemm_full_size_128x4096x4096(lib):
     _check_a8w4(lib, workloads.a8w4_gemm_128x4096x4096())
 
