@@ -47,9 +47,11 @@
 //               per warp), release of the buffer, acc += scale * I with
 //               packed f32x2 FMAs; then the partial tile, the cluster
 //               reduction and y
-// The single-thread roles poll their barriers (mbarrier.test_wait): a
-// suspending try_wait costs some hundred cycles even on a completed phase,
-// several times the issue cost of an MMA.
+// One thread per warp waits on each barrier.  The waits off the critical
+// path (stage slots and operands that are normally ready in time) park in
+// mbarrier.try_wait with a suspend-time hint, so they take no issue slots
+// from the converter and read-out warps; the two waits of the TMEM round
+// trip (free accumulator buffer, accumulators ready) poll.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -204,9 +206,37 @@ __device__ __forceinline__ void bar_sync() {
   asm volatile("bar.sync %0, %1;" ::"n"(ID), "n"(N) : "memory");
 }
 
-// Poll a barrier phase from one thread, sleeping briefly between polls so
-// the spinning warp does not take the issue slots of the warps doing the
-// arithmetic on its sub-partition; bounded like mbar_poll.
+// Wait for phase `parity` of `bar` with mbarrier.try_wait and a suspend-time
+// hint: the hardware parks the thread until the phase completes (or the
+// 20 us hint runs out, after which it asks again), so a waiting warp issues
+// a few instructions per wake-up instead of a polling loop that takes issue
+// slots from the converter and read-out warps on its sub-partition
+// (test-and-sleep polls were about half of all instructions this kernel
+// issued).  At most limit / 256 + 1 tries: about 82 ms at kSpinLimit,
+// 0.3 ms at kStallSpinLimit.
+__device__ __forceinline__ bool mbar_park(uint64_t* bar, uint32_t parity, int* status,
+                                          uint32_t limit = kSpinLimit) {
+  const uint32_t tries = (limit >> 8) + 1;
+  for (uint32_t i = 0; i < tries; ++i) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(20000u)
+        : "memory");
+    if (ok) return true;
+  }
+  record_error(status, QG_ERR_TIMEOUT);
+  return false;
+}
+
+// Poll a barrier phase from one thread, sleeping briefly between polls;
+// bounded like mbar_poll.  Kept for the two waits on the TMEM round trip
+// (the MMA issuer waiting for a free accumulator buffer, an epilogue warp
+// waiting for its accumulators), where the kernel measured slower with
+// parked waits (mbar_park) than with these polls.
 __device__ __forceinline__ bool poll_yield(uint64_t* bar, uint32_t parity, int* status,
                                            uint32_t limit) {
   for (uint32_t i = 0; i < (limit << 4); ++i) {
@@ -571,7 +601,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                            ((int64_t)tm * a.nkb + (k0 / KS)) * STAGE_BYTES;
       for (int s = 0; s < nst; ++s) {
         const int slot = s % STAGES;
-        if (s >= STAGES && !poll_yield(&empty[slot], ((s / STAGES) - 1) & 1, status, a.spin)) break;
+        if (s >= STAGES && !mbar_park(&empty[slot], ((s / STAGES) - 1) & 1, status, a.spin)) break;
         if (a.stall && s == 1) continue;
         mbar_arrive_expect_tx(&a_full[slot], STAGE_BYTES);
         bulk_g2s(sA + slot * STAGE_BYTES, src + (int64_t)s * STAGE_BYTES, STAGE_BYTES,
@@ -594,8 +624,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int s = 0; s < nst; ++s) {
         const int slot = s % STAGES, sb = s % NSB;
         const uint32_t par = (uint32_t)(s / STAGES) & 1;
-        if (!poll_yield(&a_full[slot], par, status, a.spin) ||
-            !poll_yield(&w_full[slot], par, status, a.spin) ||
+        if (!mbar_park(&a_full[slot], par, status, a.spin) ||
+            !mbar_park(&w_full[slot], par, status, a.spin) ||
             !poll_yield(&tempty[sb], ((uint32_t)(s / NSB) & 1) ^ 1, status, a.spin)) {
           failed = true;
           break;
@@ -639,11 +669,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     const uint32_t dst_row = smem_u32(sW) + (uint32_t)(r * 128);
     for (int s = 0; s < nst; ++s) {
       const int slot = s % STAGES, ns = s % NRING;
-      // thread 0 polls both barriers; a hardware barrier releases the rest
+      // thread 0 waits on both barriers; a hardware barrier releases the rest
       bool w = true;
       if (ctid == 0) {
-        if (s >= STAGES) w = poll_yield(&empty[slot], ((s / STAGES) - 1) & 1, status, a.spin);
-        w = w && poll_yield(&nib_full[ns], (s / NRING) & 1, status, a.spin);
+        if (s >= STAGES) w = mbar_park(&empty[slot], ((s / STAGES) - 1) & 1, status, a.spin);
+        w = w && mbar_park(&nib_full[ns], (s / NRING) & 1, status, a.spin);
       }
       w = bar_and<2, NCONV>(w);
       if (w) {
