@@ -306,6 +306,10 @@ __global__ void __launch_bounds__(CONV ? THREADS_CONV : THREADS, 1)
   constexpr int MMA_WARP = PW, EPI_WARP0 = PW + 1;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tiles = tiles_m * tiles_n;
+  // Launched as a programmatic dependent: the next grid in the stream may be
+  // scheduled now (on SMs this one leaves free) and set itself up; every
+  // role that touches global memory waits for the previous grid first.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -332,6 +336,7 @@ __global__ void __launch_bounds__(CONV ? THREADS_CONV : THREADS, 1)
 
   if (CONV && warp < PW) {
     // ---------------- implicit-im2col producers ----------------
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     // Thread ptid gathers row ptid of every tile.  Stage s is signalled one
     // stage late: after the copies of stage s+1 are issued, each thread
     // waits for its own copies of stage s, makes them and its zero-point
@@ -377,6 +382,7 @@ __global__ void __launch_bounds__(CONV ? THREADS_CONV : THREADS, 1)
         if ((issued >> st) & 1u) mbar_poll(&full[st], (last_ph >> st) & 1u, status);
   } else if (warp == 0) {
     // ------------------------- TMA producer -------------------------
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
@@ -448,6 +454,7 @@ __global__ void __launch_bounds__(CONV ? THREADS_CONV : THREADS, 1)
     }
   } else {
     // ------------------------- epilogue -------------------------
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int q = warp & 3;                 // TMEM lane quarter of this warp
     const int etid = threadIdx.x - 32 * EPI_WARP0;  // 0..127
     const int row_in_tile = 32 * q + lane;
@@ -638,6 +645,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   int32_t* c_sh = c_m0 + 256;                    // 31 + shift
   long long* c_rnd = (long long*)(c_sh + 256);   // 2^(30 + shift) - 1
 
+  // the next grid in the stream may be scheduled now (it waits for this one
+  // on the device before it touches memory)
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_rank_u32();
   const bool leader = rank == 0;
@@ -910,6 +920,9 @@ __global__ void __launch_bounds__(256) stage_a_kernel(int K, const int8_t* __res
   // the GEMM grid may start its prologue and its B copies now; it waits for
   // this grid before it reads the staged rows or the row sums
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // This grid is a programmatic dependent of the previous work in the
+  // stream: A is read and the workspace written only once that has finished.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   __shared__ int red[8];
   const int64_t m = blockIdx.x;
   const int8_t* src = A + m * lda;
@@ -1092,6 +1105,30 @@ static EpiArgs make_epi(int M, int N, int K, const void* packed_b, const qg_requ
   return ep;
 }
 
+// The one-CTA kernel as a programmatic dependent launch: its CTAs may become
+// resident while the previous kernel in the stream is still running and
+// wait for it on the device (griddepcontrol.wait in every role that touches
+// global memory), so barrier setup, TMEM allocation and the tensor-map
+// prefetch overlap the previous grid instead of following a launch gap.
+template <bool CONV>
+static int launch_one_cta(int grid, const CUtensorMap& tmA, const CUtensorMap& tmB, int num_kb,
+                          int tiles_m, int tiles_n, const EpiArgs& ep, const ConvGather& cg,
+                          cudaStream_t st) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(CONV ? THREADS_CONV : THREADS);
+  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, i8gemm_tc_kernel<CONV>, tmA, tmB, num_kb, tiles_m,
+                                           tiles_n, ep, cg, status_word());
+  return e == cudaSuccess ? QG_OK : QG_ERR_CUDA;
+}
+
 int i8gemm_run_packed(int M, int N, int K, const int8_t* A, int64_t lda, const void* packed_b,
                       int8_t* C, int64_t ldc, const qg_requant_t& rq, int32_t* acc_out,
                       int64_t ld_acc, void* ws, size_t ws_bytes, cudaStream_t st) {
@@ -1106,9 +1143,20 @@ int i8gemm_run_packed(int M, int N, int K, const int8_t* A, int64_t lda, const v
     int8_t* Aw = (int8_t*)ws;
     rowsum = need_rowsum ? (int32_t*)((int8_t*)ws + round_up((int64_t)M * staged_lda(K), 256))
                          : nullptr;
-    stage_a_kernel<<<M, 256, 0, st>>>(K, A, lda, need_copy ? Aw : nullptr, staged_lda(K), rowsum);
-    int rc = launch_status();
-    if (rc != QG_OK) return rc;
+    // programmatic dependent launch: scheduled while the previous kernel in
+    // the stream may still run; it waits for it on the device
+    cudaLaunchConfig_t scfg = {};
+    scfg.gridDim = dim3((unsigned)M);
+    scfg.blockDim = dim3(256);
+    scfg.stream = st;
+    cudaLaunchAttribute sattr[1];
+    sattr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    sattr[0].val.programmaticStreamSerializationAllowed = 1;
+    scfg.attrs = sattr;
+    scfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&scfg, stage_a_kernel, K, A, lda, need_copy ? Aw : (int8_t*)nullptr,
+                           (int64_t)staged_lda(K), rowsum) != cudaSuccess)
+      return QG_ERR_CUDA;
     if (need_copy) {
       Aeff = Aw;
       lda_eff = staged_lda(K);
@@ -1144,9 +1192,10 @@ int i8gemm_run_packed(int M, int N, int K, const int8_t* A, int64_t lda, const v
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
-    // after this call's staging pass: programmatic dependent launch (the
-    // staging grid started only once all earlier work had finished, so
-    // everything but its own output is complete when this grid starts)
+    // after this call's staging pass: programmatic dependent launch.  Before
+    // its grid-dependency wait the kernel reads only the packed B; the rows
+    // of A, the row sums and C wait for the staging grid, which itself waits
+    // for the work before it in the stream.
     attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
@@ -1158,9 +1207,7 @@ int i8gemm_run_packed(int M, int N, int K, const int8_t* A, int64_t lda, const v
   const int tiles_m = (int)cdiv(M, BM), tiles_n = (int)cdiv(N, BN);
   const int tiles = tiles_m * tiles_n;
   const int grid = tiles < num_sms() ? tiles : num_sms();
-  i8gemm_tc_kernel<false><<<grid, THREADS, SMEM_BYTES, st>>>(tmA, tmB, num_kb, tiles_m, tiles_n,
-                                                             ep, ConvGather{}, status_word());
-  return launch_status();
+  return launch_one_cta<false>(grid, tmA, tmB, num_kb, tiles_m, tiles_n, ep, ConvGather{}, st);
 }
 
 // ---------------------------------------------------------------------------
@@ -1211,9 +1258,7 @@ int conv_run_packed(int Nb, int H, int W, int Cin, int Cout, int KH, int KW, int
   const int tiles_m = (int)cdiv(M, BM), tiles_n = (int)cdiv(Cout, BN);
   const int tiles = tiles_m * tiles_n;
   const int grid = tiles < num_sms() ? tiles : num_sms();
-  i8gemm_tc_kernel<true><<<grid, THREADS_CONV, SMEM_BYTES, st>>>(tmB, tmB, num_kb, tiles_m, tiles_n,
-                                                            ep, cg, status_word());
-  return launch_status();
+  return launch_one_cta<true>(grid, tmB, tmB, num_kb, tiles_m, tiles_n, ep, cg, st);
 }
 
 int conv_run(int Nb, int H, int W, int Cin, int Cout, int KH, int KW, int sh, int sw, int ph,

@@ -22,7 +22,13 @@
  *     must not alias.
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
  *     default stream).  The return value reports argument checks and launch
- *     errors.  Errors found on the device (a bounded wait that ran out, an
+ *     errors.  Kernels are launched as programmatic dependents of the work
+ *     before them on the stream: they may start while it is still running
+ *     and wait for it on the device before they read activations or
+ *     workspace or write any output.  Before that wait they may read the
+ *     call's packed weights, scales and bias, so a kernel that signals its
+ *     dependents early (griddepcontrol.launch_dependents) must not write
+ *     those buffers for the call that follows it.  Errors found on the device (a bounded wait that ran out, an
  *     int4 weight out of range) are recorded in a per-device status word that
  *     qg_device_status() reads after the work has finished.
  *   - Every entry point returns QG_OK (0) or a negative qg_status.  It never
