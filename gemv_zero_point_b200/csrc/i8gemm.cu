@@ -625,7 +625,9 @@ __device__ __forceinline__ void pair_tile_coords(int t, int tiles_m, int tiles_n
   const int g = t / per_group, r = t % per_group;
   const int rows = min(P_GROUP_M, tiles_m - g * P_GROUP_M);
   tm = g * P_GROUP_M + r % rows;
-  tn = r / rows;
+  // serpentine: odd groups sweep the B panels from the last one back, so a
+  // group starts on the panels the previous one read last (still in L2)
+  tn = (g & 1) ? tiles_n - 1 - r / rows : r / rows;
 }
 
 __global__ void __launch_bounds__(THREADS, 1)
