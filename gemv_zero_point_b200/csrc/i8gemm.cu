@@ -43,9 +43,11 @@ constexpr int THREADS_CONV = (CONV_PW + 5) * 32;  // + MMA warp + 4 epilogue war
 constexpr size_t SMEM_BYTES = 1024 /*align slack*/ + STAGES * (A_STAGE + B_STAGE) + 6144;
 
 // Instruction descriptor for kind::i8: D s32, A s8, B s8, both K-major,
-// N = BN, M = BM.
-constexpr uint32_t IDESC = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
-                           ((uint32_t)(BM >> 4) << 24);
+// M = BM, N = n (a multiple of 16, 16..256).
+__host__ __device__ constexpr uint32_t idesc_i8(int n) {
+  return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) |
+         ((uint32_t)(BM >> 4) << 24);
+}
 
 // Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
 // 1024 bytes apart (sm_100 descriptor version 1).
@@ -78,11 +80,11 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 __device__ __forceinline__ void mma_i8(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
-                                       uint32_t accumulate) {
+                                       uint32_t idesc, uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
-      "l"(adesc), "l"(bdesc), "r"(IDESC), "r"(accumulate)
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
@@ -149,6 +151,8 @@ struct EpiArgs {
   int64_t ld_acc;
   int stall;        // test hook (one-CTA kernel): skip the loads of K block 1 of the first tile
   uint32_t spin;    // poll limit of the pipeline waits
+  int nmma;         // one-CTA kernel: MMA N and B-tile rows (BN, or N rounded up to 16
+                    // when one column tile covers N)
 };
 
 // ---------------------------------------------------------------------------
@@ -306,6 +310,7 @@ __global__ void __launch_bounds__(CONV ? THREADS_CONV : THREADS, 1)
   constexpr int MMA_WARP = PW, EPI_WARP0 = PW + 1;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tiles = tiles_m * tiles_n;
+  const uint32_t b_bytes = (uint32_t)ep.nmma * BK;  // B tile rows actually copied
   // Launched as a programmatic dependent: the next grid in the stream may be
   // scheduled now (on SMs this one leaves free) and set itself up; every
   // role that touches global memory waits for the previous grid first.
@@ -354,7 +359,7 @@ __global__ void __launch_bounds__(CONV ? THREADS_CONV : THREADS, 1)
         if (lane == 0) got = mbar_poll(&empty[stage], phase ^ 1, status, ep.spin);
         if (!__shfl_sync(0xffffffffu, (int)got, 0)) goto conv_done;
         if (ptid == 0) {
-          mbar_expect_tx(&full[stage], B_STAGE);
+          mbar_expect_tx(&full[stage], b_bytes);
           tma_load_2d(sB + stage * B_STAGE, &tmB, kb * BK, tn * BN, &full[stage]);
           issued |= 1u << stage;
           last_ph = (last_ph & ~(1u << stage)) | (phase << stage);
@@ -392,7 +397,7 @@ __global__ void __launch_bounds__(CONV ? THREADS_CONV : THREADS, 1)
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_poll(&empty[stage], phase ^ 1, status, ep.spin)) goto producer_done;
           if (!(ep.stall && t == (int)blockIdx.x && kb == 1)) {
-            mbar_arrive_expect_tx(&full[stage], A_STAGE + B_STAGE);
+            mbar_arrive_expect_tx(&full[stage], A_STAGE + b_bytes);
             tma_load_2d(sA + stage * A_STAGE, &tmA, kb * BK, tm * BM, &full[stage]);
             tma_load_2d(sB + stage * B_STAGE, &tmB, kb * BK, tn * BN, &full[stage]);
             issued |= 1u << stage;
@@ -436,7 +441,8 @@ __global__ void __launch_bounds__(CONV ? THREADS_CONV : THREADS, 1)
           const uint32_t b0 = smem_u32(sB + stage * B_STAGE);
 #pragma unroll
           for (int k = 0; k < BK / 32; ++k) {
-            mma_i8(d, sdesc_sw128(a0 + 32 * k), sdesc_sw128(b0 + 32 * k), (kb | k) != 0);
+            mma_i8(d, sdesc_sw128(a0 + 32 * k), sdesc_sw128(b0 + 32 * k), idesc_i8(ep.nmma),
+                   (kb | k) != 0);
           }
           mma_commit(&empty[stage]);  // frees the stage when these MMAs finish
           if (++stage == STAGES) {
@@ -1104,6 +1110,9 @@ static EpiArgs make_epi(int M, int N, int K, const void* packed_b, const qg_requ
   ep.C = C; ep.ldc = ldc; ep.acc_out = acc_out; ep.ld_acc = ld_acc;
   ep.stall = 0;
   ep.spin = kSpinLimit;
+  // One column tile: the MMA covers only the columns that exist, rounded up
+  // to the instruction's step of 16 (the packed rows beyond N are zero).
+  ep.nmma = N <= BN ? (int)round_up(N, 16) : BN;
   return ep;
 }
 
@@ -1164,15 +1173,16 @@ int i8gemm_run_packed(int M, int N, int K, const int8_t* A, int64_t lda, const v
       lda_eff = staged_lda(K);
     }
   }
-  // A pair of CTAs (M > 128) stages half of the B tile per CTA: box of BM rows.
+  // A pair of CTAs (M > 128) stages half of the B tile per CTA: box of BM
+  // rows; the one-CTA kernel copies the ep.nmma rows its MMAs read.
   const bool pair_path = M > BM;
+  EpiArgs ep = make_epi(M, N, K, packed_b, rq, rowsum, C, ldc, acc_out, ld_acc);
   CUtensorMap tmA, tmB;
   int rc = make_tmap(&tmA, Aeff, (uint64_t)K, (uint64_t)M, (uint64_t)lda_eff, BM);
   if (rc != QG_OK) return rc;
   rc = make_tmap(&tmB, packed_b, (uint64_t)d.Kp, (uint64_t)d.Np, (uint64_t)d.Kp,
-                 pair_path ? BM : BN);
+                 pair_path ? BM : ep.nmma);
   if (rc != QG_OK) return rc;
-  EpiArgs ep = make_epi(M, N, K, packed_b, rq, rowsum, C, ldc, acc_out, ld_acc);
   const int num_kb = (int)(d.Kp / BK);
   ep.stall = (M <= BM && num_kb > 1 && take_stall(kStallInt8Gemm)) ? 1 : 0;
   ep.spin = ep.stall ? kStallSpinLimit : kSpinLimit;
@@ -1245,10 +1255,10 @@ int conv_run_packed(int Nb, int H, int W, int Cin, int Cout, int KH, int KW, int
   const int64_t M = (int64_t)Nb * OH * OW;
   if (M > INT32_MAX) return QG_ERR_UNSUPPORTED;
   const PackDims d = pack_dims(K, Cout);
-  CUtensorMap tmB;
-  int rc = make_tmap(&tmB, packed_w, (uint64_t)d.Kp, (uint64_t)d.Np, (uint64_t)d.Kp, BN);
-  if (rc != QG_OK) return rc;
   EpiArgs ep = make_epi((int)M, Cout, K, packed_w, rq, nullptr, y, Cout, acc_out, Cout);
+  CUtensorMap tmB;
+  int rc = make_tmap(&tmB, packed_w, (uint64_t)d.Kp, (uint64_t)d.Np, (uint64_t)d.Kp, ep.nmma);
+  if (rc != QG_OK) return rc;
   ConvGather cg;
   cg.x = x;
   cg.H = H; cg.W = W; cg.Cin = Cin; cg.KH = KH; cg.KW = KW;
