@@ -1173,9 +1173,13 @@ int i8gemm_run_packed(int M, int N, int K, const int8_t* A, int64_t lda, const v
       lda_eff = staged_lda(K);
     }
   }
-  // A pair of CTAs (M > 128) stages half of the B tile per CTA: box of BM
-  // rows; the one-CTA kernel copies the ep.nmma rows its MMAs read.
-  const bool pair_path = M > BM;
+  // CTA pairs (256 x 256 tiles, each CTA staging half of the B tile: box of
+  // BM rows) for M > 256, or when 128 x 256 tiles of one CTA would take more
+  // than one wave; otherwise the one-CTA kernel (fewer, lighter launches on a
+  // small problem: 130x70x129 12.7 -> 12.0 us), which copies the ep.nmma rows
+  // its MMAs read.
+  const bool pair_path =
+      M > BM && (M > 2 * BM || cdiv(M, BM) * cdiv(N, BN) > (int64_t)num_sms());
   EpiArgs ep = make_epi(M, N, K, packed_b, rq, rowsum, C, ldc, acc_out, ld_acc);
   CUtensorMap tmA, tmB;
   int rc = make_tmap(&tmA, Aeff, (uint64_t)K, (uint64_t)M, (uint64_t)lda_eff, BM);
@@ -1184,7 +1188,7 @@ int i8gemm_run_packed(int M, int N, int K, const int8_t* A, int64_t lda, const v
                  pair_path ? BM : ep.nmma);
   if (rc != QG_OK) return rc;
   const int num_kb = (int)(d.Kp / BK);
-  ep.stall = (M <= BM && num_kb > 1 && take_stall(kStallInt8Gemm)) ? 1 : 0;
+  ep.stall = (!pair_path && num_kb > 1 && take_stall(kStallInt8Gemm)) ? 1 : 0;
   ep.spin = ep.stall ? kStallSpinLimit : kSpinLimit;
   if (pair_path) {
     // 2-CTA pairs on 256 x 256 tiles, one resident pair per SM pair

@@ -84,7 +84,8 @@ int qg_device_status(int reset);
  * limit.  The call itself still returns QG_OK; qg_device_status() then
  * reports QG_ERR_TIMEOUT, the call's outputs are unspecified, and the next
  * call runs normally.
- *   which: 1 = INT8 GEMM one-CTA kernel (a call with M <= 128 and K > 128),
+ *   which: 1 = INT8 GEMM one-CTA kernel (a call with K > 128 and M <= 128, or
+ *              M <= 256 when its 128 x 256 tiles fit in one wave of SMs),
  *          2 = A8W4 tensor-core kernel (an M > 1 call that takes it),
  *          0 = disarm.
  * Returns QG_OK, or QG_ERR_INVALID_ARG for another value.  Not for

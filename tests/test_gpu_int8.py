@@ -99,7 +99,8 @@ def test_gemm_shapes(lib, M, N, K, per_channel, zb):
     check_gemm(lib, w)
 
 
-# M > 128 runs on CTA pairs.  Rows the tensor-copy engine cannot address
+# M > 256 runs on CTA pairs (as does M > 128 when one-CTA tiles would take
+# more than one wave).  Rows the tensor-copy engine cannot address
 # (pitch or base not a multiple of 16 bytes) are first copied to a 16-byte
 # pitch.  Cases: pitches 8, 4 and 1 (mod 16), a base offset into the
 # allocation, b_zero_point != 0 (row sums), ragged M / N / K, and more tiles
@@ -155,11 +156,12 @@ def test_gemm_extreme_bound(lib):
     assert (acc == -K * 65025).all()
 
 
-@pytest.mark.parametrize("M", [64, 200])
+@pytest.mark.parametrize("M", [64, 200, 300])
 def test_gemm_k_at_the_overflow_bound(lib, M):
     # K = 33025 is the largest K with K*65025 <= 2^31 - 1 (no bias): every term
     # at the worst magnitude gives an accumulator of -2,147,450,625, inside
-    # int32 by 33,022.  M = 64 runs the one-CTA kernel, M = 200 the CTA pairs.
+    # int32 by 33,022.  M = 64 and 200 run the one-CTA kernel (one and two row
+    # tiles), M = 300 the CTA pairs.
     K = 33025
     w = workloads.int8_gemm(M, 64, K, seed=3, za=-128, zb=127, with_bias=False)
     w["A"][:] = 127
