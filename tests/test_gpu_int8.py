@@ -86,8 +86,11 @@ def test_gemm_130x70x129_packed_bit_exact(lib):
     check_gemm(lib, workloads.int8_gemm_130x70x129(), packed=True, ldc_pad=3)
 
 
+# Kernel choice: M <= 128 -> one CTA per 128 x 256 tile; M <= 256 -> the same
+# while its tiles fit in one wave (129x257: 4 tiles; 256x16: 2), else CTA
+# pairs (200x19000: 2 x 75 = 150 one-CTA tiles, more than the 148 SMs).
 SHAPES = [(1, 1, 1), (2, 16, 31), (127, 70, 129), (128, 256, 128), (129, 257, 256),
-          (300, 600, 300), (64, 40, 1000), (257, 513, 130)]
+          (256, 16, 200), (200, 19000, 64), (300, 600, 300), (64, 40, 1000), (257, 513, 130)]
 
 
 @pytest.mark.parametrize("M,N,K", SHAPES)
