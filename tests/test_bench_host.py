@@ -23,3 +23,15 @@ def test_every_workload_names_its_kernel_source(workload):
     src = bench.KERNEL_SOURCES[workload]
     assert os.path.exists(os.path.join(ROOT, "gemv_zero_point_b200", "csrc", src))
     assert len(bench.source_digest(workload)) == 16
+
+
+def test_power_capped_needs_a_lowered_clock():
+    # the limiter's flag with the clock at its maximum keeps the burst peak
+    assert not bench.power_capped({"sm_mhz": 1965.0, "sm_max_mhz": 1965.0,
+                                   "reasons": ["sw_power_cap"]})
+    assert bench.power_capped({"sm_mhz": 1320.0, "sm_max_mhz": 1965.0,
+                               "reasons": ["sw_power_cap"]})
+    assert not bench.power_capped({"sm_mhz": 1320.0, "sm_max_mhz": 1965.0, "reasons": []})
+    assert not bench.power_capped(None)
+    # no clock figures recorded: trust the flag
+    assert bench.power_capped({"reasons": ["sw_power_cap"]})
