@@ -225,7 +225,12 @@ class GemmCase:
         # a staging pass runs before the GEMM for row sums (zb != 0) or when A's
         # rows are not 16-byte addressable (copied to a 16-byte pitch)
         self.launches = 1 + (1 if (w["lda"] % 16 or w["zb"]) else 0)
-        self.kernel = "i8gemm_tc2_kernel" if self.M > 128 else "i8gemm_tc_kernel"
+        # the library's choice: CTA pairs for M > 256, or for M > 128 when
+        # 128 x 256 one-CTA tiles would take more than one wave of SMs
+        sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+        one_cta_tiles = -(-self.M // 128) * -(-self.N // 256)
+        pairs = self.M > 128 and (self.M > 256 or one_cta_tiles > sms)
+        self.kernel = "i8gemm_tc2_kernel" if pairs else "i8gemm_tc_kernel"
         self.h2d_host = torch.from_numpy(np.ascontiguousarray(w["A"])).pin_memory()
         self.d2h_host = torch.empty((self.M, self.N), dtype=torch.int8).pin_memory()
 
