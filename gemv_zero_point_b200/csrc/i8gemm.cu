@@ -934,20 +934,42 @@ __global__ void __launch_bounds__(256) stage_a_kernel(int K, const int8_t* __res
   __shared__ int red[8];
   const int64_t m = blockIdx.x;
   const int8_t* src = A + m * lda;
-  int8_t* dst = Aw ? Aw + m * ldw : nullptr;
+  int8_t* dst = Aw ? Aw + m * ldw : nullptr;  // 16-byte aligned rows
   int s = 0;
-  const bool vec = (((uintptr_t)src & 7) == 0);
-  const int K8 = vec ? (K & ~7) : 0;
-  for (int i = threadIdx.x * 8; i < K8; i += blockDim.x * 8) {
-    const uint2 v = *reinterpret_cast<const uint2*>(src + i);
-    if (dst) *reinterpret_cast<uint2*>(dst + i) = v;
-    s = __dp4a((int)v.x, 0x01010101, s);
-    s = __dp4a((int)v.y, 0x01010101, s);
-  }
-  for (int i = K8 + threadIdx.x; i < K; i += blockDim.x) {
-    const int8_t v = src[i];
-    if (dst) dst[i] = v;
-    s += v;
+  // Whole 16-byte chunks: output chunk j holds row bytes [16j, 16j + 16),
+  // which sit at offset a = src % 16 in the aligned source chunks j and
+  // j + 1.  A chunk is loaded only when it holds a byte of the row, so no
+  // load leaves the pages the row lies in; bytes past K in the last chunk
+  // land in the staged row's padding (never read) and are left out of the
+  // sum.
+  const int a = (int)((uintptr_t)src & 15);
+  const uint4* s4 = reinterpret_cast<const uint4*>(src - a);
+  const int nchunk = (K + 15) >> 4;
+  for (int j = threadIdx.x; j < nchunk; j += blockDim.x) {
+    const int end = min(16 * j + 16, K);  // row bytes [16j, end) are real
+    const uint4 lo = __ldg(s4 + j);
+    uint4 hi = make_uint4(0u, 0u, 0u, 0u);
+    if (a != 0 && end + a > 16 * (j + 1)) hi = __ldg(s4 + j + 1);
+    const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+    const int q = a >> 2, sh = 8 * (a & 3);
+    uint32_t o[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      // w[k + q] and w[k + q + 1] with a uniform q in 0..3
+      const uint32_t x0 = q == 0 ? w[k] : q == 1 ? w[k + 1] : q == 2 ? w[k + 2] : w[k + 3];
+      const uint32_t x1 = q == 0 ? w[k + 1] : q == 1 ? w[k + 2] : q == 2 ? w[k + 3] : w[k + 4];
+      o[k] = __funnelshift_r(x0, x1, sh);
+    }
+    if (dst) reinterpret_cast<uint4*>(dst)[j] = make_uint4(o[0], o[1], o[2], o[3]);
+    if (rowsum) {
+      const int nv = end - 16 * j;  // real bytes in this chunk (1..16)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int keep = min(max(nv - 4 * k, 0), 4);
+        const uint32_t msk = keep == 4 ? 0xFFFFFFFFu : ((1u << (8 * keep)) - 1u);
+        s = __dp4a((int)(o[k] & msk), 0x01010101, s);
+      }
+    }
   }
   if (rowsum) {
     for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
