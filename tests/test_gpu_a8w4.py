@@ -143,9 +143,11 @@ def test_gemv_shapes(lib, N, K, bias, clamp):
     _check_a8w4(lib, w, ldy_pad=2)
 
 
+# (64, 256, 320) and (40, 128, 448) take 5 and 7 split-K ranks, whose last
+# rank owns fewer rows of the tile (24 of 26, 14 of 19) in the reduction.
 @pytest.mark.parametrize("M,N,K", [(2, 64, 64), (9, 300, 1024), (17, 1000, 4096), (128, 256, 4096),
                                    (129, 520, 384), (200, 132, 128), (3, 4096, 8192),
-                                   (256, 8, 2048), (5, 96, 96)])
+                                   (256, 8, 2048), (5, 96, 96), (64, 256, 320), (40, 128, 448)])
 def test_a8w4_gemm_shapes(lib, M, N, K):
     w = workloads.a8w4(M, N, K, seed=M * 31 + N + K, clamp=(-np.inf, np.inf), ldx=K + 1)
     _check_a8w4(lib, w, ldy_pad=1)
@@ -286,7 +288,8 @@ def test_a8w4_actblock_full_size_128x4096x4096(lib):
 
 
 @pytest.mark.parametrize("M,N,K", [(2, 64, 64), (9, 300, 1024), (17, 1000, 4096),
-                                   (129, 520, 384), (200, 132, 128), (3, 4096, 8192)])
+                                   (129, 520, 384), (200, 132, 128), (3, 4096, 8192),
+                                   (40, 128, 448)])
 def test_a8w4_actblock_gemm_shapes(lib, M, N, K):
     w = workloads.a8w4(M, N, K, seed=M * 17 + N + K, clamp=(-np.inf, np.inf), ldx=K + 1)
     # blocks of magnitudes 10^-2 .. 10^0 (a 1000x spread); with a 10^5 spread
@@ -359,7 +362,8 @@ def test_a8w4_asym_full_size_128x4096x4096(lib):
 
 
 @pytest.mark.parametrize("M,N,K", [(2, 64, 64), (9, 300, 1024), (17, 1000, 4096),
-                                   (129, 520, 384), (200, 132, 128), (3, 4096, 8192)])
+                                   (129, 520, 384), (200, 132, 128), (3, 4096, 8192),
+                                   (40, 128, 448)])
 def test_a8w4_asym_gemm_shapes(lib, M, N, K):
     w = workloads.a8w4(M, N, K, seed=M * 19 + N + K, clamp=(-np.inf, np.inf), ldx=K + 1)
     _check_asym(lib, w, _asym_zeros(w, M + N + K))
