@@ -256,6 +256,20 @@ def test_conv_56x56x64_packed_weights_bit_exact(lib, x_offset):
     run_conv(lib, workloads.int8_conv_56x56x64_3x3(), packed=True, x_offset=x_offset)
 
 
+def test_conv_more_tiles_than_sms(lib):
+    # 12 x 40 x 40 output pixels = 150 row tiles of 128 on a 148-SM grid: some
+    # CTAs run two tiles, so the stage ring and the two TMEM accumulators wrap
+    # across tiles
+    w = workloads.int8_conv(12, 40, 40, 16, 8, 3, 3, (1, 1), (1, 1), seed=4411)
+    run_conv(lib, w, packed=True)
+
+
+def test_gemm_one_cta_more_tiles_than_sms(lib):
+    # M <= 128: the one-CTA kernel; 149 column tiles of 256 on 148 CTAs
+    w = workloads.int8_gemm(64, 38000, 64, seed=4412, per_channel=True)
+    check_gemm(lib, w)
+
+
 @pytest.mark.parametrize("Nb,H,W,Cin,Cout,KH,KW,s,p", [
     (2, 17, 19, 32, 96, 3, 3, 1, 1), (1, 40, 33, 16, 300, 5, 5, 2, 2), (3, 9, 9, 48, 40, 1, 3, 1, 0),
     (1, 12, 12, 3, 8, 7, 7, 2, 3), (1, 300, 3, 64, 64, 3, 3, 1, 1)])
