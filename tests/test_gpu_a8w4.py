@@ -228,7 +228,11 @@ def test_gemv_bf16_scales_full_size_1x14336x4096(lib):
 
 
 @pytest.mark.parametrize("M,N,K", [
-    (1, 300, 1024),      # streaming GEMV
+    (1, 300, 1024),      # streaming GEMV, one group per lane
+    (1, 300, 1536),      # streaming GEMV, 2 groups per lane (48 of 64 slots live), split rows
+    (1, 5000, 2048),     # streaming GEMV, 2 groups per lane, whole and split rows
+    (1, 777, 3072),      # streaming GEMV, 4 groups per lane (96 of 128 slots live)
+    (1, 1111, 8192),     # streaming GEMV, 8 groups per lane
     (1, 1000, 2080),     # plain GEMV (K % 128 != 0)
     (1, 17, 12288),      # plain GEMV (K > 8192)
     (9, 300, 1024),      # tensor cores
