@@ -26,7 +26,9 @@
 //     exact byte image the tensor cores read: for every 128-row tile and
 //     every 64-wide K block, 128 rows of 128 bytes with the 16-byte chunks of
 //     row r permuted by r % 8 (the 128-byte swizzle).  One stage of the GEMM
-//     is then one contiguous 16 KiB bulk copy.
+//     is then one contiguous 16 KiB bulk copy.  Launched as a programmatic
+//     dependent of the previous work in the stream (it waits for it on the
+//     device before reading x).
 //  2. a8w4_tc_kernel (programmatic dependent launch after 1) computes a tile
 //     of 128 weight rows (MMA M, TMEM lanes) x 128 activation rows (MMA N,
 //     TMEM columns) over a K range; the K ranges of one tile form a cluster
@@ -347,6 +349,9 @@ __global__ void __launch_bounds__(QT) a8w4_quant_tiles_kernel(QuantArgs a, int R
   // the GEMM grid may start its prologue now; it waits for this grid before
   // it reads anything written here
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // This grid is itself a programmatic dependent of the work before it in
+  // the stream: x is read and the workspace written only once that is done.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   __shared__ float red[2][QT / 32];
   const int T = QT / R;
   const int sub = threadIdx.x / T, t = threadIdx.x - sub * T;
@@ -946,8 +951,20 @@ TcPlan plan_tc(int64_t M, int N, int K, int sms) {
 
 template <int MODE, bool CONV>
 int launch_quant(const QuantArgs& qa, int grid, int R, cudaStream_t st) {
-  a8w4_quant_tiles_kernel<MODE, CONV><<<grid, QT, 0, st>>>(qa, R);
-  return launch_status();
+  // programmatic dependent launch: the CTAs are scheduled as the previous
+  // kernel in the stream drains and wait for it on the device
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(QT);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, a8w4_quant_tiles_kernel<MODE, CONV>, qa, R) == cudaSuccess
+             ? QG_OK
+             : QG_ERR_CUDA;
 }
 
 }  // namespace
