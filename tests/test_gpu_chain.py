@@ -76,11 +76,12 @@ def test_int8_conv_chain_ping_pong(lib):
     np.testing.assert_array_equal(bufs[LINKS % 2].cpu().numpy(), x)
 
 
-@pytest.mark.parametrize("M,K", [(100, 96), (100, 100), (200, 100)])
+@pytest.mark.parametrize("M,K", [(100, 96), (100, 100), (200, 100), (300, 100)])
 def test_int8_gemm_chain_ping_pong(lib, M, K):
     # N = K: C feeds the next call as A.  (100, 96): one-CTA kernel, A read
-    # in place; (100, 100): row pitch 100 bytes, so each call stages A first;
-    # (200, 100): the CTA-pair kernel after the staging pass.
+    # in place; (100, 100) and (200, 100): row pitch 100 bytes, so each call
+    # stages A first, then the one-CTA kernel (one wave of tiles); (300, 100):
+    # the CTA-pair kernel after the staging pass.
     w = workloads.int8_gemm(M, K, K, seed=3200 + M + K, per_channel=True, ratio_scale=0.05,
                             out_zp=2)
     bias = _dev(w["bias"])
@@ -123,3 +124,57 @@ def test_a8w4_chain_ring(lib, M, K, gain):
         assert np.std(x_in) > 0.12 and np.mean(np.abs(x_in) >= 6.0) < 0.1, "chain degenerate"
         y_ref = oracle.qgemm_a8w4_f32(x_in, w["qw"], w["sw"], w["bias"], -6.0, 6.0)[0]
         assert_a8w4_close(y_gpu, y_ref, f"a8w4 chain {M}x{K}x{K} link -{k}")
+
+
+def test_inputs_written_by_a_preceding_torch_kernel(lib):
+    # Each call's input is written by a torch copy kernel launched right
+    # before it on the same stream (a grid that does not signal dependents
+    # early): the A8W4 quantization grid, the INT8 staging pass and the
+    # implicit-GEMM conv must still read the new values.
+    w = workloads.a8w4(64, 384, 1024, seed=3401, clamp=(-6.0, 6.0))
+    packed = lib.pack_w4_g32(_dev(w["qw"]), _dev(w["sw"]))
+    bias = _dev(w["bias"])
+    srcs = [_dev((w["x"] * s).astype(np.float32)) for s in (0.5, 1.0, 2.0)]
+    x = torch.empty_like(srcs[0])
+    ys = [torch.empty((64, 384), dtype=torch.float32, device="cuda") for _ in srcs]
+    for src, y in zip(srcs, ys):
+        x.copy_(src)
+        lib.qgemm_a8w4_f32(x, packed, 384, bias, -6.0, 6.0, y)
+    torch.cuda.synchronize()
+    for s, y in zip((0.5, 1.0, 2.0), ys):
+        x_in = (w["x"] * s).astype(np.float32)
+        y_ref = oracle.qgemm_a8w4_f32(x_in, w["qw"], w["sw"], w["bias"], -6.0, 6.0)[0]
+        assert_a8w4_close(y.cpu().numpy(), y_ref, f"a8w4 after torch copy, scale {s}")
+
+    g = workloads.int8_gemm(300, 96, 100, seed=3402, per_channel=True, ratio_scale=0.05, out_zp=2)
+    rq, m0, sh = _requant(lib, g["ratio"], g["za"], g["zb"], _dev(g["bias"]), g["out_zp"], -128, 127)
+    pb = lib.qgemm_pack_b_s8(_dev(g["B"]))
+    rng = np.random.default_rng(3403)
+    a_list = [rng.integers(-128, 128, size=g["A"].shape, dtype=np.int8) for _ in range(3)]
+    a = torch.empty((300, 100), dtype=torch.int8, device="cuda")
+    cs = [torch.empty((300, 96), dtype=torch.int8, device="cuda") for _ in a_list]
+    for a_host, c in zip(a_list, cs):
+        a.copy_(_dev(a_host))
+        lib.qgemm_s8s8_requant_packed(a, pb, 96, c, rq, K=100)
+    torch.cuda.synchronize()
+    for a_host, c in zip(a_list, cs):
+        ref, _ = oracle.qgemm_s8s8_requant(a_host, g["B"], g["za"], g["zb"], g["bias"], m0, sh,
+                                          g["out_zp"], -128, 127)
+        np.testing.assert_array_equal(c.cpu().numpy(), ref)
+
+    v = workloads.int8_conv(1, 12, 10, 16, 8, 3, 3, (1, 1), (1, 1), seed=3404, relu=False)
+    rq, m0, sh = _requant(lib, v["ratio"], v["za"], 0, _dev(v["bias"]), v["out_zp"], -128, 127)
+    pw = lib.qconv2d_s8_pack_w(_dev(v["w"]))
+    x_list = [rng.integers(-128, 128, size=v["x"].shape, dtype=np.int8) for _ in range(3)]
+    xc = torch.empty(v["x"].shape, dtype=torch.int8, device="cuda")
+    outs = []
+    for x_host in x_list:
+        xc.copy_(_dev(x_host))
+        o = torch.empty((1, 12, 10, 8), dtype=torch.int8, device="cuda")
+        lib.qconv2d_s8_im2col_packed(xc, pw, v["w"].shape, o, rq, v["stride"], v["pad"])
+        outs.append(o)
+    torch.cuda.synchronize()
+    for x_host, o in zip(x_list, outs):
+        ref, _ = oracle.qconv2d_s8(x_host, v["w"], v["stride"], v["pad"], v["za"], v["bias"], m0, sh,
+                                   v["out_zp"], -128, 127)
+        np.testing.assert_array_equal(o.cpu().numpy(), ref)
