@@ -296,9 +296,14 @@ struct QuantArgs {
 constexpr int QT = 256;   // threads per quantization CTA
 constexpr int QCH = 4;    // most 8-wide chunks per thread (K <= 32 * threads per row)
 
+// Tap of each 8-wide K chunk of an unrolled row (Cin % 8 == 0: a chunk lies
+// in one tap): x = input channel of its first value, y = kh << 16 | kw.  The
+// same for every row, so a CTA builds it once instead of dividing per chunk.
+constexpr int kMaxChunks = QCH * QT;  // K / 8 for the largest K (QCH chunks per thread)
+
 template <bool CONV>
 __device__ __forceinline__ void load_chunk(const QuantArgs& a, int64_t m, int c, int pn, int poh,
-                                           int pow_, float (&v)[8]) {
+                                           int pow_, const int2* tap_tab, float (&v)[8]) {
   const RowSource& s = a.src;
   if (!CONV) {
     const float* p = s.x + m * s.ldx + 8 * c;
@@ -314,9 +319,8 @@ __device__ __forceinline__ void load_chunk(const QuantArgs& a, int64_t m, int c,
     return;
   }
   if (a.vec4) {  // Cin % 8 == 0: the chunk lies in one tap
-    const int k = 8 * c;
-    const int tap = k / s.Cin, ci = k - tap * s.Cin;
-    const int kh = tap / s.KW, kw = tap - kh * s.KW;
+    const int2 e = tap_tab[c];
+    const int ci = e.x, kh = e.y >> 16, kw = e.y & 0xFFFF;
     const int ih = poh * s.sh + kh - s.ph, iw = pow_ * s.sw + kw - s.pw;
     if (ih < 0 || ih >= s.H || iw < 0 || iw >= s.W) {
 #pragma unroll
@@ -349,10 +353,8 @@ __global__ void __launch_bounds__(QT) a8w4_quant_tiles_kernel(QuantArgs a, int R
   // the GEMM grid may start its prologue now; it waits for this grid before
   // it reads anything written here
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  // This grid is itself a programmatic dependent of the work before it in
-  // the stream: x is read and the workspace written only once that is done.
-  asm volatile("griddepcontrol.wait;" ::: "memory");
   __shared__ float red[2][QT / 32];
+  __shared__ int2 tap_tab[CONV ? kMaxChunks : 1];
   const int T = QT / R;
   const int sub = threadIdx.x / T, t = threadIdx.x - sub * T;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -360,19 +362,31 @@ __global__ void __launch_bounds__(QT) a8w4_quant_tiles_kernel(QuantArgs a, int R
   const int K = a.K, G = K >> 5, nchunk = K >> 3, nkb = K >> 6;
   const bool live = m < a.M;
   int pn = 0, poh = 0, pow_ = 0;
-  if (CONV && live) {
-    pow_ = (int)(m % a.src.OW);
-    const int64_t tt = m / a.src.OW;
-    poh = (int)(tt % a.src.OH);
-    pn = (int)(tt / a.src.OH);
+  if (CONV && live) {  // m < Mpad <= INT32_MAX: 32-bit divisions
+    const int mi = (int)m;
+    const int tt = mi / a.src.OW;
+    pow_ = mi - tt * a.src.OW;
+    pn = tt / a.src.OH;
+    poh = tt - pn * a.src.OH;
   }
+  if (CONV && a.vec4) {
+    for (int c = threadIdx.x; c < nchunk; c += QT) {
+      const int k = 8 * c;
+      const int tap = k / a.src.Cin, kh = tap / a.src.KW;
+      tap_tab[c] = make_int2(k - tap * a.src.Cin, (kh << 16) | (tap - kh * a.src.KW));
+    }
+    __syncthreads();
+  }
+  // This grid is itself a programmatic dependent of the work before it in
+  // the stream: x is read and the workspace written only once that is done.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   float v[QCH][8];
   float mn = 0.0f, mx = 0.0f;  // min(0, .), max(0, .); mx is max|x| when symmetric
 #pragma unroll
   for (int i = 0; i < QCH; ++i) {
     const int c = t + i * T;
     if (live && c < nchunk) {
-      load_chunk<CONV>(a, m, c, pn, poh, pow_, v[i]);
+      load_chunk<CONV>(a, m, c, pn, poh, pow_, tap_tab, v[i]);
     } else {
 #pragma unroll
       for (int e = 0; e < 8; ++e) v[i][e] = 0.0f;
