@@ -92,6 +92,8 @@ def test_dynconv_56x56x64_3x3(lib, symmetric):
     (1, 4, 4, 128, 33, 4, 4, (1, 1), (0, 0)),     # kernel the size of the image: P = 1
     (1, 7, 7, 32, 9, 3, 3, (3, 3), (2, 2)),       # pixels with mostly pad taps
     (1, 6, 6, 2048, 8, 3, 3, (1, 1), (1, 1)),     # K = 18432
+    (1, 9, 9, 4, 10, 4, 4, (1, 1), (1, 1)),       # Cin % 8 != 0 on tensor cores (K = 64)
+    (2, 8, 7, 12, 6, 4, 4, (1, 1), (2, 1)),       # Cin % 8 != 0, K = 192, uneven pads
 ])
 def test_dynconv_shapes(lib, symmetric, Nb, H, W, Cin, Cout, KH, KW, stride, pad):
     w = workloads.a8w4_conv_f32(Nb, H, W, Cin, Cout, KH, KW, stride, pad,
